@@ -1,0 +1,230 @@
+/*
+ * vkv.h -- chunk attention over a segmented KV cache, native on NVIDIA B200 (sm_100a).
+ *
+ * The queries of the current latent-frame chunk of an autoregressive video
+ * diffusion model attend over a KV cache made of sink frames, history and a
+ * local window.  Three cache modes are served by one attention entry point:
+ *
+ *   VKV_MODE_SEGMENTS      the cache is split into a local branch (sink + current
+ *                          frames) and a history branch; each branch emits its own
+ *                          partial output and log-sum-exp (LSE), and the two are
+ *                          merged exactly by online softmax.
+ *                          (ISPA summary, gist.science 2607.00712, section 2 step 1
+ *                          "Dual-Stream Warmup": decomposable attention tracked by
+ *                          LSE; contribution 2: online softmax.)
+ *   VKV_MODE_BLOCK_SPARSE  every query attends to a per-head list of persistent
+ *                          blocks plus the top-K blocks of the local window picked
+ *                          for its 64-query block, in one softmax.
+ *                          (Sparse Forcing summary, gist.science 2604.21221,
+ *                          section 2 component 3 "PBSA".)
+ *   VKV_MODE_RAGGED        each (batch, head) sequence has its own cache length;
+ *                          the caches are stored flattened with boundary offsets,
+ *                          without padding.
+ *                          (Pyramid Forcing summary, gist.science 2605.13111,
+ *                          methodology section 3 "Ragged-Cache Attention".)
+ *
+ * Conventions for every entry point:
+ *   - All tensors are device memory allocated and owned by the caller.  The
+ *     library allocates no device memory; it keeps no state between calls
+ *     except one-time per-device set-up (kernel attributes, driver entry point).
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream);
+ *     the library never synchronises.  Host arrays passed in are read during
+ *     the call only.
+ *   - bf16 tensors are described by vkv_tensor: a pointer to element 0 and the
+ *     element strides of the batch, token and head axes; the feature axis (d)
+ *     is contiguous.  Pointers must be 16-byte aligned and the three strides
+ *     multiples of 8 elements (the tensor-memory-accelerator rule), else
+ *     VKV_ERR_ALIGN.
+ *   - The return value reports host-side validation and launch errors.  Errors
+ *     found on the device (an index outside the cache, non-monotone offsets, a
+ *     pipeline wait that exceeded its time limit) are written to the optional
+ *     device word `err_word` (first error wins; 0 = no error) and the affected
+ *     work is skipped; nothing traps.  Without `err_word` they go unreported.
+ *   - Thread-safe; calls on different streams may run concurrently, provided
+ *     their output buffers do not overlap.
+ */
+#ifndef VKV_H_
+#define VKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; NULL selects the legacy default stream. */
+typedef struct CUstream_st* vkv_stream_t;
+
+typedef enum {
+  VKV_OK = 0,
+  VKV_ERR_NULL = 1,        /* a required pointer is NULL                                  */
+  VKV_ERR_SHAPE = 2,       /* a size is out of range or two sizes disagree                */
+  VKV_ERR_ALIGN = 3,       /* a pointer or stride breaks the 16-byte rule                 */
+  VKV_ERR_RANGE = 4,       /* a segment or host offset lies outside the cache             */
+  VKV_ERR_UNSUPPORTED = 5, /* valid request outside what this build implements            */
+  VKV_ERR_CUDA = 6,        /* no usable sm_100 device, or a CUDA call / launch failed     */
+  VKV_ERR_WORKSPACE = 7    /* workspace missing or smaller than the reported size         */
+} vkv_status;
+
+/* Codes written to *err_word by the device. */
+#define VKV_DEVERR_TIMEOUT 1      /* a pipeline wait ran past its limit; outputs incomplete */
+#define VKV_DEVERR_BAD_INDEX 2    /* a block index lies outside the cache or the window     */
+#define VKV_DEVERR_BAD_OFFSETS 3  /* cu_seqlens decreasing or past the flattened cache      */
+
+typedef enum {
+  VKV_MODE_SEGMENTS = 0,
+  VKV_MODE_BLOCK_SPARSE = 1,
+  VKV_MODE_RAGGED = 2
+} vkv_mode;
+
+/* Cache token rows [start, start + len) of one batch/head. */
+typedef struct {
+  int32_t start;
+  int32_t len;
+} vkv_segment;
+
+/* A bf16 tensor [B, L, H, d] with element strides sb, st, sh; d contiguous.
+ * For the flattened ragged cache [rows, d] only `ptr` and `st` (row stride) are read. */
+typedef struct {
+  void* ptr;
+  int64_t sb;
+  int64_t st;
+  int64_t sh;
+} vkv_tensor;
+
+#define VKV_MAX_BRANCHES 2
+#define VKV_MAX_SEGMENTS 8   /* per branch */
+
+typedef struct {
+  int32_t mode;  /* vkv_mode */
+  int32_t B;     /* batch                                                     */
+  int32_t H;     /* heads (queries and keys have the same head count)         */
+  int32_t Lq;    /* query rows per batch and head (the current chunk)         */
+  int32_t Lkv;   /* cache rows per batch and head; RAGGED: rows of the flat cache */
+  int32_t d;     /* head dimension: 64 or 128                                 */
+  float scale;   /* softmax scale applied to q.k (usually 1/sqrt(d))          */
+  vkv_tensor q;  /* [B, Lq, H, d]                                             */
+  vkv_tensor k;  /* SEGMENTS / BLOCK_SPARSE: [B, Lkv, H, d]; RAGGED: [Lkv, d] */
+  vkv_tensor v;  /* same layout as k                                          */
+
+  /* VKV_MODE_SEGMENTS: n_branches in {1, 2}; segs[b] is a HOST array of
+   * n_segs[b] <= VKV_MAX_SEGMENTS segments; a branch is the union of its
+   * segments (which must not overlap).  A branch may be empty (O = 0, LSE = -inf). */
+  int32_t n_branches;
+  const vkv_segment* segs[VKV_MAX_BRANCHES];
+  int32_t n_segs[VKV_MAX_BRANCHES];
+
+  /* VKV_MODE_BLOCK_SPARSE: the cache is cut into blocks of `block` (= 64) rows.
+   * persist_idx: DEVICE int32 [B*H][n_persist], absolute block ids attended by every query.
+   * sel_idx:     DEVICE int32 [B*H][ceil(Lq/block)][topk], window-relative block ids
+   *              (0 <= id < n_win_blk), distinct within a row, ascending, as written by
+   *              vkv_block_select; query block j = query rows [j*block, (j+1)*block).
+   * The window is blocks [window_blk0, window_blk0 + n_win_blk); persistent blocks
+   * must lie outside it.  Requires n_persist + min(n_win_blk, 4*topk) <= 288
+   * (one unit holds up to four query blocks; its block list has at most 288 entries). */
+  int32_t block;
+  const int32_t* persist_idx;
+  int32_t n_persist;
+  const int32_t* sel_idx;
+  int32_t topk;
+  int32_t window_blk0;
+  int32_t n_win_blk;
+
+  /* VKV_MODE_RAGGED: sequence s = b*H + h reads flat rows [cu[s], cu[s+1]).
+   * cu_seqlens: DEVICE int32 [B*H + 1] (authoritative, checked on the device).
+   * cu_seqlens_host: optional HOST copy; when given it is validated on the host and
+   * used to balance work across SMs (longest sequences first). */
+  const int32_t* cu_seqlens;
+  const int32_t* cu_seqlens_host;
+
+  /* Outputs.  o[b] bf16 [B, Lq, H, d] and lse[b] fp32 [B, H, Lq] (contiguous) per
+   * branch; BLOCK_SPARSE and RAGGED write branch 0 only.  o_merged / lse_merged
+   * (SEGMENTS with 2 branches, optional: ptr NULL = skip) receive the exact
+   * LSE merge of the two branches, i.e. attention over their union.
+   * LSE is the natural log of sum_j exp(scale * q.k_j). */
+  vkv_tensor o[VKV_MAX_BRANCHES];
+  float* lse[VKV_MAX_BRANCHES];
+  vkv_tensor o_merged;
+  float* lse_merged;
+
+  int32_t* err_word; /* optional DEVICE int32; see VKV_DEVERR_* */
+} vkv_attn_args;
+
+/*
+ * vkv_chunk_attn -- softmax attention of the chunk's queries over the cache.
+ *
+ * For each (batch b, head h, query row i) and the key set J selected by the mode:
+ *   s_j = scale * <q_i, k_j>,  O_i = sum_j softmax(s)_j v_j,  LSE_i = ln sum_j exp(s_j).
+ * Rows of the cache up to 127 past the end of a segment (SEGMENTS, RAGGED) are
+ * read but masked; where they lie inside the cache they must hold finite values.
+ * Sources: ISPA summary section 2 step 1; Sparse Forcing summary section 2
+ * component 3; Pyramid Forcing summary methodology section 3.
+ */
+vkv_status vkv_chunk_attn(const vkv_attn_args* args, vkv_stream_t stream);
+
+/*
+ * Block selection for VKV_MODE_BLOCK_SPARSE (Sparse Forcing summary, section 2
+ * component 2 "Blockified Compression": one representative token per block for
+ * coarse scoring; component 3: top-K window blocks).
+ *
+ * Each query block j (rows [j*block, (j+1)*block) of q, the last one possibly
+ * shorter) and each window block w (cache rows [(window_blk0+w)*block, +block))
+ * is reduced to the fp32 mean of its rows; score(j, w) = <qbar_j, kbar_w>
+ * (no softmax scale: a positive factor does not change the ranking).  For every
+ * (batch, head, j) the `topk` highest-scoring window blocks are written to
+ * out_idx [B*H][ceil(Lq/block)][topk] in ascending order; equal scores rank
+ * the lower block id first.  out_scores [B*H][ceil(Lq/block)][n_win_blk]
+ * (optional, fp32) receives every score.
+ * `workspace` is DEVICE scratch of at least vkv_block_select_workspace_size()
+ * bytes, 256-byte aligned, owned by the caller; its contents need no
+ * initialisation and are dead after the call.
+ */
+typedef struct {
+  int32_t B, H, d, block; /* d in {64, 128}; block = 64                       */
+  int32_t Lq;             /* query rows                                        */
+  int32_t Lkv;            /* cache rows (window blocks must lie inside)        */
+  int32_t window_blk0;    /* first window block                                */
+  int32_t n_win_blk;      /* window blocks, 1..1024                            */
+  int32_t topk;           /* 1..n_win_blk                                      */
+  vkv_tensor q;           /* [B, Lq, H, d]                                     */
+  vkv_tensor k;           /* [B, Lkv, H, d]                                    */
+  int32_t* out_idx;
+  float* out_scores;
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* err_word;      /* optional DEVICE int32                             */
+} vkv_select_args;
+
+size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,
+                                       int32_t block, int32_t d);
+vkv_status vkv_block_select(const vkv_select_args* args, vkv_stream_t stream);
+
+/*
+ * vkv_lse_merge -- exact recombination of two partial attentions over disjoint
+ * key sets (ISPA summary, section 2 step 1 and contribution 2):
+ *   M = max(lse_a, lse_b),  w_x = exp(lse_x - M),
+ *   O = (w_a O_a + w_b O_b) / (w_a + w_b),  LSE = M + ln(w_a + w_b).
+ * Rows where both LSEs are -inf give O = 0 and LSE = -inf.
+ * o_a, o_b, o_out: bf16 [B, Lq, H, d] (vkv_tensor strides); lse_*: fp32 [B, H, Lq]
+ * contiguous.  o_out may alias o_a or o_b only if it is the same tensor exactly.
+ */
+vkv_status vkv_lse_merge(vkv_tensor o_a, const float* lse_a, vkv_tensor o_b, const float* lse_b,
+                         vkv_tensor o_out, float* lse_out, int32_t B, int32_t H, int32_t Lq,
+                         int32_t d, vkv_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* vkv_status_string(vkv_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t vkv_version(void);
+
+/* sizeof() of the ABI structs, for bindings to check their layout:
+ * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment; -1 otherwise. */
+int32_t vkv_abi_sizeof(int32_t which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VKV_H_ */

@@ -1,0 +1,361 @@
+// vkv_chunk_attn: argument checks, work schedule, TMA descriptors, launch.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <functional>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <queue>
+#include <string>
+#include <vector>
+
+#include "vkv_attn_kernel.cuh"
+
+namespace vkv {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// schedule: units of one or two 128-row query tiles, balanced over the SMs
+// ---------------------------------------------------------------------------
+struct Plan {
+  int n_ctas = 0;
+  std::vector<int> cta_begin;
+  std::vector<uint32_t> units;
+};
+
+struct Cand {
+  uint32_t code;
+  double cost;
+};
+
+double single_tile_cost() {
+  static double c = [] {
+    const char* e = std::getenv("VKV_SINGLE_COST");
+    double v = e ? std::atof(e) : 0.0;
+    return (v > 0.05 && v <= 1.0) ? v : 0.6;
+  }();
+  return c;
+}
+
+// Longest-processing-time assignment of `units` to `g` CTAs; returns makespan.
+double lpt(std::vector<Cand>& units, int g, Plan* out) {
+  std::stable_sort(units.begin(), units.end(), [](const Cand& a, const Cand& b) { return a.cost > b.cost; });
+  using E = std::pair<double, int>;
+  std::priority_queue<E, std::vector<E>, std::greater<E>> heap;
+  for (int c = 0; c < g; ++c) heap.push({0.0, c});
+  std::vector<std::vector<uint32_t>> per(out ? g : 0);
+  double mk = 0;
+  for (const Cand& u : units) {
+    E e = heap.top();
+    heap.pop();
+    e.first += u.cost;
+    mk = std::max(mk, e.first);
+    if (out) per[e.second].push_back(u.code);
+    heap.push(e);
+  }
+  if (out) {
+    out->n_ctas = g;
+    out->cta_begin.assign(g + 1, 0);
+    out->units.clear();
+    for (int c = 0; c < g; ++c) {
+      out->cta_begin[c] = (int)out->units.size();
+      out->units.insert(out->units.end(), per[c].begin(), per[c].end());
+    }
+    out->cta_begin[g] = (int)out->units.size();
+  }
+  return mk;
+}
+
+inline uint32_t unit_code(int s, int tile0, bool two) {
+  return ((uint32_t)s << 14) | (two ? (1u << 13) : 0u) | (uint32_t)tile0;
+}
+
+// pair_cost[s] / single_cost[s]: estimated cost of a 2-tile / 1-tile unit of sequence s.
+bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
+               const std::vector<double>& one_cost, int n_sm, Plan* plan) {
+  // sequences by decreasing pair cost: their pairs are split first
+  std::vector<int> order(n_seq);
+  for (int s = 0; s < n_seq; ++s) order[s] = s;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return pair_cost[a] > pair_cost[b]; });
+  const int pairs_per_seq = T / 2;
+  const long long n_pairs = (long long)n_seq * pairs_per_seq;
+  auto build = [&](long long n_split, std::vector<Cand>& u) {
+    u.clear();
+    long long split = 0;
+    for (int oi = 0; oi < n_seq; ++oi) {
+      const int s = order[oi];
+      for (int i = 0; i < pairs_per_seq; ++i) {
+        if (split < n_split) {
+          u.push_back({unit_code(s, 2 * i, false), one_cost[s]});
+          u.push_back({unit_code(s, 2 * i + 1, false), one_cost[s]});
+          ++split;
+        } else {
+          u.push_back({unit_code(s, 2 * i, true), pair_cost[s]});
+        }
+      }
+      if (T & 1) u.push_back({unit_code(s, T - 1, false), one_cost[s]});
+    }
+  };
+  std::vector<long long> cands = {0};
+  for (int k = 1; k <= 16; ++k) cands.push_back((long long)k * n_sm / 4);
+  cands.push_back(n_pairs);
+  double best = 1e300;
+  long long best_split = 0;
+  std::vector<Cand> u;
+  for (long long c : cands) {
+    if (c > n_pairs) continue;
+    build(c, u);
+    if ((long long)u.size() > kMaxUnits) continue;
+    const int g = (int)std::min<long long>(n_sm, (long long)u.size());
+    const double mk = lpt(u, g, nullptr);
+    if (mk < best * 0.999) {
+      best = mk;
+      best_split = c;
+    }
+  }
+  if (best >= 1e299) return false;
+  build(best_split, u);
+  const int g = (int)std::min<long long>(n_sm, (long long)u.size());
+  lpt(u, g, plan);
+  return true;
+}
+
+std::mutex g_plan_mu;
+std::map<std::string, std::shared_ptr<Plan>> g_plans;
+
+std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T,
+                               const std::vector<double>& pc, const std::vector<double>& oc, int n_sm) {
+  {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    auto it = g_plans.find(key);
+    if (it != g_plans.end()) return it->second;
+  }
+  auto plan = std::make_shared<Plan>();
+  if (!make_plan(n_seq, T, pc, oc, n_sm, plan.get())) return nullptr;
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  if (g_plans.size() > 256) g_plans.clear();
+  g_plans[key] = plan;
+  return plan;
+}
+
+bool set_smem_attr(int dev, int D) {
+  static std::mutex mu;
+  static unsigned long long done[2] = {0, 0};
+  std::lock_guard<std::mutex> lk(mu);
+  const int k = (D == 128) ? 0 : 1;
+  if (done[k] & (1ull << dev)) return true;
+  const void* fn = (D == 128) ? reinterpret_cast<const void*>(chunk_attn_kernel<128>)
+                              : reinterpret_cast<const void*>(chunk_attn_kernel<64>);
+  const int smem = (D == 128) ? AttnCfg<128>::SMEM_BYTES : AttnCfg<64>::SMEM_BYTES;
+  cudaFuncAttributes fa;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  // the warpgroup register split needs every register the launch provides
+  if (fa.numRegs < kRegsLaunchNeeded) return false;
+  done[k] |= 1ull << dev;
+  return true;
+}
+
+bool dims_ok_for_tma(const vkv_tensor& t, int B, int L, int H, int d) {
+  const long long lim = 1ll << 39;  // strides below 2^40 bytes
+  return std::llabs(t.sb) < lim && std::llabs(t.st) < lim && std::llabs(t.sh) < lim && B > 0 && L > 0 &&
+         H > 0 && d > 0 && t.st > 0 && (H == 1 || t.sh > 0) && (B == 1 || t.sb > 0);
+}
+
+// (d, H, L, B) map with strides (sh, st, sb); size-1 axes get a natural stride.
+bool encode_bhld(CUtensorMap* tm, const vkv_tensor& t, int B, int L, int H, int d, uint32_t box_rows) {
+  const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)L, (uint64_t)B};
+  const uint64_t sh = (H == 1) ? (uint64_t)d * 2 : (uint64_t)t.sh * 2;
+  const uint64_t st = (uint64_t)t.st * 2;
+  const uint64_t sb = (B == 1) ? st * (uint64_t)L : (uint64_t)t.sb * 2;
+  const uint64_t strides[3] = {sh, st, sb};
+  const uint32_t box[4] = {64, 1, box_rows, 1};
+  return encode_tmap_bf16_4d(tm, t.ptr, dims, strides, box);
+}
+
+bool encode_flat(CUtensorMap* tm, const vkv_tensor& t, int rows, int d) {
+  const uint64_t dims[4] = {(uint64_t)d, 1, (uint64_t)rows, 1};
+  const uint64_t st = (uint64_t)t.st * 2;
+  const uint64_t strides[3] = {(uint64_t)d * 2, st, st * (uint64_t)rows};
+  const uint32_t box[4] = {64, 1, 64, 1};
+  return encode_tmap_bf16_4d(tm, t.ptr, dims, strides, box);
+}
+
+bool out_ok(const vkv_tensor& t) {
+  return t.ptr != nullptr && tensor_aligned(t);
+}
+
+}  // namespace
+
+}  // namespace vkv
+
+using namespace vkv;
+
+extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream) {
+  if (!a) return VKV_ERR_NULL;
+  const int mode = a->mode;
+  if (mode != VKV_MODE_SEGMENTS && mode != VKV_MODE_BLOCK_SPARSE && mode != VKV_MODE_RAGGED)
+    return VKV_ERR_UNSUPPORTED;
+  if (a->d != 64 && a->d != 128) return VKV_ERR_UNSUPPORTED;
+  if (a->B <= 0 || a->H <= 0 || a->Lq <= 0 || a->Lkv < 0) return VKV_ERR_SHAPE;
+  if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return VKV_ERR_SHAPE;
+  const int B = a->B, H = a->H, Lq = a->Lq, Lkv = a->Lkv, d = a->d;
+  const long long n_seq = (long long)B * H;
+  const int T = (Lq + 127) / 128;
+  if (n_seq >= (1ll << 18) || T > 8192) return VKV_ERR_UNSUPPORTED;
+  if (!a->q.ptr || !a->k.ptr || !a->v.ptr) return VKV_ERR_NULL;
+  if (!tensor_aligned(a->q) || !tensor_aligned(a->k) || !tensor_aligned(a->v)) return VKV_ERR_ALIGN;
+  if (!dims_ok_for_tma(a->q, B, Lq, H, d)) return VKV_ERR_SHAPE;
+
+  auto P = std::make_unique<AttnParams>();
+  std::memset(P.get(), 0, sizeof(AttnParams));
+  P->mode = mode;
+  P->B = B;
+  P->H = H;
+  P->Lq = Lq;
+  P->Lkv = Lkv;
+  P->d = d;
+  P->scale_log2 = a->scale * 1.4426950408889634f;
+  P->err = a->err_word;
+
+  int nb = 1;
+  std::vector<double> pc(n_seq), oc(n_seq);
+  const double c1 = single_tile_cost();
+  std::string key;
+  if (mode == VKV_MODE_SEGMENTS) {
+    nb = a->n_branches;
+    if (nb < 1 || nb > 2) return VKV_ERR_SHAPE;
+    if (Lkv <= 0 || !dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d))
+      return VKV_ERR_SHAPE;
+    P->n_branches = nb;
+    int nf = 0, total = 0;
+    for (int br = 0; br < nb; ++br) {
+      const int ns = a->n_segs[br];
+      if (ns < 0 || ns > VKV_MAX_SEGMENTS) return VKV_ERR_SHAPE;
+      if (ns > 0 && !a->segs[br]) return VKV_ERR_NULL;
+      bool first = true;
+      int steps = 0;
+      for (int i = 0; i < ns; ++i) {
+        const vkv_segment sg = a->segs[br][i];
+        if (sg.start < 0 || sg.len < 0 || (long long)sg.start + sg.len > Lkv) return VKV_ERR_RANGE;
+        if (sg.len == 0) continue;
+        P->flat_start[nf] = sg.start;
+        P->flat_len[nf] = sg.len;
+        P->flat_branch[nf] = br;
+        P->flat_first[nf] = first ? 1 : 0;
+        first = false;
+        steps += (sg.len + 127) / 128;
+        ++nf;
+      }
+      P->branch_steps[br] = steps;
+      total += steps;
+    }
+    P->n_flat = nf;
+    P->total_steps = total;
+    for (long long s = 0; s < n_seq; ++s) {
+      pc[s] = total + 2.0;
+      oc[s] = c1 * (total + 2.0);
+    }
+    key = "S" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(total);
+  } else if (mode == VKV_MODE_BLOCK_SPARSE) {
+    if (a->block != 64) return VKV_ERR_UNSUPPORTED;
+    if (Lkv <= 0 || !dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d))
+      return VKV_ERR_SHAPE;
+    if (a->n_persist < 0 || a->topk < 0 || a->n_win_blk < 0 || a->window_blk0 < 0) return VKV_ERR_SHAPE;
+    if (a->n_win_blk > 1024 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
+    if ((long long)(a->window_blk0 + a->n_win_blk) * 64 > Lkv) return VKV_ERR_RANGE;
+    if (a->n_persist + std::min(a->n_win_blk, 4 * a->topk) > kMaxListEntries) return VKV_ERR_UNSUPPORTED;
+    if ((a->n_persist > 0 && !a->persist_idx) || (a->topk > 0 && !a->sel_idx)) return VKV_ERR_NULL;
+    P->n_persist = a->n_persist;
+    P->topk = a->topk;
+    P->window_blk0 = a->window_blk0;
+    P->n_win_blk = a->n_win_blk;
+    P->n_qblk = (Lq + 63) / 64;
+    P->n_blocks_total = Lkv / 64;
+    P->persist_idx = a->persist_idx;
+    P->sel_idx = a->sel_idx;
+    const double sp = (a->n_persist + std::min(a->n_win_blk, 4 * a->topk)) * 0.5 + 2.0;
+    const double s1 = (a->n_persist + std::min(a->n_win_blk, 2 * a->topk)) * 0.5 + 2.0;
+    for (long long s = 0; s < n_seq; ++s) {
+      pc[s] = sp;
+      oc[s] = c1 * s1 * (sp > 0 ? 1.0 : 1.0);
+    }
+    key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
+          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk);
+  } else {
+    if (!a->cu_seqlens) return VKV_ERR_NULL;
+    if (Lkv <= 0 || a->k.st <= 0 || a->v.st <= 0 || (a->k.st % 8) || (a->v.st % 8)) return VKV_ERR_SHAPE;
+    if (a->cu_seqlens_host) {
+      const int32_t* cu = a->cu_seqlens_host;
+      if (cu[0] < 0) return VKV_ERR_RANGE;
+      for (long long s = 0; s < n_seq; ++s)
+        if (cu[s + 1] < cu[s] || cu[s + 1] > Lkv) return VKV_ERR_RANGE;
+      key = "R" + std::to_string(n_seq) + "/" + std::to_string(T);
+      for (long long s = 0; s < n_seq; ++s) {
+        const int steps = (cu[s + 1] - cu[s] + 127) / 128;
+        pc[s] = steps + 2.0;
+        oc[s] = c1 * (steps + 2.0);
+        key += "," + std::to_string(steps);
+      }
+    } else {
+      for (long long s = 0; s < n_seq; ++s) {
+        pc[s] = 1.0;
+        oc[s] = c1;
+      }
+      key = "R" + std::to_string(n_seq) + "/" + std::to_string(T) + "/u";
+    }
+    P->cu_seqlens = a->cu_seqlens;
+  }
+  const int nout = (mode == VKV_MODE_SEGMENTS) ? nb : 1;
+  for (int br = 0; br < nout; ++br) {
+    if (!a->lse[br]) return VKV_ERR_NULL;
+    if (!out_ok(a->o[br])) return a->o[br].ptr ? VKV_ERR_ALIGN : VKV_ERR_NULL;
+    P->o[br] = reinterpret_cast<__nv_bfloat16*>(a->o[br].ptr);
+    P->o_sb[br] = a->o[br].sb;
+    P->o_st[br] = a->o[br].st;
+    P->o_sh[br] = a->o[br].sh;
+    P->lse[br] = a->lse[br];
+  }
+  if (mode == VKV_MODE_SEGMENTS && nb == 2 && a->o_merged.ptr) {
+    if (!a->lse_merged) return VKV_ERR_NULL;
+    if (!out_ok(a->o_merged)) return VKV_ERR_ALIGN;
+    P->om = reinterpret_cast<__nv_bfloat16*>(a->o_merged.ptr);
+    P->om_sb = a->o_merged.sb;
+    P->om_st = a->o_merged.st;
+    P->om_sh = a->o_merged.sh;
+    P->lsem = a->lse_merged;
+  }
+
+  int dev = 0;
+  const int n_sm = device_sm_count(&dev);
+  if (n_sm <= 0) return VKV_ERR_CUDA;
+  const int g_max = std::min(n_sm, kMaxCtas);
+  key += "@" + std::to_string(g_max) + ":" + std::to_string(c1);
+  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, g_max);
+  if (!plan) return VKV_ERR_UNSUPPORTED;
+  P->n_ctas = plan->n_ctas;
+  std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);
+  std::copy(plan->units.begin(), plan->units.end(), P->units);
+
+  if (!encode_bhld(&P->tm_q, a->q, B, Lq, H, d, 128)) return VKV_ERR_CUDA;
+  if (mode == VKV_MODE_RAGGED) {
+    if (!encode_flat(&P->tm_k, a->k, Lkv, d) || !encode_flat(&P->tm_v, a->v, Lkv, d)) return VKV_ERR_CUDA;
+  } else {
+    if (!encode_bhld(&P->tm_k, a->k, B, Lkv, H, d, 64) || !encode_bhld(&P->tm_v, a->v, B, Lkv, H, d, 64))
+      return VKV_ERR_CUDA;
+  }
+  if (!set_smem_attr(dev, d)) return VKV_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    chunk_attn_kernel<128><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
+  else
+    chunk_attn_kernel<64><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
+  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  return VKV_OK;
+}

@@ -1,0 +1,796 @@
+// Chunk attention over a segmented KV cache: the sm_100a kernel.
+//
+// One persistent CTA per SM works through a host-built list of units.  A
+// unit is one (batch, head) and one or two 128-row query tiles; it walks a
+// stream of 128-key tiles (two 64-row halves each) and keeps an online
+// softmax per query row.  The key stream depends on the mode:
+//   SEGMENTS      consecutive 128-row tiles of each segment of each branch
+//                 (ISPA summary, section 2 step 1: local and history branches,
+//                 each closed with its own output and LSE, then merged);
+//   BLOCK_SPARSE  the unit's persistent blocks, then the union of the window
+//                 blocks selected for its 64-query blocks, two blocks per tile,
+//                 with a per-query-block visibility mask (Sparse Forcing
+//                 summary, section 2 component 3 "PBSA");
+//   RAGGED        consecutive tiles of rows [cu[s], cu[s+1]) of the flattened
+//                 cache (Pyramid Forcing summary, methodology section 3).
+//
+// Warp roles (384 threads):
+//   warp 0       TMA producer: Q tiles, K/V tiles into a ring of smem slots;
+//                builds the block list in BLOCK_SPARSE mode.
+//   warp 1       MMA issuer: S_t = Q_t K^T and O_t += P_t V with tcgen05.mma,
+//                accumulators in tensor memory (TMEM); owns the TMEM allocation.
+//   warps 2-3    idle.
+//   warps 4-7    softmax + epilogue for query tile 0 (one thread per row).
+//   warps 8-11   softmax + epilogue for query tile 1.
+//
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
+// P (bf16) is written by the softmax threads to shared memory in the same
+// 128-byte-swizzled K-major layout TMA produces, and read by the PV MMA.
+// The online softmax works in log2 units (s * scale * log2 e) and rescales the
+// O accumulator only when a row maximum grows by more than 2^8; the final
+// O / l and LSE do not depend on the reference maximum.
+#pragma once
+
+#include "vkv_internal.h"
+#include "vkv_ptx.cuh"
+
+namespace vkv {
+
+template <int D>
+struct AttnCfg {
+  static constexpr int NAC = D / 64;               // 128-byte atom columns along d
+  static constexpr int ATOM = 128 * 128;            // bytes of one 128-row atom column
+  static constexpr int QT_BYTES = 128 * D * 2;      // one 128-row Q tile
+  static constexpr int P_BYTES = 128 * 128 * 2;     // one P tile (128 rows x 128 keys)
+  static constexpr int KV_BYTES = 128 * D * 2;      // one K or V tile (128 keys)
+  static constexpr int NSLOT = (D == 128) ? 3 : 6;  // K/V ring slots
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_CTL = OFF_KV + NSLOT * KV_BYTES;
+  static constexpr int SMEM_BYTES = OFF_CTL + kCtlBytes + 1024;  // + base alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TM_O = 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Control block (barriers, block list) at the end of shared memory.
+struct Ctl {
+  uint64_t full[6];
+  uint64_t empty[6];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t list_ready, list_free, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int list_count;
+  int pad_;
+  uint32_t bitmap[4][32];
+  uint32_t list[kMaxListEntries];
+};
+static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
+
+struct TileDesc {
+  int rowA, rowB;         // first cache row of each 64-row half
+  int limA, limB;         // valid columns of each half (0..64)
+  uint32_t maskA, maskB;  // per-64-query-block visibility bits of each half
+  int branch;
+  bool first;             // first tile of its branch
+};
+
+// Walks the key-tile stream of one unit; every role runs its own copy.
+struct TileIter {
+  const AttnParams* p;
+  const Ctl* ctl;
+  int k, off;        // SEGMENTS: flat segment index, row offset inside it
+  int rstart, rlen;  // RAGGED: this sequence's rows
+  int j;
+
+  __device__ __forceinline__ void init(const AttnParams* pp, const Ctl* c, int rs, int rl) {
+    p = pp;
+    ctl = c;
+    k = 0;
+    off = 0;
+    rstart = rs;
+    rlen = rl;
+    j = 0;
+  }
+
+  __device__ __forceinline__ TileDesc next() {
+    TileDesc t;
+    if (p->mode == VKV_MODE_BLOCK_SPARSE) {
+      const int n = ctl->list_count;
+      const uint32_t e0 = ctl->list[2 * j];
+      const uint32_t e1 = (2 * j + 1 < n) ? ctl->list[2 * j + 1] : (e0 & 0xFFFFFFu);
+      t.rowA = (int)(e0 & 0xFFFFFFu) * 64;
+      t.rowB = (int)(e1 & 0xFFFFFFu) * 64;
+      t.limA = 64;
+      t.limB = 64;
+      t.maskA = e0 >> 24;
+      t.maskB = e1 >> 24;
+      t.branch = 0;
+      t.first = (j == 0);
+    } else {
+      int start, len, br;
+      bool bfirst;
+      if (p->mode == VKV_MODE_RAGGED) {
+        start = rstart;
+        len = rlen;
+        br = 0;
+        bfirst = true;
+      } else {
+        start = p->flat_start[k];
+        len = p->flat_len[k];
+        br = p->flat_branch[k];
+        bfirst = p->flat_first[k] != 0;
+      }
+      const int valid = min(128, len - off);
+      t.rowA = start + off;
+      t.rowB = start + off + 64;
+      t.limA = min(64, valid);
+      t.limB = max(0, valid - 64);
+      t.maskA = 0xFu;
+      t.maskB = 0xFu;
+      t.branch = br;
+      t.first = bfirst && off == 0;
+      off += 128;
+      if (off >= len) {
+        ++k;
+        off = 0;
+      }
+    }
+    ++j;
+    return t;
+  }
+};
+
+struct UnitInfo {
+  int s;       // sequence = b*H + h
+  int b, h;
+  int tile0;   // first 128-row query tile
+  int ntiles;  // 1 or 2
+};
+
+__device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, uint32_t code) {
+  UnitInfo u;
+  u.tile0 = (int)(code & 0x1FFFu);
+  u.ntiles = ((code >> 13) & 1u) ? 2 : 1;
+  u.s = (int)(code >> 14);
+  u.b = u.s / p.H;
+  u.h = u.s - u.b * p.H;
+  return u;
+}
+
+__device__ __forceinline__ void set_err(const AttnParams& p, int code) {
+  if (p.err) atomicCAS(p.err, 0, code);
+}
+
+// Rows [start, start+len) of a ragged sequence, checked on the device.
+__device__ __forceinline__ void ragged_range(const AttnParams& p, int s, int& start, int& len,
+                                             bool report) {
+  const int a = __ldg(p.cu_seqlens + s);
+  const int b = __ldg(p.cu_seqlens + s + 1);
+  if (a < 0 || b < a || b > p.Lkv) {
+    start = 0;
+    len = 0;
+    if (report) set_err(p, VKV_DEVERR_BAD_OFFSETS);
+  } else {
+    start = a;
+    len = b - a;
+  }
+}
+
+__device__ __forceinline__ int unit_steps(const AttnParams& p, const Ctl* ctl, int rlen) {
+  if (p.mode == VKV_MODE_SEGMENTS) return p.total_steps;
+  if (p.mode == VKV_MODE_RAGGED) return (rlen + 127) >> 7;
+  return (ctl->list_count + 1) >> 1;
+}
+
+// Build the unit's block list (BLOCK_SPARSE): persistent blocks (visible to
+// every query block of the unit) followed by the union of the window blocks
+// selected by the unit's query blocks, ascending, each tagged with the query
+// blocks that selected it.  Executed by all 32 lanes of one warp.
+__device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, const UnitInfo& u) {
+  const uint32_t lane = lane_id();
+  const int qb0 = u.tile0 * 2;
+  const int nqb = min(2 * u.ntiles, p.n_qblk - qb0);
+  const uint32_t all_mask = (nqb > 0) ? ((1u << nqb) - 1u) : 0u;
+  const int nwords = (p.n_win_blk + 31) >> 5;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ctl->bitmap[i][lane] = 0u;
+  __syncwarp();
+  for (int i = 0; i < nqb; ++i) {
+    const int* row = p.sel_idx + ((size_t)u.s * p.n_qblk + (qb0 + i)) * p.topk;
+    for (int e = lane; e < p.topk; e += 32) {
+      const int w = __ldg(row + e);
+      if (w >= 0 && w < p.n_win_blk) {
+        atomicOr(&ctl->bitmap[i][w >> 5], 1u << (w & 31));
+      } else {
+        set_err(p, VKV_DEVERR_BAD_INDEX);
+      }
+    }
+  }
+  __syncwarp();
+  int base = 0;
+  const int* prow = p.persist_idx + (size_t)u.s * p.n_persist;
+  for (int e0 = 0; e0 < p.n_persist; e0 += 32) {
+    const int e = e0 + (int)lane;
+    int blk = -1;
+    bool ok = false;
+    if (e < p.n_persist) {
+      blk = __ldg(prow + e);
+      ok = blk >= 0 && blk < p.n_blocks_total &&
+           (blk < p.window_blk0 || blk >= p.window_blk0 + p.n_win_blk);
+      if (!ok) set_err(p, VKV_DEVERR_BAD_INDEX);
+    }
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, ok);
+    if (ok) ctl->list[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)blk | (all_mask << 24);
+    base += __popc(bal);
+  }
+  // window union: lane L owns window blocks [32L, 32L + 32)
+  uint32_t m[4], uni = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = ((int)lane < nwords && i < nqb) ? ctl->bitmap[i][lane] : 0u;
+    uni |= m[i];
+  }
+  const int cnt = __popc(uni);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if ((int)lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  int pos = base + incl - cnt;
+  uint32_t rest = uni;
+  while (rest) {
+    const int bit = __ffs(rest) - 1;
+    rest &= rest - 1u;
+    uint32_t qm = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qm |= ((m[i] >> bit) & 1u) << i;
+    ctl->list[pos++] = (uint32_t)(p.window_blk0 + (int)lane * 32 + bit) | (qm << 24);
+  }
+  if (lane == 0) ctl->list_count = base + total;
+  __threadfence_block();
+  __syncwarp();
+}
+
+// 32 fp32 values -> 32 bf16 at dst (64 bytes, 16-byte aligned).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float* v) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = w;
+  }
+}
+
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float* v) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = s4[q];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e + 0] = __uint_as_float(ws[e] << 16);
+      v[8 * q + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+    }
+  }
+}
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Register split between the producer/MMA warpgroup and the two softmax
+// warpgroups.  setmaxnreg.inc only succeeds if the total stays within what the
+// CTA was launched with (384 threads x 168 registers); the host checks the
+// compiled register count against kRegsLaunchNeeded before every launch.
+constexpr int kRegsProducer = 104;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsLaunchNeeded = (128 * kRegsProducer + 256 * kRegsSoftmax + 383) / 384;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split");
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xFFFFFFFFu, v); }
+
+template <int D>
+__global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constant__ AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sP = sbase + C::OFF_P;
+  const uint32_t sKV = sbase + C::OFF_KV;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  volatile int* abort_flag = &ctl->abort_flag;
+  const uint32_t b_full0 = smem_u32(&ctl->full[0]);
+  const uint32_t b_empty0 = smem_u32(&ctl->empty[0]);
+  const uint32_t b_qfull = smem_u32(&ctl->q_full);
+  const uint32_t b_qempty = smem_u32(&ctl->q_empty);
+  const uint32_t b_sfull0 = smem_u32(&ctl->s_full[0]);
+  const uint32_t b_sfree0 = smem_u32(&ctl->s_free[0]);
+  const uint32_t b_pfull0 = smem_u32(&ctl->p_full[0]);
+  const uint32_t b_odone0 = smem_u32(&ctl->o_done[0]);
+  const uint32_t b_lready = smem_u32(&ctl->list_ready);
+  const uint32_t b_lfree = smem_u32(&ctl->list_free);
+  const uint32_t b_drain = smem_u32(&ctl->drain);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(b_full0 + 8 * i, 1);
+      mbar_init(b_empty0 + 8 * i, 1);
+    }
+    mbar_init(b_qfull, 1);
+    mbar_init(b_qempty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(b_sfull0 + 8 * t, 1);
+      mbar_init(b_sfree0 + 8 * t, 4);
+      mbar_init(b_pfull0 + 8 * t, 4);
+      mbar_init(b_odone0 + 8 * t, 1);
+    }
+    mbar_init(b_lready, 1);
+    mbar_init(b_lfree, 9);
+    mbar_init(b_drain, 1);
+    ctl->abort_flag = 0;
+    ctl->list_count = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const int u_begin = p.cta_begin[blockIdx.x];
+  const int u_end = p.cta_begin[blockIdx.x + 1];
+  const bool sparse = p.mode == VKV_MODE_BLOCK_SPARSE;
+  const bool ragged = p.mode == VKV_MODE_RAGGED;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsProducer>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t item = 0, qcnt = 0, ucnt = 0;
+      bool ok = true;
+      for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
+        const UnitInfo u = decode_unit(p, p.units[ui]);
+        int rs = 0, rl = 0;
+        if (sparse) {
+          if (ucnt > 0) {
+            bool w = true;
+            if (lane == 0) w = mbar_wait(b_lfree, (ucnt - 1) & 1, abort_flag, p.err);
+            ok = __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
+            if (!ok) break;
+          }
+          build_block_list(p, ctl, u);
+          if (lane == 0) mbar_arrive(b_lready);
+        } else if (ragged) {
+          ragged_range(p, u.s, rs, rl, lane == 0);
+        }
+        const int nsteps = unit_steps(p, ctl, rl);
+        if (nsteps == 0) continue;
+        if (lane == 0) {
+          if (qcnt > 0) ok = mbar_wait(b_qempty, (qcnt - 1) & 1, abort_flag, p.err);
+          if (ok) {
+            mbar_arrive_expect_tx(b_qfull, (uint32_t)(u.ntiles * C::QT_BYTES));
+            for (int t = 0; t < u.ntiles; ++t)
+#pragma unroll
+              for (int ac = 0; ac < C::NAC; ++ac)
+                tma_load_4d(sQ + t * C::QT_BYTES + ac * C::ATOM, &p.tm_q, ac * 64, u.h,
+                            (u.tile0 + t) * 128, u.b, b_qfull);
+            ++qcnt;
+          }
+          TileIter it;
+          it.init(&p, ctl, rs, rl);
+          const int kvh = ragged ? 0 : u.h;
+          const int kvb = ragged ? 0 : u.b;
+          for (int j = 0; j < nsteps && ok; ++j) {
+            const TileDesc td = it.next();
+            for (int kv = 0; kv < 2; ++kv) {
+              const uint32_t slot = item % C::NSLOT, use = item / C::NSLOT;
+              if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
+              if (!ok) break;
+              mbar_arrive_expect_tx(b_full0 + 8 * slot, (uint32_t)C::KV_BYTES);
+              const CUtensorMap* tm = kv ? &p.tm_v : &p.tm_k;
+              const uint32_t dst = sKV + slot * C::KV_BYTES;
+#pragma unroll
+              for (int ac = 0; ac < C::NAC; ++ac) {
+                tma_load_4d(dst + ac * C::ATOM, tm, ac * 64, kvh, td.rowA, kvb, b_full0 + 8 * slot);
+                tma_load_4d(dst + ac * C::ATOM + 64 * 128, tm, ac * 64, kvh, td.rowB, kvb,
+                            b_full0 + 8 * slot);
+              }
+              ++item;
+            }
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      if (!ok && lane == 0) {
+        // let copies already issued land before the CTA exits
+        for (uint32_t i = (item > (uint32_t)C::NSLOT ? item - C::NSLOT : 0); i < item; ++i)
+          mbar_wait_drain(b_full0 + 8 * (i % C::NSLOT), (i / C::NSLOT) & 1);
+        if (qcnt > 0) mbar_wait_drain(b_qfull, (qcnt - 1) & 1);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+        uint32_t item = 0, qcnt = 0, ucnt = 0;
+        uint32_t qk_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+        bool ok = true;
+        for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
+          const UnitInfo u = decode_unit(p, p.units[ui]);
+          int rs = 0, rl = 0;
+          if (sparse) {
+            ok = mbar_wait(b_lready, ucnt & 1, abort_flag, p.err);
+            if (!ok) break;
+          } else if (ragged) {
+            ragged_range(p, u.s, rs, rl, false);
+          }
+          const int nsteps = unit_steps(p, ctl, rl);
+          if (sparse) mbar_arrive(b_lfree);  // only the step count was needed
+          if (nsteps == 0) continue;
+          TileIter it;
+          it.init(&p, ctl, rs, rl);
+          ok = mbar_wait(b_qfull, qcnt & 1, abort_flag, p.err);
+          ++qcnt;
+          if (!ok) break;
+          // prologue: S_t = Q_t K_0^T
+          ok = mbar_wait(b_full0 + 8 * (item % C::NSLOT), (item / C::NSLOT) & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < u.ntiles && ok; ++t) {
+            if (qk_cnt[t] > 0) {
+              ok = mbar_wait(b_sfree0 + 8 * t, (qk_cnt[t] - 1) & 1, abort_flag, p.err);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t d_tm = tmem + (uint32_t)(t * 128);
+            const uint32_t qa = sQ + t * C::QT_BYTES;
+            const uint32_t kb = sKV + (item % C::NSLOT) * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+              mma_bf16_ss(d_tm, sdesc_k_sw128(qa + off), sdesc_k_sw128(kb + off), IDESC_QK, kk > 0);
+            }
+            mma_commit(b_sfull0 + 8 * t);
+            ++qk_cnt[t];
+          }
+          if (!ok) break;
+          mma_commit(b_empty0 + 8 * (item % C::NSLOT));
+          if (nsteps == 1) mma_commit(b_qempty);
+          for (int j = 0; j < nsteps && ok; ++j) {
+            const bool first = (sparse || ragged) ? (j == 0) : it.next().first;
+            const uint32_t vit = item + 2 * j + 1;
+            const uint32_t knext = item + 2 * j + 2;
+            const bool has_next = j + 1 < nsteps;
+            if (has_next) {
+              ok = mbar_wait(b_full0 + 8 * (knext % C::NSLOT), (knext / C::NSLOT) & 1, abort_flag, p.err);
+              if (!ok) break;
+            }
+            ok = mbar_wait(b_full0 + 8 * (vit % C::NSLOT), (vit / C::NSLOT) & 1, abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
+            for (int t = 0; t < u.ntiles && ok; ++t) {
+              if (has_next) {
+                ok = mbar_wait(b_sfree0 + 8 * t, (qk_cnt[t] - 1) & 1, abort_flag, p.err);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d_tm = tmem + (uint32_t)(t * 128);
+                const uint32_t qa = sQ + t * C::QT_BYTES;
+                const uint32_t kb = sKV + (knext % C::NSLOT) * C::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+                  mma_bf16_ss(d_tm, sdesc_k_sw128(qa + off), sdesc_k_sw128(kb + off), IDESC_QK,
+                              kk > 0);
+                }
+                mma_commit(b_sfull0 + 8 * t);
+                ++qk_cnt[t];
+              }
+              ok = mbar_wait(b_pfull0 + 8 * t, pv_cnt[t] & 1, abort_flag, p.err);
+              if (!ok) break;
+              tc_fence_after();
+              {
+                const uint32_t d_tm = tmem + C::TM_O + (uint32_t)(t * D);
+                const uint32_t pa = sP + t * C::P_BYTES;
+                const uint32_t vb = sKV + (vit % C::NSLOT) * C::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t aoff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+                  mma_bf16_ss(d_tm, sdesc_k_sw128(pa + aoff), sdesc_mn_sw128(vb + kk * 2048, C::ATOM),
+                              IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+                }
+              }
+              mma_commit(b_odone0 + 8 * t);
+              ++pv_cnt[t];
+            }
+            if (!ok) break;
+            if (has_next) {
+              mma_commit(b_empty0 + 8 * (knext % C::NSLOT));
+              if (j + 2 == nsteps) mma_commit(b_qempty);
+            }
+            mma_commit(b_empty0 + 8 * (vit % C::NSLOT));
+          }
+          item += 2 * nsteps;
+        }
+        // every MMA issued so far completes before TMEM is released
+        mma_commit(b_drain);
+        mbar_wait_drain(b_drain, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int t = (warp >= 8) ? 1 : 0;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + (int)lane;  // row inside the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
+    const uint32_t tO = tmem + lane_base + C::TM_O + (uint32_t)(t * D);
+    const uint32_t sPt = sP + t * C::P_BYTES;
+    const uint32_t b_sfull = b_sfull0 + 8 * t, b_sfree = b_sfree0 + 8 * t;
+    const uint32_t b_pfull = b_pfull0 + 8 * t, b_odone = b_odone0 + 8 * t;
+    const float sl2 = p.scale_log2;
+    uint32_t sf_cnt = 0, np = 0, ucnt = 0;
+    bool ok = true;
+    for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
+      const UnitInfo u = decode_unit(p, p.units[ui]);
+      int rs = 0, rl = 0;
+      if (sparse) {
+        ok = warp_all(mbar_wait(b_lready, ucnt & 1, abort_flag, p.err));
+        if (!ok) break;
+      } else if (ragged) {
+        ragged_range(p, u.s, rs, rl, false);
+      }
+      const int nsteps = unit_steps(p, ctl, rl);
+      const bool active = t < u.ntiles;
+      const int qrow = (u.tile0 + t) * 128 + r;
+      const bool row_ok = qrow < p.Lq;
+      const int qb = 2 * t + (r >> 6);
+      float m = -INFINITY, l = 0.f;            // running state of the current branch
+      float m_prev = -INFINITY, l_prev = 0.f;  // state of the branch closed before it
+      int cur_branch = -1, prev_branch = -1;
+      if (active && nsteps > 0) {
+        TileIter it;
+        it.init(&p, ctl, rs, rl);
+        for (int j = 0; j < nsteps; ++j) {
+          const TileDesc td = it.next();
+          ok = warp_all(mbar_wait(b_sfull, sf_cnt & 1, abort_flag, p.err));
+          ++sf_cnt;
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t sr[128];
+          tmem_ld32(tS + 0, sr + 0);
+          tmem_ld32(tS + 32, sr + 32);
+          tmem_ld32(tS + 64, sr + 64);
+          tmem_ld32(tS + 96, sr + 96);
+          tmem_ld_wait();
+          reg_fence<128>(sr);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_sfree);
+          bool pending_epi = false;
+          if (td.first) {
+            if (cur_branch >= 0) {
+              pending_epi = true;
+              prev_branch = cur_branch;
+              m_prev = m;
+              l_prev = l;
+            }
+            cur_branch = td.branch;
+            m = -INFINITY;
+            l = 0.f;
+          }
+          // visibility of this tile for this row
+          const int limA = ((td.maskA >> qb) & 1u) ? td.limA : 0;
+          const int limB = ((td.maskB >> qb) & 1u) ? td.limB : 0;
+          if (__any_sync(0xFFFFFFFFu, (limA < 64) || (limB < 64))) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              if (c >= limA) sr[c] = __float_as_uint(-INFINITY);
+              if (c >= limB) sr[64 + c] = __float_as_uint(-INFINITY);
+            }
+          }
+          float mx8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float mt = mx * sl2;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m == -INFINITY) {
+            m = mt;
+          } else if (mt > m + kRescaleThreshold) {
+            alpha = ex2_approx(m - mt);
+            m = mt;
+            rescale = true;
+          }
+          const float mu = (m == -INFINITY) ? 0.f : m;
+          float sm8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const float e = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -mu));
+            sr[c] = __float_as_uint(e);
+            sm8[c & 7] += e;
+          }
+          l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
+          // the previous PV of this tile must be done: P buffer free, O final
+          if (np > 0) {
+            ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          // P (bf16) -> shared memory, 128-byte swizzled K-major
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t addr =
+                sPt + (uint32_t)((c >> 3) * C::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+            st_shared_v4(addr,
+                         pack_bf16x2(__uint_as_float(sr[8 * c + 0]), __uint_as_float(sr[8 * c + 1])),
+                         pack_bf16x2(__uint_as_float(sr[8 * c + 2]), __uint_as_float(sr[8 * c + 3])),
+                         pack_bf16x2(__uint_as_float(sr[8 * c + 4]), __uint_as_float(sr[8 * c + 5])),
+                         pack_bf16x2(__uint_as_float(sr[8 * c + 6]), __uint_as_float(sr[8 * c + 7])));
+          }
+          if (pending_epi) {
+            // close the previous branch: O / l and LSE
+            const bool has = l_prev > 0.f;
+            const float inv = has ? 1.f / l_prev : 0.f;
+            __nv_bfloat16* orow = p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
+                                  (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch];
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(tO + c0, v);
+              tmem_ld_wait();
+              reg_fence<32>(v);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
+              if (row_ok) store_row32(orow + c0, reinterpret_cast<const float*>(v));
+            }
+            if (row_ok)
+              p.lse[prev_branch][(size_t)u.s * p.Lq + qrow] =
+                  has ? (m_prev + lg2_approx(l_prev)) * kLn2 : -INFINITY;
+          } else if (__any_sync(0xFFFFFFFFu, rescale)) {
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(tO + c0, v);
+              tmem_ld_wait();
+              reg_fence<32>(v);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+              tmem_st32(tO + c0, v);
+            }
+            tmem_st_wait();
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_pfull);
+          ++np;
+        }
+        if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
+        if (ok) {
+          tc_fence_after();
+          // close the last branch, and merge with the one before it when asked
+          const int lb = cur_branch;
+          const bool has = l > 0.f;
+          const float inv = has ? 1.f / l : 0.f;
+          const bool do_merge = p.om != nullptr && p.n_branches == 2 && !sparse && !ragged;
+          const bool has_prev = prev_branch >= 0 && l_prev > 0.f;
+          const float L_last = has ? m + lg2_approx(l) : -INFINITY;
+          const float L_prev = has_prev ? m_prev + lg2_approx(l_prev) : -INFINITY;
+          const float M = fmaxf(L_last, L_prev);
+          const float Ms = (M == -INFINITY) ? 0.f : M;
+          const float w_last = has ? ex2_approx(L_last - Ms) : 0.f;
+          const float w_prev = has_prev ? ex2_approx(L_prev - Ms) : 0.f;
+          const float den = w_last + w_prev;
+          const float c_last = den > 0.f ? w_last / den : 0.f;
+          const float c_prev = den > 0.f ? w_prev / den : 0.f;
+          __nv_bfloat16* orow =
+              p.o[lb] + u.b * p.o_sb[lb] + (long long)qrow * p.o_st[lb] + u.h * p.o_sh[lb];
+          __nv_bfloat16* mrow =
+              do_merge ? p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh : nullptr;
+          const __nv_bfloat16* prow =
+              has_prev ? p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
+                             (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch]
+                       : nullptr;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tO + c0, v);
+            tmem_ld_wait();
+            reg_fence<32>(v);
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]) * inv;
+            if (row_ok) {
+              store_row32(orow + c0, f);
+              if (do_merge) {
+                float g[32];
+                if (has_prev) {
+                  load_row32(prow + c0, g);
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) g[e] = c_last * f[e] + c_prev * g[e];
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) g[e] = c_last * f[e];
+                }
+                store_row32(mrow + c0, g);
+              }
+            }
+          }
+          if (row_ok) {
+            p.lse[lb][(size_t)u.s * p.Lq + qrow] = has ? L_last * kLn2 : -INFINITY;
+            if (do_merge)
+              p.lsem[(size_t)u.s * p.Lq + qrow] =
+                  (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
+          }
+        }
+      }
+      if (ok && active && row_ok) {
+        // branches without any key tile: O = 0, LSE = -inf
+        const int nb = (sparse || ragged) ? 1 : p.n_branches;
+        for (int br = 0; br < nb; ++br) {
+          const bool empty = (sparse || ragged) ? (nsteps == 0) : (p.branch_steps[br] == 0);
+          if (!empty) continue;
+          __nv_bfloat16* orow =
+              p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
+          float z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0.f;
+          for (int c0 = 0; c0 < D; c0 += 32) store_row32(orow + c0, z);
+          p.lse[br][(size_t)u.s * p.Lq + qrow] = -INFINITY;
+        }
+        if (nsteps == 0 && p.om != nullptr && p.n_branches == 2 && !sparse && !ragged) {
+          __nv_bfloat16* mrow = p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh;
+          float z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0.f;
+          for (int c0 = 0; c0 < D; c0 += 32) store_row32(mrow + c0, z);
+          p.lsem[(size_t)u.s * p.Lq + qrow] = -INFINITY;
+        }
+      }
+      if (sparse) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_lfree);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace vkv

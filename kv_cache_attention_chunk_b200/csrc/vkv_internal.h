@@ -1,0 +1,61 @@
+// Internal declarations shared by the host launchers and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "vkv.h"
+
+namespace vkv {
+
+constexpr int kMaxUnits = 6144;        // work units per launch (kernel parameter space)
+constexpr int kMaxCtas = 160;          // >= SMs of a B200 (148)
+constexpr int kMaxListEntries = 288;   // block list of one BLOCK_SPARSE unit
+constexpr int kCtlBytes = 2048;        // control block in shared memory
+constexpr int kMaxFlatSegs = VKV_MAX_BRANCHES * VKV_MAX_SEGMENTS;
+
+// Kernel parameters of the attention kernel, passed as __grid_constant__.
+// Unit code: bits [0,13) first query tile, bit 13 two tiles, bits [14,32) sequence b*H+h.
+struct AttnParams {
+  CUtensorMap tm_q;  // dims (d, H, Lq, B); box (64, 1, 128, 1); 128 B swizzle
+  CUtensorMap tm_k;  // dims (d, H, Lkv, B) or (d, 1, rows, 1); box (64, 1, 64, 1)
+  CUtensorMap tm_v;
+  int mode, B, H, Lq, Lkv, d;
+  float scale_log2;  // softmax scale * log2(e)
+  int n_branches;
+  int branch_steps[VKV_MAX_BRANCHES];
+  int total_steps;
+  int n_flat;  // SEGMENTS: non-empty segments in branch order
+  int flat_start[kMaxFlatSegs];
+  int flat_len[kMaxFlatSegs];
+  int flat_branch[kMaxFlatSegs];
+  int flat_first[kMaxFlatSegs];
+  // BLOCK_SPARSE
+  int n_persist, topk, window_blk0, n_win_blk, n_qblk, n_blocks_total;
+  const int* persist_idx;
+  const int* sel_idx;
+  // RAGGED
+  const int* cu_seqlens;
+  // outputs
+  __nv_bfloat16* o[VKV_MAX_BRANCHES];
+  long long o_sb[VKV_MAX_BRANCHES], o_st[VKV_MAX_BRANCHES], o_sh[VKV_MAX_BRANCHES];
+  float* lse[VKV_MAX_BRANCHES];
+  __nv_bfloat16* om;
+  long long om_sb, om_st, om_sh;
+  float* lsem;
+  int* err;
+  // schedule: CTA c runs units[cta_begin[c] .. cta_begin[c+1])
+  int n_ctas;
+  int cta_begin[kMaxCtas + 1];
+  uint32_t units[kMaxUnits];
+};
+
+// Host helpers (vkv_common.cu).
+int device_sm_count(int* dev_out);                // -1 when no usable sm_100 device
+bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
+                         const uint64_t strides_bytes[3], const uint32_t box[4]);
+bool tensor_aligned(const vkv_tensor& t);
+
+}  // namespace vkv

@@ -1,0 +1,291 @@
+"""ctypes binding of libvkv (include/vkv.h): argument marshalling only.
+
+Every computation runs in the library's sm_100a kernels; this module turns
+torch tensors into the C structs, passes the current CUDA stream and raises
+on a non-OK status.  There is no fallback: if libvkv.so is missing or no
+sm_100 device is present the calls raise.
+
+Raw entry points with the C names: ``vkv_chunk_attn``, ``vkv_block_select``,
+``vkv_block_select_workspace_size``, ``vkv_lse_merge``, ``vkv_status_string``.
+Convenience wrappers that allocate outputs with torch: ``chunk_attn_segments``,
+``chunk_attn_block_sparse``, ``chunk_attn_ragged``, ``block_select``, ``lse_merge``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int32, c_int64, c_size_t, c_void_p
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvkv.so")
+
+MODE_SEGMENTS, MODE_BLOCK_SPARSE, MODE_RAGGED = 0, 1, 2
+MAX_BRANCHES, MAX_SEGMENTS = 2, 8
+DEVERR_TIMEOUT, DEVERR_BAD_INDEX, DEVERR_BAD_OFFSETS = 1, 2, 3
+STATUS = {0: "VKV_OK", 1: "VKV_ERR_NULL", 2: "VKV_ERR_SHAPE", 3: "VKV_ERR_ALIGN", 4: "VKV_ERR_RANGE",
+          5: "VKV_ERR_UNSUPPORTED", 6: "VKV_ERR_CUDA", 7: "VKV_ERR_WORKSPACE"}
+
+
+class VkvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({vkv_status_string(status)})")
+
+
+class vkv_segment(ctypes.Structure):
+    _fields_ = [("start", c_int32), ("len", c_int32)]
+
+
+class vkv_tensor(ctypes.Structure):
+    _fields_ = [("ptr", c_void_p), ("sb", c_int64), ("st", c_int64), ("sh", c_int64)]
+
+
+class vkv_attn_args(ctypes.Structure):
+    _fields_ = [
+        ("mode", c_int32), ("B", c_int32), ("H", c_int32), ("Lq", c_int32), ("Lkv", c_int32),
+        ("d", c_int32), ("scale", c_float),
+        ("q", vkv_tensor), ("k", vkv_tensor), ("v", vkv_tensor),
+        ("n_branches", c_int32),
+        ("segs", POINTER(vkv_segment) * MAX_BRANCHES),
+        ("n_segs", c_int32 * MAX_BRANCHES),
+        ("block", c_int32),
+        ("persist_idx", c_void_p), ("n_persist", c_int32),
+        ("sel_idx", c_void_p), ("topk", c_int32), ("window_blk0", c_int32), ("n_win_blk", c_int32),
+        ("cu_seqlens", c_void_p), ("cu_seqlens_host", POINTER(c_int32)),
+        ("o", vkv_tensor * MAX_BRANCHES), ("lse", c_void_p * MAX_BRANCHES),
+        ("o_merged", vkv_tensor), ("lse_merged", c_void_p),
+        ("err_word", c_void_p),
+    ]
+
+
+class vkv_select_args(ctypes.Structure):
+    _fields_ = [
+        ("B", c_int32), ("H", c_int32), ("d", c_int32), ("block", c_int32),
+        ("Lq", c_int32), ("Lkv", c_int32), ("window_blk0", c_int32), ("n_win_blk", c_int32),
+        ("topk", c_int32),
+        ("q", vkv_tensor), ("k", vkv_tensor),
+        ("out_idx", c_void_p), ("out_scores", c_void_p),
+        ("workspace", c_void_p), ("workspace_bytes", c_size_t),
+        ("err_word", c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvkv.so (built in-tree by kv_cache_attention_chunk_b200.build); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_attention_chunk_b200.build`"
+                           " (there is no fallback implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    L.vkv_chunk_attn.argtypes = [POINTER(vkv_attn_args), c_void_p]
+    L.vkv_chunk_attn.restype = c_int32
+    L.vkv_block_select.argtypes = [POINTER(vkv_select_args), c_void_p]
+    L.vkv_block_select.restype = c_int32
+    L.vkv_block_select_workspace_size.argtypes = [c_int32] * 6
+    L.vkv_block_select_workspace_size.restype = c_size_t
+    L.vkv_lse_merge.argtypes = [vkv_tensor, c_void_p, vkv_tensor, c_void_p, vkv_tensor, c_void_p,
+                                c_int32, c_int32, c_int32, c_int32, c_void_p]
+    L.vkv_lse_merge.restype = c_int32
+    L.vkv_status_string.argtypes = [c_int32]
+    L.vkv_status_string.restype = ctypes.c_char_p
+    L.vkv_version.argtypes = []
+    L.vkv_version.restype = c_int32
+    L.vkv_abi_sizeof.argtypes = [c_int32]
+    L.vkv_abi_sizeof.restype = c_int32
+    for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment)):
+        if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
+            raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
+                               f"binding {ctypes.sizeof(st)} B")
+    _lib = L
+    return L
+
+
+# ---------------------------------------------------------------------------
+# raw entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+def vkv_status_string(status: int) -> str:
+    return lib().vkv_status_string(int(status)).decode()
+
+
+def vkv_chunk_attn(args: vkv_attn_args, stream: int | None) -> int:
+    return int(lib().vkv_chunk_attn(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
+    return int(lib().vkv_block_select(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_block_select_workspace_size(B, H, Lq, n_win_blk, block, d) -> int:
+    return int(lib().vkv_block_select_workspace_size(B, H, Lq, n_win_blk, block, d))
+
+
+def vkv_lse_merge(o_a: vkv_tensor, lse_a, o_b: vkv_tensor, lse_b, o_out: vkv_tensor, lse_out,
+                  B, H, Lq, d, stream: int | None) -> int:
+    return int(lib().vkv_lse_merge(o_a, c_void_p(lse_a), o_b, c_void_p(lse_b), o_out, c_void_p(lse_out),
+                                   B, H, Lq, d, c_void_p(stream or 0)))
+
+
+# ---------------------------------------------------------------------------
+# torch helpers
+# ---------------------------------------------------------------------------
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def tensor_desc(x: torch.Tensor) -> vkv_tensor:
+    """[B, L, H, d] bf16 with a contiguous last axis -> vkv_tensor."""
+    if x.dim() != 4 or x.dtype != torch.bfloat16 or x.stride(3) != 1:
+        raise ValueError("expected a bf16 [B, L, H, d] tensor with contiguous d")
+    return vkv_tensor(x.data_ptr(), x.stride(0), x.stride(1), x.stride(2))
+
+
+def flat_desc(x: torch.Tensor) -> vkv_tensor:
+    """[rows, d] bf16 with contiguous d -> vkv_tensor (row stride in st)."""
+    if x.dim() != 2 or x.dtype != torch.bfloat16 or x.stride(1) != 1:
+        raise ValueError("expected a bf16 [rows, d] tensor with contiguous d")
+    return vkv_tensor(x.data_ptr(), 0, x.stride(0), 0)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise VkvError(status, what)
+
+
+def _base_args(mode, q, Lkv, d, scale, k_desc, v_desc, err):
+    B, Lq, H, dq = q.shape
+    if dq != d:
+        raise ValueError("head dimension mismatch")
+    a = vkv_attn_args()
+    a.mode = mode
+    a.B, a.H, a.Lq, a.Lkv, a.d = B, H, Lq, Lkv, d
+    a.scale = float(scale if scale is not None else 1.0 / np.sqrt(d))
+    a.q = tensor_desc(q)
+    a.k = k_desc
+    a.v = v_desc
+    a.block = 64
+    a.err_word = err.data_ptr() if err is not None else None
+    return a
+
+
+def _new_out(q):
+    B, Lq, H, d = q.shape
+    return (torch.empty((B, Lq, H, d), dtype=torch.bfloat16, device=q.device),
+            torch.empty((B, H, Lq), dtype=torch.float32, device=q.device))
+
+
+def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, stream=None, out=None):
+    """Dual-branch (or single-branch) chunk attention over token segments.
+
+    branches: list (length 1 or 2) of lists of (start, len) cache-row segments.
+    Returns dict(o=[...], lse=[...], o_merged, lse_merged).
+    """
+    nb = len(branches)
+    d = q.shape[3]
+    a = _base_args(MODE_SEGMENTS, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
+    a.n_branches = nb
+    keep = []
+    for i, br in enumerate(branches):
+        arr = (vkv_segment * max(1, len(br)))(*[vkv_segment(int(s), int(n)) for s, n in br])
+        keep.append(arr)
+        a.segs[i] = ctypes.cast(arr, POINTER(vkv_segment))
+        a.n_segs[i] = len(br)
+    res = out if out is not None else {}
+    if out is None:
+        res["o"], res["lse"] = [], []
+        for _ in range(nb):
+            o, l = _new_out(q)
+            res["o"].append(o)
+            res["lse"].append(l)
+        res["o_merged"], res["lse_merged"] = _new_out(q) if (merged and nb == 2) else (None, None)
+    for i in range(nb):
+        a.o[i] = tensor_desc(res["o"][i])
+        a.lse[i] = res["lse"][i].data_ptr()
+    if res.get("o_merged") is not None:
+        a.o_merged = tensor_desc(res["o_merged"])
+        a.lse_merged = res["lse_merged"].data_ptr()
+    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    return res
+
+
+def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_blk, scale=None,
+                            err=None, stream=None, out=None):
+    """Persistent blocks + selected window blocks (device int32 index tensors)."""
+    d = q.shape[3]
+    a = _base_args(MODE_BLOCK_SPARSE, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
+    persist_idx = persist_idx.contiguous()
+    sel_idx = sel_idx.contiguous()
+    a.persist_idx = persist_idx.data_ptr() if persist_idx.numel() else None
+    a.n_persist = persist_idx.shape[-1]
+    a.sel_idx = sel_idx.data_ptr() if sel_idx.numel() else None
+    a.topk = sel_idx.shape[-1]
+    a.window_blk0 = int(window_blk0)
+    a.n_win_blk = int(n_win_blk)
+    o, l = out if out is not None else _new_out(q)
+    a.o[0] = tensor_desc(o)
+    a.lse[0] = l.data_ptr()
+    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    return o, l
+
+
+def chunk_attn_ragged(q, k_flat, v_flat, cu_seqlens, cu_seqlens_host=None, scale=None, err=None,
+                      stream=None, out=None):
+    """Ragged per-(batch, head) caches stored flattened with boundary offsets."""
+    d = q.shape[3]
+    a = _base_args(MODE_RAGGED, q, k_flat.shape[0], d, scale, flat_desc(k_flat), flat_desc(v_flat), err)
+    a.cu_seqlens = cu_seqlens.data_ptr()
+    host = None
+    if cu_seqlens_host is not None:
+        host = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+        a.cu_seqlens_host = host.ctypes.data_as(POINTER(c_int32))
+    o, l = out if out is not None else _new_out(q)
+    a.o[0] = tensor_desc(o)
+    a.lse[0] = l.data_ptr()
+    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    return o, l
+
+
+def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=False, err=None, stream=None,
+                 out_idx=None):
+    """Top-K window blocks per 64-query block; returns (idx [B*H, nQblk, topk], scores or None)."""
+    B, Lq, H, d = q.shape
+    n_qblk = -(-Lq // 64)
+    a = vkv_select_args()
+    a.B, a.H, a.d, a.block = B, H, d, 64
+    a.Lq, a.Lkv = Lq, k.shape[1]
+    a.window_blk0, a.n_win_blk, a.topk = int(window_blk0), int(n_win_blk), int(topk)
+    a.q = tensor_desc(q)
+    a.k = tensor_desc(k)
+    idx = out_idx if out_idx is not None else torch.empty((B * H, n_qblk, topk), dtype=torch.int32,
+                                                          device=q.device)
+    a.out_idx = idx.data_ptr()
+    sc = None
+    if scores:
+        sc = torch.empty((B * H, n_qblk, n_win_blk), dtype=torch.float32, device=q.device)
+        a.out_scores = sc.data_ptr()
+    need = vkv_block_select_workspace_size(B, H, Lq, n_win_blk, 64, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a.err_word = err.data_ptr() if err is not None else None
+    _check(vkv_block_select(a, _stream(stream)), "vkv_block_select")
+    return idx, sc
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, stream=None, out=None):
+    B, Lq, H, d = o_a.shape
+    o, l = out if out is not None else _new_out(o_a)
+    _check(vkv_lse_merge(tensor_desc(o_a), lse_a.data_ptr(), tensor_desc(o_b), lse_b.data_ptr(),
+                         tensor_desc(o), l.data_ptr(), B, H, Lq, d, _stream(stream)), "vkv_lse_merge")
+    return o, l
