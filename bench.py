@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of chunk attention over a segmented KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload: the Wan-14B-shaped dense dual-branch chunk (B=1, 40 heads,
+d=128, 1560 tokens per latent frame; Q = a 3-frame chunk of 4680 tokens; KV =
+1 sink + 20 history + 3 current frames = 37 440 tokens; local branch = sink +
+current, history branch = the 20 history frames; both branch outputs with
+their LSEs plus the LSE-merged output).  One step = one vkv_chunk_attn call.
+Metric: effective TFLOP/s counting 4*d per visited (query, key) pair, its
+fraction of the measured bf16 dense peak, and ms per chunk.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
+(independent seeds) with no collective on the data path (weak scaling); the
+time is the max over ranks; rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores (bounded samples
+of the same workload); under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_attention_chunk_b200 import workloads as W  # noqa: E402
+
+METRIC = "chunk-attn effective TFLOP/s & % of bf16 tensor peak; ms per 3-frame chunk"
+WORKLOAD = ("wan14b dense dual-branch chunk: B=1, H=40, d=128, 1560 tok/frame, Q 4680 (3 frames), "
+            "KV 37440 (1 sink + 20 history + 3 current frames), local=sink+current, history=20 frames, "
+            "outputs O/LSE per branch + LSE-merged O/LSE")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (also exercised by the gloo tests)
+# ---------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def dist_setup(backend: str | None = None):
+    import torch.distributed as dist
+    rank, local, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws an independent chunk of the same shape."""
+    return base + 7919 * rank
+
+
+def headline_case(rank: int = 0):
+    return W.make_dual_branch("wan14b", rank_seed(4, rank), H=40, d=128, frame_tokens=1560, q_frames=3,
+                              hist_frames=20)
+
+
+def headline_flops() -> int:
+    loc, hist = W.dual_branch_layout(1560, 1, 20, 3)
+    n = sum(l for _, l in loc) + sum(l for _, l in hist)
+    return 4 * 128 * 40 * 4680 * n
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, profiles
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_attention_chunk_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "attn_wan14b_traffic.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        if d.get("kernel_source_hash") == kernel_source_hash():
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.idx, self.period, self.proc, self.out = gpu_index, period_ms, None, ""
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", f"-lms={self.period}"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            self.out = ""
+        rows = [r.split(", ") for r in self.out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw) if p > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+def host_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info()]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(case, rows: int, head: int = 0):
+    """Run the fp64 oracle (both branches + their LSE merge) on `rows` query rows of one head."""
+    import oracle
+    q = oracle.to64(case.q[0, :rows, head])
+    k = oracle.to64(case.k[0, :, head])
+    v = oracle.to64(case.v[0, :, head])
+    t0 = time.perf_counter()
+    parts = []
+    for br in case.branches:
+        idx = oracle.segment_rows(br)
+        parts.append(oracle.attend(q, k[idx], v[idx], case.scale))
+    oracle.lse_merge(parts[0][0], parts[0][1], parts[1][0], parts[1][1])
+    dt = time.perf_counter() - t0
+    n_keys = sum(l for br in case.branches for _, l in br)
+    return dt, 4 * case.d * rows * n_keys
+
+
+def calibrate_rows(case, seconds: float) -> int:
+    dt, _ = oracle_sample(case, 32)
+    rows = int(32 * seconds / max(dt, 1e-3))
+    return max(16, min(case.Lq, rows))
+
+
+def cpu_baseline(case, seconds: float = 12.0):
+    rows = calibrate_rows(case, seconds)
+    dt, fl = oracle_sample(case, rows)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"head 0, query rows 0..{rows - 1} of the wan14b chunk (both branches + LSE merge, "
+                      f"fp64 NumPy), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    case = headline_case(0)
+    budget = 150.0
+    per_step = max(0.05, budget / max(1, args.steps + args.warmup))
+    rows = calibrate_rows(case, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(case, rows)
+    tot_t, tot_f = 0.0, 0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(case, rows)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_step": rows, "sample_head": 0},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                             "sample": f"head 0, query rows 0..{rows - 1} per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def timed(fn, iters: int, stream) -> list:
+    ts = []
+    for _ in range(iters):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return ts
+
+
+def extras(dev, peaks):
+    """Per-mode timings of the other workloads (parity cases, reported for context)."""
+    from kv_cache_attention_chunk_b200 import vkv
+    import oracle
+    out = {}
+    st = torch.cuda.current_stream()
+    # Wan-1.3B-shaped dense dual-branch chunk
+    c = W.cfg_wan13b()
+    q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+    res = vkv.chunk_attn_segments(q, k, v, c.branches, scale=c.scale)
+    ms = statistics.median(timed(lambda: vkv.chunk_attn_segments(q, k, v, c.branches, scale=c.scale, out=res),
+                                 20, st))
+    fl = oracle.visited_flops_segments(1, 12, c.Lq, 128, c.branches)
+    out["wan13b_dense"] = {"ms": ms, "tflops": fl / ms / 1e9}
+    # standalone merge on the Wan-1.3B partials
+    mo = vkv.lse_merge(res["o"][0], res["lse"][0], res["o"][1], res["lse"][1])
+    ms = statistics.median(timed(lambda: vkv.lse_merge(res["o"][0], res["lse"][0], res["o"][1], res["lse"][1],
+                                                       out=mo), 50, st))
+    nbytes = 3 * res["o"][0].numel() * 2 + 3 * res["lse"][0].numel() * 4
+    out["lse_merge_wan13b"] = {"ms": ms, "gbs": nbytes / ms / 1e6, "bytes": nbytes,
+                               "frac_hbm": nbytes / ms / 1e6 / peaks["hbm_gbs"]}
+    del q, k, v, res, mo
+    # block-sparse: persistent + top-K window blocks
+    c = W.cfg_sparse()
+    q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+    pers = torch.from_numpy(c.persist_idx).to(dev)
+    sp = {}
+    for frac in W.SPARSE_TOPK_FRACTIONS:
+        K = W.topk_for_fraction(frac, c.n_win_blk)
+        ws = torch.empty(vkv.vkv_block_select_workspace_size(1, 12, c.Lq, c.n_win_blk, 64, 128),
+                         dtype=torch.uint8, device=dev)
+        idx, _ = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws)
+        ms_sel = statistics.median(timed(lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K,
+                                                                  workspace=ws, out_idx=idx), 30, st))
+        o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale)
+        ms_att = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
+            q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o), 20, st))
+        fl = oracle.visited_flops_sparse(1, 12, c.Lq, 128, 64, c.persist_idx.shape[1], K)
+        sel_bytes = (c.Lq + c.n_win_blk * 64) * 12 * 128 * 2
+        sp[f"K{K}"] = {"attn_ms": ms_att, "attn_tflops": fl / ms_att / 1e9, "select_ms": ms_sel,
+                       "select_gbs": sel_bytes / ms_sel / 1e6, "visited_frac": (32 + K) / (32 + c.n_win_blk)}
+    full = sp[f"K{c.n_win_blk}"]["attn_ms"]
+    for kk in sp:
+        sp[kk]["time_frac_of_K_all"] = sp[kk]["attn_ms"] / full
+    out["sparse"] = sp
+    del q, k, v
+    # ragged per-head cache
+    c = W.cfg_ragged()
+    q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+    cu = torch.from_numpy(c.cu_seqlens).to(dev)
+    o = vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale)
+    ms = statistics.median(timed(lambda: vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale, out=o),
+                                 20, st))
+    fl = oracle.visited_flops_ragged(1, 12, c.Lq, 128, c.cu_seqlens)
+    out["ragged"] = {"ms": ms, "tflops": fl / ms / 1e9}
+    return out
+
+
+def run_ours(args):
+    from kv_cache_attention_chunk_b200 import build, vkv
+    rank, local, world = dist_setup()
+    if local == 0:
+        build.build()
+    barrier()
+    vkv.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    case = headline_case(rank)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = vkv.chunk_attn_segments(q, k, v, case.branches, scale=case.scale, err=err)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vkv.chunk_attn_segments(q, k, v, case.branches, scale=case.scale, err=err, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(vis.split(",")[local].strip() if vis else local)
+    if rank == 0 or world == 1:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if (rank == 0 or world == 1) else None
+    total_ms = e0.elapsed_time(e1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(total_ms, dev if world > 1 and torch.distributed.get_backend() == "nccl" else "cpu")
+    ms_step = total_ms / args.steps
+    fl = headline_flops()
+    value = world * fl / (ms_step * 1e-3) / 1e12
+    avg_launch = statistics.mean(launch_ms)
+    achieved = fl / (avg_launch * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+
+    # end to end through the C ABI with host buffers: H2D inputs, call, D2H outputs
+    hq, hk, hv = (t.cpu().pin_memory() for t in (case.q, case.k, case.v))
+    hout = [t.cpu().pin_memory() for t in out["o"] + [out["o_merged"]] + out["lse"] + [out["lse_merged"]]]
+    dout = out["o"] + [out["o_merged"]] + out["lse"] + [out["lse_merged"]]
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        for h, d_ in zip(hout, dout):
+            h.copy_(d_, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / e2e_steps,
+                            dev if world > 1 and torch.distributed.get_backend() == "nccl" else "cpu")
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+
+    if rank != 0:
+        barrier()
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "parallelism": f"independent chunk per GPU x{world}",
+                   "l2": "no flush: each step reads 961 MB of inputs, larger than the 126 MB L2",
+                   "ms_per_chunk": ms_step, "pct_of_bf16_peak": 100.0 * value / world / peak,
+                   "flops_per_chunk": fl},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(),
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": "chunk_attn_kernel<128>",
+                     "launch_ms_median": statistics.median(launch_ms)},
+        "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case)
+    if world == 1 and not args.no_extras:
+        del q, k, v, out
+        torch.cuda.empty_cache()
+        line["modes"] = extras(dev, peaks)
+    barrier()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_profile(args):
+    """Small fixed cases for ncu captures: warmup + steps launches of one kernel, no JSON contract."""
+    from kv_cache_attention_chunk_b200 import build, vkv
+    build.build()
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream()
+    if args.profile in ("wan13b", "wan14b"):
+        c = W.cfg_wan13b() if args.profile == "wan13b" else headline_case(0)
+        q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+        out = vkv.chunk_attn_segments(q, k, v, c.branches, scale=c.scale)
+        fn = lambda: vkv.chunk_attn_segments(q, k, v, c.branches, scale=c.scale, out=out)  # noqa: E731
+    elif args.profile == "merge":
+        oa, la, ob, lb = (t.to(dev) for t in W.make_merge_inputs(5, 1, 4680, 40, 128))
+        o = vkv.lse_merge(oa, la, ob, lb)
+        fn = lambda: vkv.lse_merge(oa, la, ob, lb, out=o)  # noqa: E731
+    elif args.profile in ("select", "sparse9", "sparse144"):
+        c = W.cfg_sparse()
+        q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+        K = 9 if args.profile != "sparse144" else 144
+        idx, _ = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K)
+        if args.profile == "select":
+            fn = lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, out_idx=idx)  # noqa: E731
+        else:
+            pers = torch.from_numpy(c.persist_idx).to(dev)
+            o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale)
+            fn = lambda: vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk,  # noqa: E731
+                                                     scale=c.scale, out=o)
+    elif args.profile == "ragged":
+        c = W.cfg_ragged()
+        q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
+        cu = torch.from_numpy(c.cu_seqlens).to(dev)
+        o = vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale)
+        fn = lambda: vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale, out=o)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown profile case {args.profile}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = timed(fn, args.steps, st)
+    print(json.dumps({"profile": args.profile, "ms": ts}), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", default=None,
+                    help="run one small case for an ncu capture: wan13b, wan14b, merge, select, sparse9, "
+                         "sparse144, ragged")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-mode timings")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.profile:
+        return run_profile(args)
+    try:
+        return run_ours(args)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -285,6 +285,40 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float* v) {
   }
 }
 
+// 32 fp32 values stored as two bf16-sized rows: the high 16 bits of each value
+// at `hi`, the low 16 bits at `lo` (64 bytes each, 16-byte aligned).
+__device__ __forceinline__ void store_split32(__nv_bfloat16* hi, __nv_bfloat16* lo, const uint32_t* v) {
+  uint4* h4 = reinterpret_cast<uint4*>(hi);
+  uint4* l4 = reinterpret_cast<uint4*>(lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t a = v[8 * q + 2 * e], b = v[8 * q + 2 * e + 1];
+      hw[e] = (b & 0xFFFF0000u) | (a >> 16);
+      lw[e] = (b << 16) | (a & 0xFFFFu);
+    }
+    h4[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    l4[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+__device__ __forceinline__ void load_split32(const __nv_bfloat16* hi, const __nv_bfloat16* lo, float* v) {
+  const uint4* h4 = reinterpret_cast<const uint4*>(hi);
+  const uint4* l4 = reinterpret_cast<const uint4*>(lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 H = h4[q], L = l4[q];
+    const uint32_t hw[4] = {H.x, H.y, H.z, H.w}, lw[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = __uint_as_float((hw[e] << 16) | (lw[e] & 0xFFFFu));
+      v[8 * q + 2 * e + 1] = __uint_as_float((hw[e] & 0xFFFF0000u) | (lw[e] >> 16));
+    }
+  }
+}
+
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Register split between the producer/MMA warpgroup and the two softmax
@@ -664,6 +698,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             const float inv = has ? 1.f / l_prev : 0.f;
             __nv_bfloat16* orow = p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
                                   (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch];
+            const bool split_prev = p.om != nullptr && p.n_branches == 2 && !sparse && !ragged;
+            __nv_bfloat16* mrow_split =
+                split_prev ? p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t v[32];
@@ -672,7 +709,15 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               reg_fence<32>(v);
 #pragma unroll
               for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
-              if (row_ok) store_row32(orow + c0, reinterpret_cast<const float*>(v));
+              if (row_ok) {
+                if (split_prev) {
+                  // keep the exact fp32 partial for the merge: high halves in the merged
+                  // row, low halves in this branch's row; both rows are rewritten at the end
+                  store_split32(mrow_split + c0, orow + c0, v);
+                } else {
+                  store_row32(orow + c0, reinterpret_cast<const float*>(v));
+                }
+              }
             }
             if (row_ok)
               p.lse[prev_branch][(size_t)u.s * p.Lq + qrow] =
@@ -719,9 +764,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           __nv_bfloat16* mrow =
               do_merge ? p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh : nullptr;
           const __nv_bfloat16* prow =
-              has_prev ? p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
-                             (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch]
-                       : nullptr;
+              prev_branch >= 0 ? p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
+                                     (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch]
+                               : nullptr;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t v[32];
@@ -735,8 +780,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               store_row32(orow + c0, f);
               if (do_merge) {
                 float g[32];
-                if (has_prev) {
-                  load_row32(prow + c0, g);
+                if (prev_branch >= 0) {
+                  // exact fp32 partial of the earlier branch, stored split at its close
+                  load_split32(mrow + c0, prow + c0, g);
+                  store_row32(const_cast<__nv_bfloat16*>(prow) + c0, g);
 #pragma unroll
                   for (int e = 0; e < 32; ++e) g[e] = c_last * f[e] + c_prev * g[e];
                 } else {
