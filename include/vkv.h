@@ -201,6 +201,29 @@ size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t
 vkv_status vkv_block_select(const vkv_select_args* args, vkv_stream_t stream);
 
 /*
+ * vkv_block_select_noalloc -- vkv_block_select for callers that cannot allocate.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory when they call in (for example a
+ * serving loop whose device memory is fully planned at start-up and that
+ * gives the library no allocator, or a host program that drives the library
+ * through this C interface alone and cannot size and own a workspace).
+ *
+ * Same arguments, results and errors as vkv_block_select, except that
+ * `workspace` / `workspace_bytes` are ignored: the pooled block vectors go to
+ * a fixed scratch array inside the library, VKV_NOALLOC_SCRATCH_BYTES in size,
+ * which every GPU that loads the library holds until the process exits.
+ * Requests whose vkv_block_select_workspace_size() exceeds that size return
+ * VKV_ERR_WORKSPACE.  The call allocates nothing (no cudaMalloc / cudaFree).
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls on a device share the array and leave the last call's
+ * contents in it; calls that overlap on the GPU (e.g. on two streams at once)
+ * race on it.  Nothing in it needs clearing between calls.
+ */
+#define VKV_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+vkv_status vkv_block_select_noalloc(const vkv_select_args* args, vkv_stream_t stream);
+
+/*
  * vkv_lse_merge -- exact recombination of two partial attentions over disjoint
  * key sets (ISPA summary, section 2 step 1 and contribution 2):
  *   M = max(lse_a, lse_b),  w_x = exp(lse_x - M),

@@ -15,6 +15,7 @@
 //                   iff fewer than K blocks beat it (higher score, or equal score
 //                   and lower index); kept blocks are written in ascending order.
 #include <algorithm>
+#include <mutex>
 
 #include "vkv_internal.h"
 #include "vkv_ptx.cuh"
@@ -196,6 +197,111 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   pp.n_win = a->n_win_blk;
   pp.win_row0 = a->window_blk0 * a->block;
   pp.qbar = reinterpret_cast<float*>(a->workspace);
+  pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
+  dim3 pg(n_qblk + a->n_win_blk, BH);
+  if (a->d == 128)
+    pool_kernel<128><<<pg, 128, 0, st>>>(pp);
+  else
+    pool_kernel<64><<<pg, 128, 0, st>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  SelParams sp;
+  sp.qbar = pp.qbar;
+  sp.kbar = pp.kbar;
+  sp.BH = BH;
+  sp.n_qblk = n_qblk;
+  sp.n_win = a->n_win_blk;
+  sp.topk = a->topk;
+  sp.out_idx = a->out_idx;
+  sp.out_scores = a->out_scores;
+  const long long tasks = (long long)BH * n_qblk;
+  const int grid = (int)((tasks + 7) / 8);
+  const size_t smem = (size_t)8 * a->n_win_blk * sizeof(float);
+  if (a->d == 128)
+    select_kernel<128><<<grid, 256, smem, st>>>(sp);
+  else
+    select_kernel<64><<<grid, 256, smem, st>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  return VKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// vkv_block_select_noalloc: the same selection with library-owned scratch.
+//
+// Some callers cannot allocate device memory when they call in: a serving
+// loop whose device memory was fully planned at start-up and that hands the
+// library no allocator, or a host program that drives the library only
+// through this C interface and has no way to size, own and free a workspace.
+// For them the pooled block vectors live in one file-scope device array of
+// fixed size, kNoallocScratchBytes, which every GPU that loads the library
+// holds until the process exits.
+//
+// In host code `g_select_scratch` is only a host-side stand-in for the array;
+// its device address is looked up once per device (cudaGetSymbolAddress, with
+// that device current) on the first call made on it, and cached.  Every call
+// on a device shares the array and leaves the last call's contents behind;
+// nothing needs clearing, because every element the select kernel reads is
+// written by the pool kernel of the same call.  Calls that overlap on the GPU
+// (for example on two streams at once) race on the array.
+// ---------------------------------------------------------------------------
+namespace vkv {
+namespace {
+
+constexpr size_t kNoallocScratchBytes = VKV_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) float g_select_scratch[kNoallocScratchBytes / sizeof(float)];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+
+// Device address of the scratch array on the current device; nullptr on failure.
+void* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace vkv
+
+extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_stream_t stream) {
+  if (!a) return VKV_ERR_NULL;
+  if (a->d != 64 && a->d != 128) return VKV_ERR_UNSUPPORTED;
+  if (a->block != 64) return VKV_ERR_UNSUPPORTED;
+  if (a->B <= 0 || a->H <= 0 || a->Lq <= 0 || a->Lkv <= 0) return VKV_ERR_SHAPE;
+  if (a->n_win_blk < 1 || a->n_win_blk > 1024 || a->topk < 1 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
+  if (a->window_blk0 < 0 || (long long)(a->window_blk0 + a->n_win_blk) * a->block > a->Lkv) return VKV_ERR_RANGE;
+  if (!a->q.ptr || !a->k.ptr || !a->out_idx) return VKV_ERR_NULL;
+  if (!tensor_aligned(a->q) || !tensor_aligned(a->k)) return VKV_ERR_ALIGN;
+  if ((long long)a->B * a->H > 65535) return VKV_ERR_UNSUPPORTED;
+  const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
+  if (need > kNoallocScratchBytes) return VKV_ERR_WORKSPACE;  // larger than the fixed scratch array
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
+  void* scratch = noalloc_scratch(dev);
+  if (!scratch) return VKV_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = a->B * a->H;
+  const int n_qblk = (a->Lq + 63) / 64;
+  PoolParams pp;
+  pp.q = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
+  pp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
+  pp.q_sb = a->q.sb; pp.q_st = a->q.st; pp.q_sh = a->q.sh;
+  pp.k_sb = a->k.sb; pp.k_st = a->k.st; pp.k_sh = a->k.sh;
+  pp.B = a->B;
+  pp.H = a->H;
+  pp.d = a->d;
+  pp.Lq = a->Lq;
+  pp.n_qblk = n_qblk;
+  pp.n_win = a->n_win_blk;
+  pp.win_row0 = a->window_blk0 * a->block;
+  pp.qbar = reinterpret_cast<float*>(scratch);
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
   dim3 pg(n_qblk + a->n_win_blk, BH);
   if (a->d == 128)

@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvkv.so")
 MODE_SEGMENTS, MODE_BLOCK_SPARSE, MODE_RAGGED = 0, 1, 2
 MAX_BRANCHES, MAX_SEGMENTS = 2, 8
 DEVERR_TIMEOUT, DEVERR_BAD_INDEX, DEVERR_BAD_OFFSETS = 1, 2, 3
+NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024  # VKV_NOALLOC_SCRATCH_BYTES in include/vkv.h
 STATUS = {0: "VKV_OK", 1: "VKV_ERR_NULL", 2: "VKV_ERR_SHAPE", 3: "VKV_ERR_ALIGN", 4: "VKV_ERR_RANGE",
           5: "VKV_ERR_UNSUPPORTED", 6: "VKV_ERR_CUDA", 7: "VKV_ERR_WORKSPACE"}
 
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
     L.vkv_chunk_attn.restype = c_int32
     L.vkv_block_select.argtypes = [POINTER(vkv_select_args), c_void_p]
     L.vkv_block_select.restype = c_int32
+    L.vkv_block_select_noalloc.argtypes = [POINTER(vkv_select_args), c_void_p]
+    L.vkv_block_select_noalloc.restype = c_int32
     L.vkv_block_select_workspace_size.argtypes = [c_int32] * 6
     L.vkv_block_select_workspace_size.restype = c_size_t
     L.vkv_lse_merge.argtypes = [vkv_tensor, c_void_p, vkv_tensor, c_void_p, vkv_tensor, c_void_p,
@@ -120,6 +123,11 @@ def vkv_chunk_attn(args: vkv_attn_args, stream: int | None) -> int:
 
 def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
     return int(lib().vkv_block_select(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_block_select_noalloc(args: vkv_select_args, stream: int | None) -> int:
+    """vkv_block_select with the library's own fixed scratch array (no workspace argument)."""
+    return int(lib().vkv_block_select_noalloc(ctypes.byref(args), c_void_p(stream or 0)))
 
 
 def vkv_block_select_workspace_size(B, H, Lq, n_win_blk, block, d) -> int:
