@@ -107,14 +107,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the attention kernel's sources (ties recorded ncu counters to a kernel version)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_attention_chunk_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as fh:
-                h.update(name.encode() + fh.read())
+    for name in ATTN_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
 
 

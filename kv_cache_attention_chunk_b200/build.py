@@ -51,9 +51,9 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str, verbose: bool) -> tuple[str, str]:
-    obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, defines=(), tag: str = "") -> tuple[str, str]:
+    obj = os.path.join(BUILD, tag + os.path.basename(src).replace(".cu", ".o"))
+    cmd = [nvcc(), *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     log = r.stdout + r.stderr
     if r.returncode != 0:
@@ -63,24 +63,29 @@ def _compile(src: str, verbose: bool) -> tuple[str, str]:
     return obj, log
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link libvkv.so; returns its path."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
+    """Compile every CUDA source for sm_100a and link libvkv.so; returns its path.
+
+    `out` / `defines` build a variant library (extra -D macros) at another path.
+    """
+    target = out or LIB
+    if not force and out is None and not defines and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
+    tag = "" if out is None else os.path.basename(out).replace(".so", "") + "_"
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), _sources()))
+        results = list(ex.map(lambda s: _compile(s, verbose, defines, tag), _sources()))
     objs = [o for o, _ in results]
-    with open(os.path.join(BUILD, "ptxas.log"), "w") as fh:
+    with open(os.path.join(BUILD, tag + "ptxas.log"), "w") as fh:
         for o, log in results:
             fh.write(f"== {os.path.basename(o)}\n{log}\n")
-    tmp = LIB + ".tmp"
+    tmp = target + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lrt", "-ldl", "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n" + r.stdout + r.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

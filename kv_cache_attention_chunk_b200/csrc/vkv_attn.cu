@@ -249,6 +249,7 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
         P->flat_len[nf] = sg.len;
         P->flat_branch[nf] = br;
         P->flat_first[nf] = first ? 1 : 0;
+        P->flat_step0[nf] = total + steps;
         first = false;
         steps += (sg.len + 127) / 128;
         ++nf;
@@ -359,3 +360,15 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }
+
+#ifdef VKV_TRACE
+// Development only (not in the public header): copy CTA 0's pipeline timeline.
+extern "C" int vkv_debug_trace(void* dst, size_t bytes) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(dst, vkv::g_vkv_trace, bytes < sizeof(vkv::g_vkv_trace) ? bytes : sizeof(vkv::g_vkv_trace));
+}
+extern "C" int vkv_debug_trace_clear() {
+  static unsigned long long zeros[2 * 28672];
+  return (int)cudaMemcpyToSymbol(vkv::g_vkv_trace, zeros, sizeof(zeros));
+}
+#endif

@@ -24,8 +24,12 @@
 //   warps 8-11   softmax + epilogue for query tile 1.
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
-// P (bf16) is written by the softmax threads to shared memory in the same
-// 128-byte-swizzled K-major layout TMA produces, and read by the PV MMA.
+// The softmax threads read S_t, then write P_t (bf16, two per 32-bit column)
+// over the first 64 columns of S_t; the PV MMA reads P_t from TMEM (A operand)
+// and V from shared memory.  Per tile the MMA thread issues O_t += P_t(j) V_j
+// before S_t(j+1) = Q_t K_{j+1}^T, so P_t(j) is consumed before S_t is
+// overwritten (tcgen05.mma ops of one thread execute in issue order).
+// Keeping P out of shared memory leaves room for a 5-slot K/V ring (d = 128).
 // The online softmax works in log2 units (s * scale * log2 e) and rescales the
 // O accumulator only when a row maximum grows by more than 2^8; the final
 // O / l and LSE do not depend on the reference maximum.
@@ -41,12 +45,10 @@ struct AttnCfg {
   static constexpr int NAC = D / 64;               // 128-byte atom columns along d
   static constexpr int ATOM = 128 * 128;            // bytes of one 128-row atom column
   static constexpr int QT_BYTES = 128 * D * 2;      // one 128-row Q tile
-  static constexpr int P_BYTES = 128 * 128 * 2;     // one P tile (128 rows x 128 keys)
   static constexpr int KV_BYTES = 128 * D * 2;      // one K or V tile (128 keys)
-  static constexpr int NSLOT = (D == 128) ? 3 : 6;  // K/V ring slots
+  static constexpr int NSLOT = (D == 128) ? 5 : 8;  // K/V ring slots
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = OFF_Q + 2 * QT_BYTES;
-  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_KV = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_CTL = OFF_KV + NSLOT * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_CTL + kCtlBytes + 1024;  // + base alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
@@ -54,12 +56,14 @@ struct AttnCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+constexpr int kMaxSlots = 8;
+
 // Control block (barriers, block list) at the end of shared memory.
 struct Ctl {
-  uint64_t full[6];
-  uint64_t empty[6];
+  uint64_t full[kMaxSlots];
+  uint64_t empty[kMaxSlots];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t list_ready, list_free, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -319,14 +323,61 @@ __device__ __forceinline__ void load_split32(const __nv_bfloat16* hi, const __nv
   }
 }
 
+// Optional exp2 on the FMA pipe for part of the columns, to unload the MUFU
+// pipe (one exponential per score; MUFU and the tensor pipe are co-critical).
+// Measured on B200 with this kernel it does not pay (the per-row softmax is
+// latency-bound rather than MUFU-bound), so it is compiled out by default.  2^x = 2^r * q(f) with r = round(x) taken by the 1.5*2^23 rounding
+// trick and f = x - r in [-1/2, 1/2]; q is a cubic fitted here to 2^f by
+// relative-error minimax (max relative error 7.5e-5, far below the 2^-9
+// rounding of P to bf16); 2^r is added into the exponent field as an integer.
+// Arguments below -125 give exactly 0 (masked scores are -inf).
+#ifndef VKV_EXP_EMU16
+#define VKV_EXP_EMU16 0
+#endif
+constexpr int kExpEmu16 = VKV_EXP_EMU16;
+
+// Development timeline (compiled only with -DVKV_TRACE): SM clock stamps of the
+// pipeline events of CTA 0, read back with vkv_debug_trace().
+#ifdef VKV_TRACE
+__device__ unsigned long long g_vkv_trace[2 * 28672];
+#define VKV_STAMP(idx)                                                        \
+  do {                                                                        \
+    const int i_ = (idx);                                                     \
+    if (blockIdx.x == 0 && i_ >= 0 && i_ < 28672) {                           \
+      g_vkv_trace[i_] = clock64();                                            \
+      g_vkv_trace[28672 + i_] = globaltimer();                                \
+    }                                                                         \
+  } while (0)
+#else
+#define VKV_STAMP(idx) \
+  do {                 \
+  } while (0)
+#endif
+// 2^x for a pair of arguments (x <= 8).  Arguments below -126 give a value of
+// at most 2^-126 (masked scores are -inf), which no output can resolve.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float& e1) {
+  const uint64_t xc = pack2f(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = pack2f(12582912.f, 12582912.f);
+  const uint64_t t = add2f(xc, magic);
+  const uint64_t f = sub2f(xc, sub2f(t, magic));
+  uint64_t q = fma2f(pack2f(0.0551716685f, 0.0551716685f), f, pack2f(0.242611140f, 0.242611140f));
+  q = fma2f(q, f, pack2f(0.693260968f, 0.693260968f));
+  q = fma2f(q, f, pack2f(0.999928057f, 0.999928057f));
+  float q0, q1, t0, t1;
+  unpack2f(q, q0, q1);
+  unpack2f(t, t0, t1);
+  e0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
+  e1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
+}
+
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Register split between the producer/MMA warpgroup and the two softmax
 // warpgroups.  setmaxnreg.inc only succeeds if the total stays within what the
 // CTA was launched with (384 threads x 168 registers); the host checks the
 // compiled register count against kRegsLaunchNeeded before every launch.
-constexpr int kRegsProducer = 104;
-constexpr int kRegsSoftmax = 200;
+constexpr int kRegsProducer = 88;
+constexpr int kRegsSoftmax = 208;
 constexpr int kRegsLaunchNeeded = (128 * kRegsProducer + 256 * kRegsSoftmax + 383) / 384;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= 384 * 168, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -342,7 +393,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::OFF_CTL);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::OFF_Q;
-  const uint32_t sP = sbase + C::OFF_P;
   const uint32_t sKV = sbase + C::OFF_KV;
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
@@ -352,7 +402,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   const uint32_t b_qfull = smem_u32(&ctl->q_full);
   const uint32_t b_qempty = smem_u32(&ctl->q_empty);
   const uint32_t b_sfull0 = smem_u32(&ctl->s_full[0]);
-  const uint32_t b_sfree0 = smem_u32(&ctl->s_free[0]);
   const uint32_t b_pfull0 = smem_u32(&ctl->p_full[0]);
   const uint32_t b_odone0 = smem_u32(&ctl->o_done[0]);
   const uint32_t b_lready = smem_u32(&ctl->list_ready);
@@ -368,7 +417,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     mbar_init(b_qempty, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(b_sfull0 + 8 * t, 1);
-      mbar_init(b_sfree0 + 8 * t, 4);
       mbar_init(b_pfull0 + 8 * t, 4);
       mbar_init(b_odone0 + 8 * t, 1);
     }
@@ -441,6 +489,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               const uint32_t slot = item % C::NSLOT, use = item / C::NSLOT;
               if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
               if (!ok) break;
+              VKV_STAMP(20480 + (int)item);
               mbar_arrive_expect_tx(b_full0 + 8 * slot, (uint32_t)C::KV_BYTES);
               const CUtensorMap* tm = kv ? &p.tm_v : &p.tm_k;
               const uint32_t dst = sKV + slot * C::KV_BYTES;
@@ -466,12 +515,28 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
+      // Per step j and tile t: O_t += P_t(j) V_j (A = P_t from TMEM), then
+      // S_t(j+1) = Q_t K_{j+1}^T; each after a suspending wait on its inputs.
       if (lane == 0) {
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
         uint32_t item = 0, qcnt = 0, ucnt = 0;
-        uint32_t qk_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+        uint32_t pv_cnt[2] = {0, 0};
         bool ok = true;
+        auto wait_item = [&](uint32_t it_) {
+          return mbar_wait(b_full0 + 8 * (it_ % C::NSLOT), (it_ / C::NSLOT) & 1, abort_flag, p.err);
+        };
+        auto issue_qk = [&](int t, uint32_t kslot) {
+          const uint32_t d_tm = tmem + (uint32_t)(t * 128);
+          const uint32_t qa = sQ + t * C::QT_BYTES;
+          const uint32_t kb = sKV + kslot * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+            mma_bf16_ss(d_tm, sdesc_k_sw128(qa + off), sdesc_k_sw128(kb + off), IDESC_QK, kk > 0);
+          }
+          mma_commit(b_sfull0 + 8 * t);
+        };
         for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
           const UnitInfo u = decode_unit(p, p.units[ui]);
           int rs = 0, rl = 0;
@@ -489,28 +554,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ok = mbar_wait(b_qfull, qcnt & 1, abort_flag, p.err);
           ++qcnt;
           if (!ok) break;
-          // prologue: S_t = Q_t K_0^T
-          ok = mbar_wait(b_full0 + 8 * (item % C::NSLOT), (item / C::NSLOT) & 1, abort_flag, p.err);
+          // prologue: S_t(0) = Q_t K_0^T
+          ok = wait_item(item);
           if (!ok) break;
           tc_fence_after();
-          for (int t = 0; t < u.ntiles && ok; ++t) {
-            if (qk_cnt[t] > 0) {
-              ok = mbar_wait(b_sfree0 + 8 * t, (qk_cnt[t] - 1) & 1, abort_flag, p.err);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            const uint32_t d_tm = tmem + (uint32_t)(t * 128);
-            const uint32_t qa = sQ + t * C::QT_BYTES;
-            const uint32_t kb = sKV + (item % C::NSLOT) * C::KV_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
-              mma_bf16_ss(d_tm, sdesc_k_sw128(qa + off), sdesc_k_sw128(kb + off), IDESC_QK, kk > 0);
-            }
-            mma_commit(b_sfull0 + 8 * t);
-            ++qk_cnt[t];
-          }
-          if (!ok) break;
+          for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % C::NSLOT);
           mma_commit(b_empty0 + 8 * (item % C::NSLOT));
           if (nsteps == 1) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
@@ -518,53 +566,46 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             const uint32_t vit = item + 2 * j + 1;
             const uint32_t knext = item + 2 * j + 2;
             const bool has_next = j + 1 < nsteps;
-            if (has_next) {
-              ok = mbar_wait(b_full0 + 8 * (knext % C::NSLOT), (knext / C::NSLOT) & 1, abort_flag, p.err);
-              if (!ok) break;
-            }
-            ok = mbar_wait(b_full0 + 8 * (vit % C::NSLOT), (vit / C::NSLOT) & 1, abort_flag, p.err);
+            const int trm = (pv_cnt[0] < 256) ? 16384 + (int)(pv_cnt[0]) * 16 : -100;
+            ok = wait_item(vit);
             if (!ok) break;
-            tc_fence_after();
+            VKV_STAMP(trm);
+            bool k_ready = false;
             for (int t = 0; t < u.ntiles && ok; ++t) {
-              if (has_next) {
-                ok = mbar_wait(b_sfree0 + 8 * t, (qk_cnt[t] - 1) & 1, abort_flag, p.err);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t d_tm = tmem + (uint32_t)(t * 128);
-                const uint32_t qa = sQ + t * C::QT_BYTES;
-                const uint32_t kb = sKV + (knext % C::NSLOT) * C::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t off = (kk >> 2) * C::ATOM + (kk & 3) * 32;
-                  mma_bf16_ss(d_tm, sdesc_k_sw128(qa + off), sdesc_k_sw128(kb + off), IDESC_QK,
-                              kk > 0);
-                }
-                mma_commit(b_sfull0 + 8 * t);
-                ++qk_cnt[t];
-              }
               ok = mbar_wait(b_pfull0 + 8 * t, pv_cnt[t] & 1, abort_flag, p.err);
               if (!ok) break;
+              VKV_STAMP(trm + 1 + 4 * t);
               tc_fence_after();
               {
                 const uint32_t d_tm = tmem + C::TM_O + (uint32_t)(t * D);
-                const uint32_t pa = sP + t * C::P_BYTES;
+                const uint32_t pa = tmem + (uint32_t)(t * 128);
                 const uint32_t vb = sKV + (vit % C::NSLOT) * C::KV_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                  const uint32_t aoff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
-                  mma_bf16_ss(d_tm, sdesc_k_sw128(pa + aoff), sdesc_mn_sw128(vb + kk * 2048, C::ATOM),
-                              IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                  mma_bf16_ts(d_tm, pa + 8 * kk, sdesc_mn_sw128(vb + kk * 2048, C::ATOM), IDESC_PV,
+                              (!first || kk > 0) ? 1u : 0u);
               }
               mma_commit(b_odone0 + 8 * t);
+              VKV_STAMP(trm + 2 + 4 * t);
               ++pv_cnt[t];
+              if (has_next) {
+                if (!k_ready) {
+                  ok = wait_item(knext);
+                  if (!ok) break;
+                  tc_fence_after();
+                  k_ready = true;
+                  VKV_STAMP(trm + 3 + 4 * t);
+                }
+                issue_qk(t, knext % C::NSLOT);
+                VKV_STAMP(trm + 4 + 4 * t);
+              }
             }
             if (!ok) break;
+            mma_commit(b_empty0 + 8 * (vit % C::NSLOT));
             if (has_next) {
               mma_commit(b_empty0 + 8 * (knext % C::NSLOT));
               if (j + 2 == nsteps) mma_commit(b_qempty);
             }
-            mma_commit(b_empty0 + 8 * (vit % C::NSLOT));
           }
           item += 2 * nsteps;
         }
@@ -583,8 +624,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
     const uint32_t tO = tmem + lane_base + C::TM_O + (uint32_t)(t * D);
-    const uint32_t sPt = sP + t * C::P_BYTES;
-    const uint32_t b_sfull = b_sfull0 + 8 * t, b_sfree = b_sfree0 + 8 * t;
+    const uint32_t b_sfull = b_sfull0 + 8 * t;
     const uint32_t b_pfull = b_pfull0 + 8 * t, b_odone = b_odone0 + 8 * t;
     const float sl2 = p.scale_log2;
     uint32_t sf_cnt = 0, np = 0, ucnt = 0;
@@ -611,7 +651,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         it.init(&p, ctl, rs, rl);
         for (int j = 0; j < nsteps; ++j) {
           const TileDesc td = it.next();
+          const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
+          VKV_STAMP(tr);
           ok = warp_all(mbar_wait(b_sfull, sf_cnt & 1, abort_flag, p.err));
+          VKV_STAMP(tr < 0 ? -1 : tr + 1);
           ++sf_cnt;
           if (!ok) break;
           tc_fence_after();
@@ -622,9 +665,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           tmem_ld32(tS + 96, sr + 96);
           tmem_ld_wait();
           reg_fence<128>(sr);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(b_sfree);
+          VKV_STAMP(tr < 0 ? -1 : tr + 2);
           bool pending_epi = false;
           if (td.first) {
             if (cur_branch >= 0) {
@@ -649,12 +690,20 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           }
           float mx8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+          for (int i = 0; i < 8; ++i) mx8[i] = max3f(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
+                                                     __uint_as_float(sr[16 + i]));
 #pragma unroll
-          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          for (int c = 24; c < 120; c += 16) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              mx8[i] = max3f(mx8[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], __uint_as_float(sr[120 + i]));
+          const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7]));
           const float mt = mx * sl2;
+          VKV_STAMP(tr < 0 ? -1 : tr + 6);
           float alpha = 1.f;
           bool rescale = false;
           if (m == -INFINITY) {
@@ -665,33 +714,48 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             rescale = true;
           }
           const float mu = (m == -INFINITY) ? 0.f : m;
-          float sm8[8];
+          // p = 2^(s * scale * log2 e - m): pairs on the f32x2 path, kExpEmu16 of every
+          // 16 columns on the FMA pipe, the rest on MUFU; P (bf16 pairs) -> the first
+          // 64 TMEM columns of S_t, 32 columns at a time
+          const uint64_t sl2x2 = pack2f(sl2, sl2), nmu2 = pack2f(-mu, -mu);
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) sm8[i] = 0.f;
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float e = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -mu));
-            sr[c] = __float_as_uint(e);
-            sm8[c & 7] += e;
-          }
-          l = l * alpha + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
-          // the previous PV of this tile must be done: P buffer free, O final
-          if (np > 0) {
-            ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
-            if (!ok) break;
-            tc_fence_after();
-          }
-          // P (bf16) -> shared memory, 128-byte swizzled K-major
+            for (int g = 0; g < 64; g += 16) {
+              const int c0 = h * 64 + g;
+              float a[16], e[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t addr =
-                sPt + (uint32_t)((c >> 3) * C::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-            st_shared_v4(addr,
-                         pack_bf16x2(__uint_as_float(sr[8 * c + 0]), __uint_as_float(sr[8 * c + 1])),
-                         pack_bf16x2(__uint_as_float(sr[8 * c + 2]), __uint_as_float(sr[8 * c + 3])),
-                         pack_bf16x2(__uint_as_float(sr[8 * c + 4]), __uint_as_float(sr[8 * c + 5])),
-                         pack_bf16x2(__uint_as_float(sr[8 * c + 6]), __uint_as_float(sr[8 * c + 7])));
+              for (int i = 0; i < 16; i += 2)
+                unpack2f(fma2f(pack2f(__uint_as_float(sr[c0 + i]), __uint_as_float(sr[c0 + i + 1])), sl2x2, nmu2),
+                         a[i], a[i + 1]);
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                if (i >= 16 - kExpEmu16) {
+                  exp2_poly2(a[i], a[i + 1], e[i], e[i + 1]);
+                } else {
+                  e[i] = ex2_approx(a[i]);
+                  e[i + 1] = ex2_approx(a[i + 1]);
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                acc2[(i >> 1) & 3] = add2f(acc2[(i >> 1) & 3], pack2f(e[i], e[i + 1]));
+                pk[(g + i) >> 1] = pack_bf16x2(e[i], e[i + 1]);
+              }
+            }
+            tmem_st32(tS + (uint32_t)(h * 32), pk);
+            VKV_STAMP(tr < 0 ? -1 : tr + 7 + h);
           }
+          float sum_lo, sum_hi;
+          unpack2f(add2f(add2f(acc2[0], acc2[1]), add2f(acc2[2], acc2[3])), sum_lo, sum_hi);
+          l = l * alpha + (sum_lo + sum_hi);
+          VKV_STAMP(tr < 0 ? -1 : tr + 3);
+          // O_t already holds every PV up to step j-1: S_t(j) was committed after
+          // O_t += P_t(j-1) V_{j-1}, and a commit covers all earlier MMAs.
+          const bool need_o = pending_epi || __any_sync(0xFFFFFFFFu, rescale);
+          VKV_STAMP(tr < 0 ? -1 : tr + 4);
           if (pending_epi) {
             // close the previous branch: O / l and LSE
             const bool has = l_prev > 0.f;
@@ -722,7 +786,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             if (row_ok)
               p.lse[prev_branch][(size_t)u.s * p.Lq + qrow] =
                   has ? (m_prev + lg2_approx(l_prev)) * kLn2 : -INFINITY;
-          } else if (__any_sync(0xFFFFFFFFu, rescale)) {
+          } else if (need_o) {
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t v[32];
@@ -733,11 +797,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
               tmem_st32(tO + c0, v);
             }
-            tmem_st_wait();
           }
-          fence_proxy_async_smem();
+          tmem_st_wait();
           tc_fence_before();
           __syncwarp();
+          VKV_STAMP(tr < 0 ? -1 : tr + 5);
           if (lane == 0) mbar_arrive(b_pfull);
           ++np;
         }

@@ -32,6 +32,7 @@ struct AttnParams {
   int flat_len[kMaxFlatSegs];
   int flat_branch[kMaxFlatSegs];
   int flat_first[kMaxFlatSegs];
+  int flat_step0[kMaxFlatSegs];  // first key-tile step of each flat segment
   // BLOCK_SPARSE
   int n_persist, topk, window_blk0, n_win_blk, n_qblk, n_blocks_total;
   const int* persist_idx;

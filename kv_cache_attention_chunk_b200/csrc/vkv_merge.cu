@@ -3,9 +3,9 @@
 // branch outputs tracked with their log-sum-exp, merged by online softmax).
 //
 // Bandwidth-bound: every output row reads 2 x d bf16 + 2 fp32 and writes
-// d bf16 + 1 fp32.  One thread handles 8 features (one 16-byte vector) of a
-// row; consecutive threads cover consecutive 16-byte chunks of the
-// [B, Lq, H, d] tensors, so loads and stores are fully coalesced.
+// d bf16 + 1 fp32.  A thread handles 16-byte chunks (8 features) of rows;
+// consecutive threads cover consecutive chunks of the [B, Lq, H, d] tensors,
+// so loads and stores are fully coalesced.
 #include "vkv_internal.h"
 #include "vkv_ptx.cuh"
 
@@ -24,44 +24,68 @@ struct MergeParams {
   long long n_chunks;  // B * Lq * H * (d / 8)
 };
 
+constexpr int kMergePos = 8;  // consecutive (b, i) query positions per thread
+
+// grid: x = ceil(B * Lq / kMergePos) position groups, y = ceil(H * d/8 / 256) column blocks.
+// Thread: one 16-byte column (head h, chunk ch) of kMergePos consecutive query
+// positions; all its loads are issued before the first merge, and the index
+// of the next position is advanced without division.  The output may alias an
+// input (in-place merge): each chunk is read before it is written, by the same
+// thread.
+template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeParams p) {
-  const int cpr = p.d >> 3;  // 16-byte chunks per row
-  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < p.n_chunks;
-       t += (long long)gridDim.x * blockDim.x) {
-    const long long row = t / cpr;
-    const int ch = (int)(t - row * cpr);
-    const int h = (int)(row % p.H);
-    const long long bi = row / p.H;
-    const int i = (int)(bi % p.Lq);
-    const int b = (int)(bi / p.Lq);
-    const size_t li = ((size_t)b * p.H + h) * p.Lq + i;
-    const float la = __ldg(p.la + li);
-    const float lb = __ldg(p.lb + li);
-    const float M = fmaxf(la, lb);
+  constexpr int CPR = D / 8;
+  const int col = blockIdx.y * blockDim.x + threadIdx.x;
+  if (col >= p.H * CPR) return;
+  const int h = col / CPR, ch = col % CPR;
+  const int pos0 = blockIdx.x * kMergePos;
+  const int n_pos = p.B * p.Lq;
+  int b = pos0 / p.Lq, i = pos0 - (pos0 / p.Lq) * p.Lq;
+  uint4 va[kMergePos], vb[kMergePos];
+  float la[kMergePos], lb[kMergePos];
+  int bb[kMergePos], ii[kMergePos];
+#pragma unroll
+  for (int k = 0; k < kMergePos; ++k) {
+    bb[k] = b;
+    ii[k] = i;
+    if (pos0 + k < n_pos) {
+      const size_t li = ((size_t)b * p.H + h) * p.Lq + i;
+      va[k] = __ldcs(reinterpret_cast<const uint4*>(p.oa + b * p.a_sb + (long long)i * p.a_st + h * p.a_sh) + ch);
+      vb[k] = __ldcs(reinterpret_cast<const uint4*>(p.ob + b * p.b_sb + (long long)i * p.b_st + h * p.b_sh) + ch);
+      la[k] = __ldg(p.la + li);
+      lb[k] = __ldg(p.lb + li);
+    }
+    if (++i == p.Lq) {
+      i = 0;
+      ++b;
+    }
+  }
+  constexpr float kLog2e = 1.4426950408889634f;
+#pragma unroll
+  for (int k = 0; k < kMergePos; ++k) {
+    if (pos0 + k >= n_pos) break;
+    const float M = fmaxf(la[k], lb[k]);
     const bool empty = (M == -INFINITY);
     const float Ms = empty ? 0.f : M;
-    constexpr float kLog2e = 1.4426950408889634f;
-    const float wa = ex2_approx((la - Ms) * kLog2e);
-    const float wb = ex2_approx((lb - Ms) * kLog2e);
+    const float wa = ex2_approx((la[k] - Ms) * kLog2e);
+    const float wb = ex2_approx((lb[k] - Ms) * kLog2e);
     const float den = wa + wb;
     const float ca = empty ? 0.f : wa / den;
     const float cb = empty ? 0.f : wb / den;
-    const uint4 va = __ldcs(reinterpret_cast<const uint4*>(p.oa + b * p.a_sb + (long long)i * p.a_st +
-                                                            h * p.a_sh) + ch);
-    const uint4 vb = __ldcs(reinterpret_cast<const uint4*>(p.ob + b * p.b_sb + (long long)i * p.b_st +
-                                                            h * p.b_sh) + ch);
-    const uint32_t xa[4] = {va.x, va.y, va.z, va.w};
-    const uint32_t xb[4] = {vb.x, vb.y, vb.z, vb.w};
-    uint32_t r[4];
+    const uint32_t xa[4] = {va[k].x, va[k].y, va[k].z, va[k].w};
+    const uint32_t xb[4] = {vb[k].x, vb[k].y, vb[k].z, vb[k].w};
+    uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float a0 = __uint_as_float(xa[e] << 16), a1 = __uint_as_float(xa[e] & 0xFFFF0000u);
       const float b0 = __uint_as_float(xb[e] << 16), b1 = __uint_as_float(xb[e] & 0xFFFF0000u);
-      r[e] = pack_bf16x2(ca * a0 + cb * b0, ca * a1 + cb * b1);
+      o[e] = pack_bf16x2(ca * a0 + cb * b0, ca * a1 + cb * b1);
     }
-    __stcs(reinterpret_cast<uint4*>(p.oo + b * p.o_sb + (long long)i * p.o_st + h * p.o_sh) + ch,
-           make_uint4(r[0], r[1], r[2], r[3]));
-    if (ch == 0) p.lo[li] = empty ? -INFINITY : Ms + lg2_approx(den) * 0.6931471805599453f;
+    __stcs(reinterpret_cast<uint4*>(p.oo + bb[k] * p.o_sb + (long long)ii[k] * p.o_st + h * p.o_sh) + ch,
+           make_uint4(o[0], o[1], o[2], o[3]));
+    if (ch == 0)
+      p.lo[((size_t)bb[k] * p.H + h) * p.Lq + ii[k]] =
+          empty ? -INFINITY : Ms + lg2_approx(den) * 0.6931471805599453f;
   }
 }
 
@@ -75,7 +99,9 @@ extern "C" vkv_status vkv_lse_merge(vkv_tensor o_a, const float* lse_a, vkv_tens
                                     int32_t d, vkv_stream_t stream) {
   if (!o_a.ptr || !o_b.ptr || !o_out.ptr || !lse_a || !lse_b || !lse_out) return VKV_ERR_NULL;
   if (B <= 0 || H <= 0 || Lq <= 0) return VKV_ERR_SHAPE;
-  if (d <= 0 || d % 8 != 0 || d > 1024) return VKV_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return VKV_ERR_UNSUPPORTED;
+  if ((long long)B * Lq >= (1ll << 31) - kMergePos || (long long)H * (d / 8) >= (1ll << 31))
+    return VKV_ERR_UNSUPPORTED;
   if (!tensor_aligned(o_a) || !tensor_aligned(o_b) || !tensor_aligned(o_out)) return VKV_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(lse_a) | reinterpret_cast<uintptr_t>(lse_b) |
        reinterpret_cast<uintptr_t>(lse_out)) & 3u)
@@ -98,9 +124,14 @@ extern "C" vkv_status vkv_lse_merge(vkv_tensor o_a, const float* lse_a, vkv_tens
   p.Lq = Lq;
   p.d = d;
   p.n_chunks = (long long)B * Lq * H * (d / 8);
-  const long long want = (p.n_chunks + 255) / 256;
-  const int grid = (int)std::min<long long>(want, (long long)n_sm * 16);
-  lse_merge_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  const long long n_pos = (long long)B * Lq;
+  const dim3 grid((unsigned)((n_pos + kMergePos - 1) / kMergePos), (unsigned)((H * (d / 8) + 255) / 256));
+  if (grid.y > 65535u) return VKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    lse_merge_kernel<128><<<grid, 256, 0, st>>>(p);
+  else
+    lse_merge_kernel<64><<<grid, 256, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }

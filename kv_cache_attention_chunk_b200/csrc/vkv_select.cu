@@ -5,15 +5,17 @@
 //
 // Two kernels on the caller's stream:
 //   pool_kernel     mean of every 64-row block of Q and of the window part of K,
-//                   in fp32, written to the caller's workspace.  One CTA of 128
-//                   threads per (block, batch*head): 16 threads cover a 256-byte
-//                   row with 16-byte loads, 8 row groups of 8 rows each; the
-//                   groups are combined in shared memory.  HBM-bound.
-//   select_kernel   one warp per (batch*head, query block): scores against every
-//                   window block (coalesced reads of the pooled keys, warp
-//                   reduction), then an exact rank-based top-K: block w is kept
-//                   iff fewer than K blocks beat it (higher score, or equal score
-//                   and lower index); kept blocks are written in ascending order.
+//                   in fp32, written to the caller's workspace.  One CTA of 256
+//                   threads per (block, batch, group of 4 heads): the group's
+//                   contiguous slice of each row is read with 16-byte loads,
+//                   16 rows per thread in flight; row groups are combined in
+//                   shared memory.  HBM-bound.
+//   select_kernel   one CTA per (batch*head, 4 query blocks), one warp per query
+//                   block: pooled keys are staged in shared memory 64 blocks at a
+//                   time, each lane scores its own blocks, then an exact
+//                   rank-based top-K: block w is kept iff fewer than K blocks beat
+//                   it (higher score, or equal score and lower index); kept
+//                   blocks are written in ascending order.
 #include <algorithm>
 #include <mutex>
 
@@ -32,18 +34,28 @@ struct PoolParams {
   float* kbar;  // [B*H][n_win][d]
 };
 
-// grid: x = block index over n_qblk + n_win, y = b*H + h; 128 threads.
+constexpr int kPoolHeads = 4;  // heads per pooling CTA (a contiguous slice of each row)
+
+// grid: x = block index over n_qblk + n_win, y = b * ceil(H / kPoolHeads) + head group;
+// 256 threads.  Thread (g, c): column c = (head, 16-byte chunk) of the head
+// group's slice, rows g*RPG .. g*RPG + RPG - 1 of the 64-row block; the row
+// groups are combined in shared memory.
 template <int D>
-__global__ void __launch_bounds__(128) pool_kernel(const PoolParams p) {
-  constexpr int CPR = D / 8;        // 16-byte chunks per row
-  constexpr int GROUPS = 128 / CPR;  // row groups
-  constexpr int RPG = 64 / GROUPS;   // rows per group
-  __shared__ float part[GROUPS][D];
+__global__ void __launch_bounds__(256) pool_kernel(const PoolParams p) {
+  constexpr int CPR = D / 8;                  // 16-byte chunks per head row
+  constexpr int COLS = kPoolHeads * CPR;      // columns of the slice
+  constexpr int GROUPS = 256 / COLS;          // row groups
+  constexpr int RPG = 64 / GROUPS;            // rows per group
+  __shared__ float part[GROUPS][COLS * 8];
   const int blk = blockIdx.x;
-  const int s = blockIdx.y;
-  const int b = s / p.H, h = s - (s / p.H) * p.H;
-  const int ch = threadIdx.x % CPR;
-  const int g = threadIdx.x / CPR;
+  const int n_hg = (p.H + kPoolHeads - 1) / kPoolHeads;
+  const int b = blockIdx.y / n_hg;
+  const int h0 = (blockIdx.y - b * n_hg) * kPoolHeads;
+  const int nh = min(kPoolHeads, p.H - h0);
+  const int c = threadIdx.x % COLS;
+  const int g = threadIdx.x / COLS;
+  const int hc = c / CPR, ch = c % CPR;
+  const bool col_ok = hc < nh;
   const bool is_q = blk < p.n_qblk;
   const __nv_bfloat16* base;
   long long st;
@@ -51,24 +63,25 @@ __global__ void __launch_bounds__(128) pool_kernel(const PoolParams p) {
   if (is_q) {
     row0 = blk * 64;
     nrows = min(64, p.Lq - row0);
-    base = p.q + b * p.q_sb + h * p.q_sh;
+    base = p.q + b * p.q_sb + (h0 + hc) * p.q_sh;
     st = p.q_st;
   } else {
     row0 = p.win_row0 + (blk - p.n_qblk) * 64;
     nrows = 64;
-    base = p.k + b * p.k_sb + h * p.k_sh;
+    base = p.k + b * p.k_sb + (h0 + hc) * p.k_sh;
     st = p.k_st;
   }
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   uint4 v[RPG];
 #pragma unroll
   for (int i = 0; i < RPG; ++i) {
     const int r = g * RPG + i;
-    v[i] = (r < nrows) ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)(row0 + r) * st) + ch)
-                       : make_uint4(0, 0, 0, 0);
+    v[i] = (col_ok && r < nrows)
+               ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)(row0 + r) * st) + ch)
+               : make_uint4(0, 0, 0, 0);
   }
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
   for (int i = 0; i < RPG; ++i) {
     const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -79,16 +92,19 @@ __global__ void __launch_bounds__(128) pool_kernel(const PoolParams p) {
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[g][ch * 8 + e] = acc[e];
+  for (int e = 0; e < 8; ++e) part[g][c * 8 + e] = acc[e];
   __syncthreads();
   const float inv = 1.f / (float)nrows;
-  for (int c = threadIdx.x; c < D; c += 128) {
+  for (int x = threadIdx.x; x < COLS * 8; x += 256) {
+    const int hx = x / D, cx = x % D;
+    if (hx >= nh) continue;
     float sum = 0.f;
 #pragma unroll
-    for (int gg = 0; gg < GROUPS; ++gg) sum += part[gg][c];
+    for (int gg = 0; gg < GROUPS; ++gg) sum += part[gg][x];
+    const int s = b * p.H + h0 + hx;
     float* dst = is_q ? p.qbar + ((size_t)s * p.n_qblk + blk) * D
                       : p.kbar + ((size_t)s * p.n_win + (blk - p.n_qblk)) * D;
-    dst[c] = sum * inv;
+    dst[cx] = sum * inv;
   }
 }
 
@@ -100,57 +116,146 @@ struct SelParams {
   float* out_scores;
 };
 
-// 8 warps per CTA, one warp per (s, query block); scores staged in shared memory.
-template <int D>
-__global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
-  extern __shared__ float sc_all[];  // [8][n_win]
+constexpr int kSelWarps = 4;     // query blocks per CTA (one warp each)
+constexpr int kSelMaxSmem = (kSelWarps * 128 + 64 * 129 + kSelWarps * 1024) * 4;
+constexpr int kSelChunk = 64;    // window blocks staged in shared memory at a time
+
+// grid: x = ceil(n_qblk / kSelWarps), y = b*H + h; 128 threads.
+// Shared memory: pooled queries [kSelWarps][D], a chunk of pooled keys
+// [kSelChunk][D + 1] (padded: lane l reads row l, so rows land in distinct
+// banks) and the scores [kSelWarps][n_win].
+template <int D, int kMaxPerLane>
+__global__ void __launch_bounds__(128) select_kernel(const SelParams p) {
+  extern __shared__ float sm[];
+  float* qs = sm;                              // kSelWarps * D
+  float* ks = qs + kSelWarps * D;              // kSelChunk * (D + 1)
+  float* scs = ks + kSelChunk * (D + 1);       // kSelWarps * n_win
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * 8 + warp;
-  if (task >= (long long)p.BH * p.n_qblk) return;
-  const int s = (int)(task / p.n_qblk);
-  const int j = (int)(task - (long long)s * p.n_qblk);
-  float* sc = sc_all + warp * p.n_win;
-  constexpr int PER = D / 32;
-  float qv[PER];
-  const float* qrow = p.qbar + ((size_t)s * p.n_qblk + j) * D;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) qv[e] = qrow[lane * PER + e];
+  const int s = blockIdx.y;
+  const int j0 = blockIdx.x * kSelWarps;
+  const int j = j0 + warp;
+  const bool active = j < p.n_qblk;
+  for (int x = threadIdx.x; x < kSelWarps * D; x += blockDim.x) {
+    const int jj = j0 + x / D;
+    qs[x] = (jj < p.n_qblk) ? p.qbar[((size_t)s * p.n_qblk + jj) * D + (x % D)] : 0.f;
+  }
   const float* kb = p.kbar + (size_t)s * p.n_win * D;
-  for (int w = 0; w < p.n_win; ++w) {
-    const float* kr = kb + (size_t)w * D + lane * PER;
-    float part = 0.f;
+  float* sc = scs + warp * p.n_win;
+  for (int w0 = 0; w0 < p.n_win; w0 += kSelChunk) {
+    const int nw = min(kSelChunk, p.n_win - w0);
+    __syncthreads();  // previous chunk fully consumed (and qs written, first time)
+    for (int x = threadIdx.x; x < nw * (D / 4); x += blockDim.x) {
+      const int r = x / (D / 4), c4 = x % (D / 4);
+      const float4 v = reinterpret_cast<const float4*>(kb + (size_t)(w0 + r) * D)[c4];
+      float* dst = ks + r * (D + 1) + c4 * 4;
+      dst[0] = v.x;
+      dst[1] = v.y;
+      dst[2] = v.z;
+      dst[3] = v.w;
+    }
+    __syncthreads();
+    if (active) {
+      const float* q = qs + warp * D;
+      for (int r = lane; r < nw; r += 32) {
+        const float* kr = ks + r * (D + 1);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int e = 0; e < PER; ++e) part = fmaf(qv[e], kr[e], part);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
-    if (lane == 0) {
-      sc[w] = (part != part) ? -INFINITY : part;  // NaN ranks last
+        for (int c = 0; c < D; c += 4) {
+          acc[0] = fmaf(q[c], kr[c], acc[0]);
+          acc[1] = fmaf(q[c + 1], kr[c + 1], acc[1]);
+          acc[2] = fmaf(q[c + 2], kr[c + 2], acc[2]);
+          acc[3] = fmaf(q[c + 3], kr[c + 3], acc[3]);
+        }
+        const float v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        sc[w0 + r] = (v != v) ? -INFINITY : v;  // NaN ranks last
+      }
     }
   }
   __syncwarp();
+  if (!active) return;
   if (p.out_scores) {
     float* so = p.out_scores + ((size_t)s * p.n_qblk + j) * p.n_win;
     for (int w = lane; w < p.n_win; w += 32) so[w] = sc[w];
   }
-  int* oi = p.out_idx + ((size_t)s * p.n_qblk + j) * p.topk;
-  int written = 0;
-  for (int w0 = 0; w0 < p.n_win; w0 += 32) {
-    const int w = w0 + lane;
-    bool keep = false;
-    if (w < p.n_win) {
-      const float x = sc[w];
-      int rank = 0;
-      for (int u = 0; u < p.n_win; ++u) {
-        const float y = sc[u];
-        rank += (y > x) || (y == x && u < w);
-      }
-      keep = rank < p.topk;
+  // exact top-K by radix selection of the topk-th largest score on
+  // order-preserving integer keys (32 ballot rounds); every block above that
+  // score is kept, and of the blocks equal to it the lowest indices are kept.
+  // Each lane owns blocks w = lane + 32m.
+  const int per = (p.n_win + 31) >> 5;  // <= kMaxPerLane
+  uint32_t key[kMaxPerLane];
+#pragma unroll
+  for (int m = 0; m < kMaxPerLane; ++m) {
+    const int w = lane + 32 * m;
+    if (m < per && w < p.n_win) {
+      const uint32_t u = __float_as_uint(sc[w]);
+      key[m] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);  // larger score -> larger key
+    } else {
+      key[m] = 0u;  // absent: below every real score (whose keys are >= 0x007FFFFF)
     }
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-    if (keep) oi[written + __popc(bal & ((1u << lane) - 1u))] = w;
-    written += __popc(bal);
   }
+  uint32_t prefix = 0u, mask = 0u;
+  int need = p.topk;  // rank, among the not-yet-excluded keys, of the threshold
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t want = prefix | (1u << bit), mk = mask | (1u << bit);
+    int cnt = 0;
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m)
+      if (m < per) cnt += ((key[m] & mk) == want) ? 1 : 0;
+    cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+    if (cnt >= need) {
+      prefix = want;
+    } else {
+      need -= cnt;
+    }
+    mask = mk;
+  }
+  // prefix = key of the topk-th largest score; `need` of its equals are kept
+  int* oi = p.out_idx + ((size_t)s * p.n_qblk + j) * p.topk;
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int m = 0; m < kMaxPerLane; ++m) {
+    if (m < per) {
+      const int w = lane + 32 * m;
+      const bool valid = w < p.n_win;
+      const bool eq = valid && key[m] == prefix;
+      const uint32_t beq = __ballot_sync(0xFFFFFFFFu, eq);
+      const int eq_rank = eq_seen + __popc(beq & ((1u << lane) - 1u));
+      const bool keep = valid && (key[m] > prefix || (eq && eq_rank < need));
+      eq_seen += __popc(beq);
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) oi[written + __popc(bal & ((1u << lane) - 1u))] = w;
+      written += __popc(bal);
+    }
+  }
+}
+
+// Instantiation by head dimension and by window size (candidates per lane).
+template <int D, int PER>
+bool launch_select_t(dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(select_kernel<D, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxSmem) !=
+        cudaSuccess)
+      return false;
+    attr_set[dev] = true;
+  }
+  select_kernel<D, PER><<<g, 32 * kSelWarps, smem, st>>>(sp);
+  return true;
+}
+
+template <int D>
+bool launch_select_d(int n_win, dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
+  if (n_win <= 160) return launch_select_t<D, 5>(g, smem, st, sp);
+  if (n_win <= 256) return launch_select_t<D, 8>(g, smem, st, sp);
+  if (n_win <= 512) return launch_select_t<D, 16>(g, smem, st, sp);
+  return launch_select_t<D, 32>(g, smem, st, sp);
+}
+
+bool launch_select(int d, int n_win, dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
+  return d == 128 ? launch_select_d<128>(n_win, g, smem, st, sp) : launch_select_d<64>(n_win, g, smem, st, sp);
 }
 
 }  // namespace
@@ -198,11 +303,11 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   pp.win_row0 = a->window_blk0 * a->block;
   pp.qbar = reinterpret_cast<float*>(a->workspace);
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  dim3 pg(n_qblk + a->n_win_blk, BH);
+  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + kPoolHeads - 1) / kPoolHeads));
   if (a->d == 128)
-    pool_kernel<128><<<pg, 128, 0, st>>>(pp);
+    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
   else
-    pool_kernel<64><<<pg, 128, 0, st>>>(pp);
+    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   SelParams sp;
   sp.qbar = pp.qbar;
@@ -213,13 +318,10 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   sp.topk = a->topk;
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
-  const long long tasks = (long long)BH * n_qblk;
-  const int grid = (int)((tasks + 7) / 8);
-  const size_t smem = (size_t)8 * a->n_win_blk * sizeof(float);
-  if (a->d == 128)
-    select_kernel<128><<<grid, 256, smem, st>>>(sp);
-  else
-    select_kernel<64><<<grid, 256, smem, st>>>(sp);
+  const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
+  const size_t smem = ((size_t)kSelWarps * a->d + (size_t)kSelChunk * (a->d + 1) +
+                       (size_t)kSelWarps * a->n_win_blk) * sizeof(float);
+  if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }
@@ -303,11 +405,11 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   pp.win_row0 = a->window_blk0 * a->block;
   pp.qbar = reinterpret_cast<float*>(scratch);
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  dim3 pg(n_qblk + a->n_win_blk, BH);
+  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + kPoolHeads - 1) / kPoolHeads));
   if (a->d == 128)
-    pool_kernel<128><<<pg, 128, 0, st>>>(pp);
+    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
   else
-    pool_kernel<64><<<pg, 128, 0, st>>>(pp);
+    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   SelParams sp;
   sp.qbar = pp.qbar;
@@ -318,13 +420,10 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   sp.topk = a->topk;
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
-  const long long tasks = (long long)BH * n_qblk;
-  const int grid = (int)((tasks + 7) / 8);
-  const size_t smem = (size_t)8 * a->n_win_blk * sizeof(float);
-  if (a->d == 128)
-    select_kernel<128><<<grid, 256, smem, st>>>(sp);
-  else
-    select_kernel<64><<<grid, 256, smem, st>>>(sp);
+  const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
+  const size_t smem = ((size_t)kSelWarps * a->d + (size_t)kSelChunk * (a->d + 1) +
+                       (size_t)kSelWarps * a->n_win_blk) * sizeof(float);
+  if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }

@@ -322,3 +322,60 @@ def test_ragged_bad_offsets_set_error_word():
                            scale=c.scale, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == vk().DEVERR_BAD_OFFSETS
+
+
+# ---------------------------------------------------------------------------
+# selection edge cases: ties, larger windows, d = 64; merge at d = 64
+# ---------------------------------------------------------------------------
+def test_block_select_all_ties_pick_lowest_indices():
+    """Identical window blocks: every score ties, so top-K = the K lowest block ids."""
+    c = _small_sparse(seed=85)
+    k = c.k.clone()
+    w0 = c.window_blk0 * 64
+    blk = k[:, w0:w0 + 64].clone()
+    for b in range(c.n_win_blk):
+        k[:, w0 + b * 64:w0 + (b + 1) * 64] = blk
+    for topk in (1, 5, c.n_win_blk - 1):
+        idx, _ = vk().block_select(c.q.to(DEV), k.to(DEV), c.window_blk0, c.n_win_blk, topk)
+        torch.cuda.synchronize()
+        ref, _ = oracle.block_select(c.q, k, c.window_blk0, c.n_win_blk, c.block, topk)
+        assert np.array_equal(ref, np.tile(np.arange(topk), ref.shape[:-1] + (1,)))
+        assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("win_frames,d", [(75, 128), (175, 64), (40, 64)])
+def test_block_select_large_windows(win_frames, d):
+    """Windows of 300 / 700 / 160 blocks exercise the wider per-lane instantiations."""
+    c = W.make_block_sparse("wide", seed=86 + win_frames, H=2, d=d, frame_tokens=256, block=64, hist_frames=1,
+                            win_frames=win_frames, q_frames=1, n_persist=2)
+    for topk in (7, c.n_win_blk // 3):
+        idx, sc = vk().block_select(c.q.to(DEV), c.k.to(DEV), c.window_blk0, c.n_win_blk, topk, scores=True)
+        torch.cuda.synchronize()
+        ref_s = oracle.block_scores(c.q, c.k, c.window_blk0, c.n_win_blk, c.block)
+        assert np.abs(to_np(sc) - ref_s).max() < 1e-3
+        gap = oracle.topk_gap(ref_s, topk)
+        exact = gap > 1e-4  # rows whose ranking fp32 scores can resolve
+        got = idx.cpu().numpy()
+        ref = oracle.select_topk(ref_s, topk)
+        assert np.array_equal(got[exact], ref[exact])
+        # every row holds topk distinct ascending window ids
+        assert np.all(np.diff(got, axis=-1) > 0) and got.min() >= 0 and got.max() < c.n_win_blk
+
+
+def test_lse_merge_kernel_d64():
+    oa, la, ob, lb = W.make_merge_inputs(6, 3, 77, 5, 64, neg_inf_frac=0.1)
+    o, l = vk().lse_merge(oa.to(DEV), la.to(DEV), ob.to(DEV), lb.to(DEV))
+    torch.cuda.synchronize()
+    ro, rl = oracle.lse_merge(to_np(oa), np.moveaxis(to_np(la), 1, 2), to_np(ob), np.moveaxis(to_np(lb), 1, 2))
+    assert_bf16_close(o, ro, "merge O d64")
+    assert_lse_close(l, np.moveaxis(rl, 2, 1), "merge LSE d64")
+
+
+def test_lse_merge_in_place():
+    oa, la, ob, lb = W.make_merge_inputs(7, 1, 200, 4, 128)
+    ref_o, ref_l = oracle.lse_merge(to_np(oa), np.moveaxis(to_np(la), 1, 2), to_np(ob), np.moveaxis(to_np(lb), 1, 2))
+    a, al = oa.to(DEV), la.to(DEV)
+    vk().lse_merge(a, al, ob.to(DEV), lb.to(DEV), out=(a, al))
+    torch.cuda.synchronize()
+    assert_bf16_close(a, ref_o, "in-place merge O")
+    assert_lse_close(al, np.moveaxis(ref_l, 2, 1), "in-place merge LSE")
