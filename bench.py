@@ -260,17 +260,29 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def timed(fn, iters: int, stream) -> list:
-    ts = []
-    for _ in range(iters):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+def timed(fn, iters: int, stream, flush=None) -> list:
+    """Device time of each call of `fn` (ms), CUDA events on `stream`.
+
+    The calls are queued behind a device-side sleep, so the host-side cost of
+    each call (argument marshalling, launch) is hidden and only GPU time is
+    measured.  With `flush` (a device buffer larger than L2), the buffer is
+    overwritten before every call, outside the timed interval, so each call
+    starts with a cold L2.
+    """
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    torch.cuda._sleep(int(4e5) * iters + int(2e6))  # ~0.2 ms of host enqueue time per call at ~2 GHz
+    for a, b in evs:
+        if flush is not None:
+            flush.zero_()
+        a.record(stream)
         fn()
-        e1.record(stream)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    return ts
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+L2_FLUSH_BYTES = 256 << 20  # twice the B200 L2
 
 
 def extras(dev, peaks):
@@ -279,6 +291,7 @@ def extras(dev, peaks):
     import oracle
     out = {}
     st = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     # Wan-1.3B-shaped dense dual-branch chunk
     c = W.cfg_wan13b()
     q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
@@ -290,11 +303,19 @@ def extras(dev, peaks):
     # standalone merge on the Wan-1.3B partials
     mo = vkv.lse_merge(res["o"][0], res["lse"][0], res["o"][1], res["lse"][1])
     ms = statistics.median(timed(lambda: vkv.lse_merge(res["o"][0], res["lse"][0], res["o"][1], res["lse"][1],
-                                                       out=mo), 50, st))
+                                                       out=mo), 50, st, flush))
     nbytes = 3 * res["o"][0].numel() * 2 + 3 * res["lse"][0].numel() * 4
     out["lse_merge_wan13b"] = {"ms": ms, "gbs": nbytes / ms / 1e6, "bytes": nbytes,
                                "frac_hbm": nbytes / ms / 1e6 / peaks["hbm_gbs"]}
     del q, k, v, res, mo
+    # standalone merge at the headline size (40 heads): inputs larger than L2
+    oa, la, ob, lb = (t.to(dev) for t in W.make_merge_inputs(5, 1, 4680, 40, 128))
+    mo = vkv.lse_merge(oa, la, ob, lb)
+    ms = statistics.median(timed(lambda: vkv.lse_merge(oa, la, ob, lb, out=mo), 50, st, flush))
+    nbytes = 3 * oa.numel() * 2 + 3 * la.numel() * 4
+    out["lse_merge_wan14b"] = {"ms": ms, "gbs": nbytes / ms / 1e6, "bytes": nbytes,
+                               "frac_hbm": nbytes / ms / 1e6 / peaks["hbm_gbs"]}
+    del oa, la, ob, lb, mo
     # block-sparse: persistent + top-K window blocks
     c = W.cfg_sparse()
     q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
@@ -306,7 +327,7 @@ def extras(dev, peaks):
                          dtype=torch.uint8, device=dev)
         idx, _ = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws)
         ms_sel = statistics.median(timed(lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K,
-                                                                  workspace=ws, out_idx=idx), 30, st))
+                                                                  workspace=ws, out_idx=idx), 30, st, flush))
         o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale)
         ms_att = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
             q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o), 20, st))

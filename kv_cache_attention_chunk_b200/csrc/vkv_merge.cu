@@ -26,7 +26,8 @@ struct MergeParams {
 
 constexpr int kMergePos = 8;  // consecutive (b, i) query positions per thread
 
-// grid: x = ceil(B * Lq / kMergePos) position groups, y = ceil(H * d/8 / 256) column blocks.
+// grid: x = ceil(B * Lq / kMergePos) position groups, y = column blocks of at
+// most 256 threads (H * d/8 columns split as evenly as whole warps allow).
 // Thread: one 16-byte column (head h, chunk ch) of kMergePos consecutive query
 // positions; all its loads are issued before the first merge, and the index
 // of the next position is advanced without division.  The output may alias an
@@ -125,13 +126,17 @@ extern "C" vkv_status vkv_lse_merge(vkv_tensor o_a, const float* lse_a, vkv_tens
   p.d = d;
   p.n_chunks = (long long)B * Lq * H * (d / 8);
   const long long n_pos = (long long)B * Lq;
-  const dim3 grid((unsigned)((n_pos + kMergePos - 1) / kMergePos), (unsigned)((H * (d / 8) + 255) / 256));
+  // column blocks of at most 256 threads, as even as warps allow (few idle lanes)
+  const int cols = H * (d / 8);
+  const int n_cb = (cols + 255) / 256;
+  const int width = (((cols + n_cb - 1) / n_cb) + 31) / 32 * 32;
+  const dim3 grid((unsigned)((n_pos + kMergePos - 1) / kMergePos), (unsigned)n_cb);
   if (grid.y > 65535u) return VKV_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128)
-    lse_merge_kernel<128><<<grid, 256, 0, st>>>(p);
+    lse_merge_kernel<128><<<grid, width, 0, st>>>(p);
   else
-    lse_merge_kernel<64><<<grid, 256, 0, st>>>(p);
+    lse_merge_kernel<64><<<grid, width, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }

@@ -6,16 +6,19 @@
 // Two kernels on the caller's stream:
 //   pool_kernel     mean of every 64-row block of Q and of the window part of K,
 //                   in fp32, written to the caller's workspace.  One CTA of 256
-//                   threads per (block, batch, group of 4 heads): the group's
+//                   threads per (block, batch, group of 256/d heads): the group's
 //                   contiguous slice of each row is read with 16-byte loads,
-//                   16 rows per thread in flight; row groups are combined in
+//                   8 rows per thread in flight; row groups are combined in
 //                   shared memory.  HBM-bound.
-//   select_kernel   one CTA per (batch*head, 4 query blocks), one warp per query
-//                   block: pooled keys are staged in shared memory 64 blocks at a
-//                   time, each lane scores its own blocks, then an exact
-//                   rank-based top-K: block w is kept iff fewer than K blocks beat
-//                   it (higher score, or equal score and lower index); kept
-//                   blocks are written in ascending order.
+//   select_kernel   one CTA per (batch*head, 8 query blocks): the pooled keys
+//                   are copied to shared memory 160 blocks at a time (cp.async),
+//                   each thread scores one window block against the CTA's eight
+//                   pooled queries, then one warp per query block runs an exact
+//                   top-K: radix selection of the K-th largest score on
+//                   order-preserving keys, ties at the threshold to the lower
+//                   block index; kept blocks are written in ascending order.
+//                   Launched as a programmatic dependent of the pooling kernel,
+//                   so its launch overlaps the pooling kernel's last CTAs.
 #include <algorithm>
 #include <mutex>
 
@@ -23,6 +26,22 @@
 #include "vkv_ptx.cuh"
 
 namespace vkv {
+
+// Development timeline (compiled only with -DVKV_TRACE): clock stamps of the
+// phases of select CTA (0, 0), read back with vkv_debug_sel_trace().
+#ifdef VKV_TRACE
+__device__ unsigned long long g_vkv_sel_trace[64];
+#define VKV_SEL_STAMP(i)                                                              \
+  do {                                                                                \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && (threadIdx.x & 31) == 0)               \
+      g_vkv_sel_trace[(threadIdx.x >> 5) * 8 + (i)] = clock64();                     \
+  } while (0)
+#else
+#define VKV_SEL_STAMP(i) \
+  do {                   \
+  } while (0)
+#endif
+
 namespace {
 
 struct PoolParams {
@@ -34,14 +53,18 @@ struct PoolParams {
   float* kbar;  // [B*H][n_win][d]
 };
 
-constexpr int kPoolHeads = 4;  // heads per pooling CTA (a contiguous slice of each row)
+// Heads per pooling CTA: a contiguous 512-byte slice of each row (2 heads at
+// d = 128, 4 at d = 64), 8 rows per thread in flight.
+template <int D>
+__host__ __device__ constexpr int pool_heads() { return 256 / D; }
 
 // grid: x = block index over n_qblk + n_win, y = b * ceil(H / kPoolHeads) + head group;
 // 256 threads.  Thread (g, c): column c = (head, 16-byte chunk) of the head
 // group's slice, rows g*RPG .. g*RPG + RPG - 1 of the 64-row block; the row
 // groups are combined in shared memory.
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(const PoolParams p) {
+__global__ void __launch_bounds__(256, 4) pool_kernel(const PoolParams p) {
+  constexpr int kPoolHeads = pool_heads<D>();
   constexpr int CPR = D / 8;                  // 16-byte chunks per head row
   constexpr int COLS = kPoolHeads * CPR;      // columns of the slice
   constexpr int GROUPS = 256 / COLS;          // row groups
@@ -82,6 +105,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolParams p) {
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  // every load of this CTA is issued: the select kernel may be scheduled now
+  // (it waits for this grid's completion before reading the pooled vectors)
+  griddep_launch_dependents();
 #pragma unroll
   for (int i = 0; i < RPG; ++i) {
     const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -116,70 +142,98 @@ struct SelParams {
   float* out_scores;
 };
 
-constexpr int kSelWarps = 4;     // query blocks per CTA (one warp each)
-constexpr int kSelMaxSmem = (kSelWarps * 128 + 64 * 129 + kSelWarps * 1024) * 4;
-constexpr int kSelChunk = 64;    // window blocks staged in shared memory at a time
+constexpr int kSelWarps = 8;     // query blocks per CTA (one warp each for the top-K)
+constexpr int kSelChunk = 160;   // window blocks staged in shared memory at a time
 
-// grid: x = ceil(n_qblk / kSelWarps), y = b*H + h; 128 threads.
-// Shared memory: pooled queries [kSelWarps][D], a chunk of pooled keys
-// [kSelChunk][D + 1] (padded: lane l reads row l, so rows land in distinct
-// banks) and the scores [kSelWarps][n_win].
+template <int D>
+__host__ __device__ constexpr int sel_row_stride() { return D + 4; }  // floats; keeps rows 16-byte aligned
+
+template <int D>
+constexpr size_t sel_smem_bytes(int n_win) {
+  return ((size_t)kSelWarps * D + (size_t)kSelChunk * sel_row_stride<D>() + (size_t)kSelWarps * n_win) *
+         sizeof(float);
+}
+constexpr int kSelMaxSmem = (int)sel_smem_bytes<128>(1024);
+
+// grid: x = ceil(n_qblk / kSelWarps), y = b*H + h; 32 * kSelWarps threads.
+// Shared memory: the CTA's pooled queries [kSelWarps][D], a chunk of pooled
+// keys [kSelChunk][D + 4] and the scores [kSelWarps][n_win].  Pooled vectors
+// are copied with cp.async (every copy of a chunk in flight at once).  Thread i
+// scores window block w0 + i against all of the CTA's pooled queries: its key
+// row is read from shared memory once (float4 reads; with the 4-float pad the
+// eight rows of a quarter warp fall in distinct banks), the query rows are
+// broadcast.  Then warp q selects the top-K of query block j0 + q.
 template <int D, int kMaxPerLane>
-__global__ void __launch_bounds__(128) select_kernel(const SelParams p) {
-  extern __shared__ float sm[];
+__global__ void __launch_bounds__(32 * kSelWarps) select_kernel(const SelParams p) {
+  extern __shared__ __align__(16) float sm[];
+  constexpr int RS = sel_row_stride<D>();
+  constexpr int D4 = D / 4;
   float* qs = sm;                              // kSelWarps * D
-  float* ks = qs + kSelWarps * D;              // kSelChunk * (D + 1)
-  float* scs = ks + kSelChunk * (D + 1);       // kSelWarps * n_win
+  float* ks = qs + kSelWarps * D;              // kSelChunk * RS
+  float* scs = ks + kSelChunk * RS;            // kSelWarps * n_win
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int s = blockIdx.y;
   const int j0 = blockIdx.x * kSelWarps;
+  const int nq = min(kSelWarps, p.n_qblk - j0);
   const int j = j0 + warp;
-  const bool active = j < p.n_qblk;
-  for (int x = threadIdx.x; x < kSelWarps * D; x += blockDim.x) {
-    const int jj = j0 + x / D;
-    qs[x] = (jj < p.n_qblk) ? p.qbar[((size_t)s * p.n_qblk + jj) * D + (x % D)] : 0.f;
+  const bool active = warp < nq;
+  VKV_SEL_STAMP(0);
+  griddep_wait();  // the pooling kernel before this one on the stream has completed
+  VKV_SEL_STAMP(1);
+  const float* qsrc = p.qbar + ((size_t)s * p.n_qblk + j0) * D;
+  for (int x = threadIdx.x; x < kSelWarps * D4; x += blockDim.x) {
+    if (x < nq * D4)
+      cp_async16(qs + 4 * x, qsrc + 4 * x);
+    else
+      reinterpret_cast<float4*>(qs)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const float* kb = p.kbar + (size_t)s * p.n_win * D;
-  float* sc = scs + warp * p.n_win;
   for (int w0 = 0; w0 < p.n_win; w0 += kSelChunk) {
     const int nw = min(kSelChunk, p.n_win - w0);
-    __syncthreads();  // previous chunk fully consumed (and qs written, first time)
-    for (int x = threadIdx.x; x < nw * (D / 4); x += blockDim.x) {
-      const int r = x / (D / 4), c4 = x % (D / 4);
-      const float4 v = reinterpret_cast<const float4*>(kb + (size_t)(w0 + r) * D)[c4];
-      float* dst = ks + r * (D + 1) + c4 * 4;
-      dst[0] = v.x;
-      dst[1] = v.y;
-      dst[2] = v.z;
-      dst[3] = v.w;
+    __syncthreads();  // the previous chunk is fully consumed
+    for (int x = threadIdx.x; x < nw * D4; x += blockDim.x) {
+      const int r = x / D4, c4 = x - (x / D4) * D4;
+      cp_async16(ks + r * RS + 4 * c4, kb + (size_t)(w0 + r) * D + 4 * c4);
     }
+    cp_async_wait_all();
     __syncthreads();
-    if (active) {
-      const float* q = qs + warp * D;
-      for (int r = lane; r < nw; r += 32) {
-        const float* kr = ks + r * (D + 1);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    VKV_SEL_STAMP(2);
+    for (int r = threadIdx.x; r < nw; r += blockDim.x) {
+      const float4* kr = reinterpret_cast<const float4*>(ks + r * RS);
+      float acc[kSelWarps][4];
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
-          acc[0] = fmaf(q[c], kr[c], acc[0]);
-          acc[1] = fmaf(q[c + 1], kr[c + 1], acc[1]);
-          acc[2] = fmaf(q[c + 2], kr[c + 2], acc[2]);
-          acc[3] = fmaf(q[c + 3], kr[c + 3], acc[3]);
+      for (int q = 0; q < kSelWarps; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < D4; ++c) {
+        const float4 kv = kr[c];
+#pragma unroll
+        for (int q = 0; q < kSelWarps; ++q) {
+          const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[c];
+          acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
+          acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
+          acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
+          acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
         }
-        const float v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        sc[w0 + r] = (v != v) ? -INFINITY : v;  // NaN ranks last
+      }
+#pragma unroll
+      for (int q = 0; q < kSelWarps; ++q) {
+        const float v = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
+        // NaN ranks last; -0 becomes +0 so that equal scores tie on the block index
+        scs[q * p.n_win + w0 + r] = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
       }
     }
   }
-  __syncwarp();
+  __syncthreads();
+  VKV_SEL_STAMP(3);
+  const float* sc = scs + warp * p.n_win;
   if (!active) return;
   if (p.out_scores) {
     float* so = p.out_scores + ((size_t)s * p.n_qblk + j) * p.n_win;
     for (int w = lane; w < p.n_win; w += 32) so[w] = sc[w];
   }
   // exact top-K by radix selection of the topk-th largest score on
-  // order-preserving integer keys (32 ballot rounds); every block above that
+  // order-preserving integer keys (32 rounds); every block above that
   // score is kept, and of the blocks equal to it the lowest indices are kept.
   // Each lane owns blocks w = lane + 32m.
   const int per = (p.n_win + 31) >> 5;  // <= kMaxPerLane
@@ -196,6 +250,8 @@ __global__ void __launch_bounds__(128) select_kernel(const SelParams p) {
   }
   uint32_t prefix = 0u, mask = 0u;
   int need = p.topk;  // rank, among the not-yet-excluded keys, of the threshold
+  // one bit per round, most significant first (one warp sum per round: warp
+  // collectives are the cost here, so the fewest of them wins)
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t want = prefix | (1u << bit), mk = mask | (1u << bit);
     int cnt = 0;
@@ -210,6 +266,7 @@ __global__ void __launch_bounds__(128) select_kernel(const SelParams p) {
     }
     mask = mk;
   }
+  VKV_SEL_STAMP(4);
   // prefix = key of the topk-th largest score; `need` of its equals are kept
   int* oi = p.out_idx + ((size_t)s * p.n_qblk + j) * p.topk;
   int written = 0, eq_seen = 0;
@@ -228,6 +285,7 @@ __global__ void __launch_bounds__(128) select_kernel(const SelParams p) {
       written += __popc(bal);
     }
   }
+  VKV_SEL_STAMP(5);
 }
 
 // Instantiation by head dimension and by window size (candidates per lane).
@@ -242,8 +300,18 @@ bool launch_select_t(dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) 
       return false;
     attr_set[dev] = true;
   }
-  select_kernel<D, PER><<<g, 32 * kSelWarps, smem, st>>>(sp);
-  return true;
+  // programmatic dependent launch: set-up overlaps the tail of the pooling kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = g;
+  cfg.blockDim = dim3(32 * kSelWarps);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_kernel<D, PER>, sp) == cudaSuccess;
 }
 
 template <int D>
@@ -262,6 +330,15 @@ bool launch_select(int d, int n_win, dim3 g, size_t smem, cudaStream_t st, const
 }  // namespace vkv
 
 using namespace vkv;
+
+#ifdef VKV_TRACE
+// Development only (not in the public header): copy select CTA (0, 0)'s stamps.
+extern "C" int vkv_debug_sel_trace(void* dst, size_t bytes) {
+  cudaDeviceSynchronize();
+  return (int)cudaMemcpyFromSymbol(dst, vkv::g_vkv_sel_trace,
+                                   bytes < sizeof(vkv::g_vkv_sel_trace) ? bytes : sizeof(vkv::g_vkv_sel_trace));
+}
+#endif
 
 extern "C" size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,
                                                   int32_t block, int32_t d) {
@@ -303,7 +380,8 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   pp.win_row0 = a->window_blk0 * a->block;
   pp.qbar = reinterpret_cast<float*>(a->workspace);
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + kPoolHeads - 1) / kPoolHeads));
+  const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
+  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + ph - 1) / ph));
   if (a->d == 128)
     pool_kernel<128><<<pg, 256, 0, st>>>(pp);
   else
@@ -319,8 +397,7 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
   const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
-  const size_t smem = ((size_t)kSelWarps * a->d + (size_t)kSelChunk * (a->d + 1) +
-                       (size_t)kSelWarps * a->n_win_blk) * sizeof(float);
+  const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
   if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
@@ -405,7 +482,8 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   pp.win_row0 = a->window_blk0 * a->block;
   pp.qbar = reinterpret_cast<float*>(scratch);
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + kPoolHeads - 1) / kPoolHeads));
+  const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
+  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + ph - 1) / ph));
   if (a->d == 128)
     pool_kernel<128><<<pg, 256, 0, st>>>(pp);
   else
@@ -421,8 +499,7 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
   const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
-  const size_t smem = ((size_t)kSelWarps * a->d + (size_t)kSelChunk * (a->d + 1) +
-                       (size_t)kSelWarps * a->n_win_blk) * sizeof(float);
+  const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
   if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
