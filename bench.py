@@ -325,19 +325,30 @@ def extras(dev, peaks):
         K = W.topk_for_fraction(frac, c.n_win_blk)
         ws = torch.empty(vkv.vkv_block_select_workspace_size(1, 12, c.Lq, c.n_win_blk, 64, 128),
                          dtype=torch.uint8, device=dev)
-        idx, _ = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws)
+        idx, _, order = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws, order=True)
         ms_sel = statistics.median(timed(lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K,
-                                                                  workspace=ws, out_idx=idx), 30, st, flush))
-        o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale)
+                                                                  workspace=ws, out_idx=idx, out_order=order),
+                                         30, st, flush))
+        o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale,
+                                        qblk_order=order)
         ms_att = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
+            q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o, qblk_order=order), 20, st))
+        ms_nat = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
             q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o), 20, st))
         fl = oracle.visited_flops_sparse(1, 12, c.Lq, 128, 64, c.persist_idx.shape[1], K)
         sel_bytes = (c.Lq + c.n_win_blk * 64) * 12 * 128 * 2
-        sp[f"K{K}"] = {"attn_ms": ms_att, "attn_tflops": fl / ms_att / 1e9, "select_ms": ms_sel,
-                       "select_gbs": sel_bytes / ms_sel / 1e6, "visited_frac": (32 + K) / (32 + c.n_win_blk)}
+        sp[f"K{K}"] = {"attn_ms": ms_att, "attn_tflops": fl / ms_att / 1e9, "attn_ms_natural_order": ms_nat,
+                       "select_ms": ms_sel, "select_gbs": sel_bytes / ms_sel / 1e6,
+                       "chunk_ms": ms_sel + ms_att, "visited_frac": (32 + K) / (32 + c.n_win_blk)}
     full = sp[f"K{c.n_win_blk}"]["attn_ms"]
     for kk in sp:
         sp[kk]["time_frac_of_K_all"] = sp[kk]["attn_ms"] / full
+    xs = np.array([sp[kk]["visited_frac"] for kk in sp])
+    ys = np.array([sp[kk]["time_frac_of_K_all"] for kk in sp])
+    slope, icpt = np.polyfit(xs, ys, 1)
+    r2 = 1.0 - float(((ys - (slope * xs + icpt)) ** 2).sum()) / float(((ys - ys.mean()) ** 2).sum())
+    sp["scaling_fit"] = {"slope": float(slope), "intercept": float(icpt), "r2": r2,
+                         "target": "t(K)/t(144) = visited fraction: slope 1, intercept 0"}
     out["sparse"] = sp
     del q, k, v
     # ragged per-head cache
@@ -485,14 +496,16 @@ def run_profile(args):
         c = W.cfg_sparse()
         q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
         K = 9 if args.profile != "sparse144" else 144
-        idx, _ = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K)
+        idx, _, order = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
         if args.profile == "select":
-            fn = lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, out_idx=idx)  # noqa: E731
+            fn = lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, out_idx=idx,  # noqa: E731
+                                          out_order=order)
         else:
             pers = torch.from_numpy(c.persist_idx).to(dev)
-            o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale)
+            o = vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale,
+                                            qblk_order=order)
             fn = lambda: vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk,  # noqa: E731
-                                                     scale=c.scale, out=o)
+                                                     scale=c.scale, out=o, qblk_order=order)
     elif args.profile == "ragged":
         c = W.cfg_ragged()
         q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)

@@ -149,6 +149,17 @@ typedef struct {
   float* lse_merged;
 
   int32_t* err_word; /* optional DEVICE int32; see VKV_DEVERR_* */
+
+  /* VKV_MODE_BLOCK_SPARSE, optional (NULL = natural order): DEVICE int32
+   * [B*H][ceil(Lq/block)], for each (b, h) a permutation of its query blocks.
+   * Work is cut into units of four consecutive entries (two 128-row tiles of
+   * two query blocks each) and a unit streams the union of its query blocks'
+   * selections, so an order that puts query blocks with similar selections
+   * side by side (vkv_block_select's out_order) shrinks the work.  Results do
+   * not depend on the order beyond rounding.  An entry outside
+   * [0, ceil(Lq/block)) raises VKV_DEVERR_BAD_INDEX; a repeated entry leaves
+   * some query block unwritten (not checked). */
+  const int32_t* qblk_order;
 } vkv_attn_args;
 
 /*
@@ -194,6 +205,13 @@ typedef struct {
   void* workspace;
   size_t workspace_bytes;
   int32_t* err_word;      /* optional DEVICE int32                             */
+  /* optional DEVICE int32 [B*H][ceil(Lq/block)] (NULL = skip): for each (b, h)
+   * a permutation of its query blocks, sorted by their selections (ascending
+   * lexicographic order of the first six selected ids, then by block index),
+   * so that query blocks with similar selections are adjacent; pass it to
+   * vkv_chunk_attn as qblk_order.  Not part of the pages' method: it only
+   * groups work. */
+  int32_t* out_order;
 } vkv_select_args;
 
 size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,

@@ -31,11 +31,15 @@ struct Cand {
   double cost;
 };
 
+// Time of a one-tile unit relative to a two-tile unit over the same keys.  A
+// lone tile cannot hide its softmax behind another tile's MMAs, so it costs
+// almost as much as a pair (measured on B200: 0.9 balances the dense, ragged
+// and block-sparse schedules best; VKV_SINGLE_COST overrides it).
 double single_tile_cost() {
   static double c = [] {
     const char* e = std::getenv("VKV_SINGLE_COST");
     double v = e ? std::atof(e) : 0.0;
-    return (v > 0.05 && v <= 1.0) ? v : 0.6;
+    return (v > 0.05 && v <= 1.0) ? v : 0.9;
   }();
   return c;
 }
@@ -100,7 +104,7 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
     }
   };
   std::vector<long long> cands = {0};
-  for (int k = 1; k <= 16; ++k) cands.push_back((long long)k * n_sm / 4);
+  for (int k = 1; k <= 32; ++k) cands.push_back((long long)k * n_sm / 8);
   cands.push_back(n_pairs);
   double best = 1e300;
   long long best_split = 0;
@@ -281,14 +285,20 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     P->n_blocks_total = Lkv / 64;
     P->persist_idx = a->persist_idx;
     P->sel_idx = a->sel_idx;
-    const double sp = (a->n_persist + std::min(a->n_win_blk, 4 * a->topk)) * 0.5 + 2.0;
-    const double s1 = (a->n_persist + std::min(a->n_win_blk, 2 * a->topk)) * 0.5 + 2.0;
+    P->qblk_order = a->qblk_order;
+    // expected key tiles of a unit: persistent blocks + the union of its query blocks'
+    // selections (two blocks per tile); a grouped order keeps the union near one selection
+    const bool grouped = a->qblk_order != nullptr;
+    const double u4 = std::min<double>(a->n_win_blk, (grouped ? 1.5 : 4.0) * a->topk);
+    const double u2 = std::min<double>(a->n_win_blk, (grouped ? 1.25 : 2.0) * a->topk);
+    const double sp = (a->n_persist + u4) * 0.5 + 2.0;
+    const double s1 = (a->n_persist + u2) * 0.5 + 2.0;
     for (long long s = 0; s < n_seq; ++s) {
       pc[s] = sp;
-      oc[s] = c1 * s1 * (sp > 0 ? 1.0 : 1.0);
+      oc[s] = c1 * s1;
     }
     key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
-          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk);
+          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n");
   } else {
     if (!a->cu_seqlens) return VKV_ERR_NULL;
     if (Lkv <= 0 || a->k.st <= 0 || a->v.st <= 0 || (a->k.st % 8) || (a->v.st % 8)) return VKV_ERR_SHAPE;
@@ -344,7 +354,8 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);
   std::copy(plan->units.begin(), plan->units.end(), P->units);
 
-  if (!encode_bhld(&P->tm_q, a->q, B, Lq, H, d, 128)) return VKV_ERR_CUDA;
+  // BLOCK_SPARSE loads a query tile as two 64-row blocks (a unit's blocks follow qblk_order)
+  if (!encode_bhld(&P->tm_q, a->q, B, Lq, H, d, mode == VKV_MODE_BLOCK_SPARSE ? 64 : 128)) return VKV_ERR_CUDA;
   if (mode == VKV_MODE_RAGGED) {
     if (!encode_flat(&P->tm_k, a->k, Lkv, d) || !encode_flat(&P->tm_v, a->v, Lkv, d)) return VKV_ERR_CUDA;
   } else {

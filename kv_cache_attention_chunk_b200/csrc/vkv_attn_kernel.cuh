@@ -8,9 +8,11 @@
 //                 (ISPA summary, section 2 step 1: local and history branches,
 //                 each closed with its own output and LSE, then merged);
 //   BLOCK_SPARSE  the unit's persistent blocks, then the union of the window
-//                 blocks selected for its 64-query blocks, two blocks per tile,
-//                 with a per-query-block visibility mask (Sparse Forcing
-//                 summary, section 2 component 3 "PBSA");
+//                 blocks selected for its four 64-query blocks (consecutive in
+//                 the caller's query-block order, which may group blocks with
+//                 similar selections), two blocks per tile, with a per-query-
+//                 block visibility mask (Sparse Forcing summary, section 2
+//                 component 3 "PBSA");
 //   RAGGED        consecutive tiles of rows [cu[s], cu[s+1]) of the flattened
 //                 cache (Pyramid Forcing summary, methodology section 3).
 //
@@ -169,6 +171,20 @@ __device__ __forceinline__ void set_err(const AttnParams& p, int code) {
   if (p.err) atomicCAS(p.err, 0, code);
 }
 
+// BLOCK_SPARSE: query block at position `pos` of sequence s's unit order
+// (qblk_order, or the natural order); -1 past the last block.  An entry out of
+// range records VKV_DEVERR_BAD_INDEX and falls back to the natural order.
+__device__ __forceinline__ int unit_qblk(const AttnParams& p, int s, int pos, bool report) {
+  if (pos >= p.n_qblk) return -1;
+  if (!p.qblk_order) return pos;
+  const int q = __ldg(p.qblk_order + (size_t)s * p.n_qblk + pos);
+  if (q < 0 || q >= p.n_qblk) {
+    if (report) set_err(p, VKV_DEVERR_BAD_INDEX);
+    return pos;
+  }
+  return q;
+}
+
 // Rows [start, start+len) of a ragged sequence, checked on the device.
 __device__ __forceinline__ void ragged_range(const AttnParams& p, int s, int& start, int& len,
                                              bool report) {
@@ -204,7 +220,8 @@ __device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, 
   for (int i = 0; i < 4; ++i) ctl->bitmap[i][lane] = 0u;
   __syncwarp();
   for (int i = 0; i < nqb; ++i) {
-    const int* row = p.sel_idx + ((size_t)u.s * p.n_qblk + (qb0 + i)) * p.topk;
+    const int qbi = unit_qblk(p, u.s, qb0 + i, lane == 0);
+    const int* row = p.sel_idx + ((size_t)u.s * p.n_qblk + qbi) * p.topk;
     for (int e = lane; e < p.topk; e += 32) {
       const int w = __ldg(row + e);
       if (w >= 0 && w < p.n_win_blk) {
@@ -472,11 +489,25 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           if (qcnt > 0) ok = mbar_wait(b_qempty, (qcnt - 1) & 1, abort_flag, p.err);
           if (ok) {
             mbar_arrive_expect_tx(b_qfull, (uint32_t)(u.ntiles * C::QT_BYTES));
-            for (int t = 0; t < u.ntiles; ++t)
+            for (int t = 0; t < u.ntiles; ++t) {
+              if (sparse) {
+                // two 64-row query blocks in unit order; a missing one reads rows past
+                // Lq, which the TMA fills with zeros
+                for (int half = 0; half < 2; ++half) {
+                  const int qb = unit_qblk(p, u.s, 2 * (u.tile0 + t) + half, false);
+                  const int row = qb >= 0 ? qb * 64 : p.n_qblk * 64;
 #pragma unroll
-              for (int ac = 0; ac < C::NAC; ++ac)
-                tma_load_4d(sQ + t * C::QT_BYTES + ac * C::ATOM, &p.tm_q, ac * 64, u.h,
-                            (u.tile0 + t) * 128, u.b, b_qfull);
+                  for (int ac = 0; ac < C::NAC; ++ac)
+                    tma_load_4d(sQ + t * C::QT_BYTES + ac * C::ATOM + half * 64 * 128, &p.tm_q, ac * 64, u.h,
+                                row, u.b, b_qfull);
+                }
+              } else {
+#pragma unroll
+                for (int ac = 0; ac < C::NAC; ++ac)
+                  tma_load_4d(sQ + t * C::QT_BYTES + ac * C::ATOM, &p.tm_q, ac * 64, u.h,
+                              (u.tile0 + t) * 128, u.b, b_qfull);
+              }
+            }
             ++qcnt;
           }
           TileIter it;
@@ -640,7 +671,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       }
       const int nsteps = unit_steps(p, ctl, rl);
       const bool active = t < u.ntiles;
-      const int qrow = (u.tile0 + t) * 128 + r;
+      int qrow = (u.tile0 + t) * 128 + r;
+      if (sparse) {
+        const int qbr = unit_qblk(p, u.s, 2 * (u.tile0 + t) + (r >> 6), false);
+        qrow = qbr >= 0 ? qbr * 64 + (r & 63) : p.Lq;
+      }
       const bool row_ok = qrow < p.Lq;
       const int qb = 2 * t + (r >> 6);
       float m = -INFINITY, l = 0.f;            // running state of the current branch

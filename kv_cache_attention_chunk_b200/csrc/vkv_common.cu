@@ -88,7 +88,7 @@ extern "C" const char* vkv_status_string(vkv_status s) {
   return "unknown status";
 }
 
-extern "C" int32_t vkv_version(void) { return 100; }
+extern "C" int32_t vkv_version(void) { return 101; }
 
 extern "C" int32_t vkv_abi_sizeof(int32_t which) {
   switch (which) {

@@ -19,7 +19,7 @@ constexpr int kMaxFlatSegs = VKV_MAX_BRANCHES * VKV_MAX_SEGMENTS;
 // Kernel parameters of the attention kernel, passed as __grid_constant__.
 // Unit code: bits [0,13) first query tile, bit 13 two tiles, bits [14,32) sequence b*H+h.
 struct AttnParams {
-  CUtensorMap tm_q;  // dims (d, H, Lq, B); box (64, 1, 128, 1); 128 B swizzle
+  CUtensorMap tm_q;  // dims (d, H, Lq, B); box (64, 1, 128 or 64 (BLOCK_SPARSE), 1); 128 B swizzle
   CUtensorMap tm_k;  // dims (d, H, Lkv, B) or (d, 1, rows, 1); box (64, 1, 64, 1)
   CUtensorMap tm_v;
   int mode, B, H, Lq, Lkv, d;
@@ -37,6 +37,7 @@ struct AttnParams {
   int n_persist, topk, window_blk0, n_win_blk, n_qblk, n_blocks_total;
   const int* persist_idx;
   const int* sel_idx;
+  const int* qblk_order;  // optional [B*H][n_qblk] query-block permutation
   // RAGGED
   const int* cu_seqlens;
   // outputs

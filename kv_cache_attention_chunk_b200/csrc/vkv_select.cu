@@ -288,6 +288,55 @@ __global__ void __launch_bounds__(32 * kSelWarps) select_kernel(const SelParams 
   VKV_SEL_STAMP(5);
 }
 
+// Query-block order that groups blocks with similar selections (a work-grouping
+// aid for the block-sparse attention, not part of the selection itself).
+// Signature of query block j: its first kOrderIds selected ids (ascending),
+// 10 bits each, the first id most significant; order = ascending signature,
+// then ascending block index.  One CTA per (batch*head); rank by counting.
+struct OrderParams {
+  const int* sel;  // [BH][n_qblk][topk]
+  int* order;      // [BH][n_qblk]
+  int n_qblk, topk;
+};
+
+constexpr int kOrderIds = 6;
+constexpr int kOrderMaxQblk = 4096;  // signatures of one (batch, head) in shared memory
+
+__global__ void __launch_bounds__(256) order_kernel(const OrderParams p) {
+  extern __shared__ unsigned long long sig[];
+  const int s = blockIdx.x;
+  const int* rows = p.sel + (size_t)s * p.n_qblk * p.topk;
+  for (int j = threadIdx.x; j < p.n_qblk; j += blockDim.x) {
+    unsigned long long key = 0ull;
+#pragma unroll
+    for (int e = 0; e < kOrderIds; ++e) {
+      const unsigned id = e < p.topk ? (unsigned)rows[(size_t)j * p.topk + e] & 1023u : 0u;
+      key = (key << 10) | id;
+    }
+    sig[j] = key;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < p.n_qblk; j += blockDim.x) {
+    const unsigned long long kj = sig[j];
+    int rank = 0;
+    for (int i = 0; i < p.n_qblk; ++i) {
+      const unsigned long long ki = sig[i];
+      rank += (ki < kj || (ki == kj && i < j)) ? 1 : 0;
+    }
+    p.order[(size_t)s * p.n_qblk + rank] = j;
+  }
+}
+
+bool launch_order(const int* sel, int* order, int BH, int n_qblk, int topk, cudaStream_t st) {
+  OrderParams op;
+  op.sel = sel;
+  op.order = order;
+  op.n_qblk = n_qblk;
+  op.topk = topk;
+  order_kernel<<<BH, 256, (size_t)n_qblk * sizeof(unsigned long long), st>>>(op);
+  return cudaGetLastError() == cudaSuccess;
+}
+
 // Instantiation by head dimension and by window size (candidates per lane).
 template <int D, int PER>
 bool launch_select_t(dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
@@ -361,6 +410,7 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   if (!a->workspace || a->workspace_bytes < need) return VKV_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
   if ((long long)a->B * a->H > 65535) return VKV_ERR_UNSUPPORTED;
+  if (a->out_order && (a->Lq + a->block - 1) / a->block > kOrderMaxQblk) return VKV_ERR_UNSUPPORTED;
   int dev = 0;
   if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -400,6 +450,7 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
   if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  if (a->out_order && !launch_order(a->out_idx, a->out_order, BH, n_qblk, a->topk, st)) return VKV_ERR_CUDA;
   return VKV_OK;
 }
 
@@ -459,6 +510,7 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   if (!a->q.ptr || !a->k.ptr || !a->out_idx) return VKV_ERR_NULL;
   if (!tensor_aligned(a->q) || !tensor_aligned(a->k)) return VKV_ERR_ALIGN;
   if ((long long)a->B * a->H > 65535) return VKV_ERR_UNSUPPORTED;
+  if (a->out_order && (a->Lq + a->block - 1) / a->block > kOrderMaxQblk) return VKV_ERR_UNSUPPORTED;
   const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
   if (need > kNoallocScratchBytes) return VKV_ERR_WORKSPACE;  // larger than the fixed scratch array
   int dev = 0;
@@ -502,5 +554,6 @@ extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_str
   const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
   if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  if (a->out_order && !launch_order(a->out_idx, a->out_order, BH, n_qblk, a->topk, st)) return VKV_ERR_CUDA;
   return VKV_OK;
 }

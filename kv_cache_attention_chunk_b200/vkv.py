@@ -58,6 +58,7 @@ class vkv_attn_args(ctypes.Structure):
         ("o", vkv_tensor * MAX_BRANCHES), ("lse", c_void_p * MAX_BRANCHES),
         ("o_merged", vkv_tensor), ("lse_merged", c_void_p),
         ("err_word", c_void_p),
+        ("qblk_order", c_void_p),
     ]
 
 
@@ -70,6 +71,7 @@ class vkv_select_args(ctypes.Structure):
         ("out_idx", c_void_p), ("out_scores", c_void_p),
         ("workspace", c_void_p), ("workspace_bytes", c_size_t),
         ("err_word", c_void_p),
+        ("out_order", c_void_p),
     ]
 
 
@@ -227,8 +229,12 @@ def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, st
 
 
 def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_blk, scale=None,
-                            err=None, stream=None, out=None):
-    """Persistent blocks + selected window blocks (device int32 index tensors)."""
+                            err=None, stream=None, out=None, qblk_order=None):
+    """Persistent blocks + selected window blocks (device int32 index tensors).
+
+    qblk_order (optional device int32 [B*H, nQblk]): query-block permutation that
+    groups blocks with similar selections into the same units (from block_select).
+    """
     d = q.shape[3]
     a = _base_args(MODE_BLOCK_SPARSE, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
     persist_idx = persist_idx.contiguous()
@@ -239,6 +245,9 @@ def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_bl
     a.topk = sel_idx.shape[-1]
     a.window_blk0 = int(window_blk0)
     a.n_win_blk = int(n_win_blk)
+    if qblk_order is not None:
+        qblk_order = qblk_order.contiguous()
+        a.qblk_order = qblk_order.data_ptr()
     o, l = out if out is not None else _new_out(q)
     a.o[0] = tensor_desc(o)
     a.lse[0] = l.data_ptr()
@@ -264,8 +273,12 @@ def chunk_attn_ragged(q, k_flat, v_flat, cu_seqlens, cu_seqlens_host=None, scale
 
 
 def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=False, err=None, stream=None,
-                 out_idx=None):
-    """Top-K window blocks per 64-query block; returns (idx [B*H, nQblk, topk], scores or None)."""
+                 out_idx=None, order=False, out_order=None):
+    """Top-K window blocks per 64-query block; returns (idx [B*H, nQblk, topk], scores or None).
+
+    With order=True (or an out_order tensor) also returns the query-block order
+    [B*H, nQblk] that groups blocks with similar selections: (idx, scores, order).
+    """
     B, Lq, H, d = q.shape
     n_qblk = -(-Lq // 64)
     a = vkv_select_args()
@@ -287,7 +300,13 @@ def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=Fals
     a.workspace = workspace.data_ptr()
     a.workspace_bytes = workspace.numel() * workspace.element_size()
     a.err_word = err.data_ptr() if err is not None else None
+    if order and out_order is None:
+        out_order = torch.empty((B * H, n_qblk), dtype=torch.int32, device=q.device)
+    if out_order is not None:
+        a.out_order = out_order.data_ptr()
     _check(vkv_block_select(a, _stream(stream)), "vkv_block_select")
+    if out_order is not None:
+        return idx, sc, out_order
     return idx, sc
 
 

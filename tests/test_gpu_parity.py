@@ -266,6 +266,103 @@ def test_sparse_bad_index_sets_error_word():
     assert int(err.item()) == vk().DEVERR_BAD_INDEX
 
 
+def _order_reference(sel):
+    """Query-block order of the grouping aid: ascending (first six selected ids, 10 bits
+    each, first id most significant), then ascending block index."""
+    BH, nq, K = sel.shape
+    out = np.zeros((BH, nq), dtype=np.int32)
+    for s in range(BH):
+        keys = []
+        for j in range(nq):
+            key = 0
+            for e in range(6):
+                key = (key << 10) | ((int(sel[s, j, e]) & 1023) if e < K else 0)
+            keys.append((key, j))
+        out[s] = [j for _, j in sorted(keys)]
+    return out
+
+
+@pytest.mark.parametrize("topk", [1, 9, 36, 144])
+def test_block_select_order_definition(topk):
+    c = W.cfg_sparse()
+    q, k = c.q.to(DEV), c.k.to(DEV)
+    idx, _, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, topk, order=True)
+    torch.cuda.synchronize()
+    sel = idx.cpu().numpy()
+    got = order.cpu().numpy()
+    assert np.array_equal(np.sort(got, axis=1), np.tile(np.arange(c.n_qblk), (c.B * c.H, 1)))
+    assert np.array_equal(got, _order_reference(sel))
+
+
+@pytest.mark.parametrize("frame_tokens,qf,topk", [(256, 2, 3), (192, 1, 4), (192, 3, 2)])
+def test_block_sparse_grouped_order_matches_oracle(frame_tokens, qf, topk):
+    # (192, 1): three query blocks, so the second tile's second block is missing
+    c = W.make_block_sparse("grp", seed=85, H=2, d=128, frame_tokens=frame_tokens, block=64, hist_frames=3,
+                            win_frames=4, q_frames=qf, n_persist=5)
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    idx, _, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, topk, order=True)
+    err = err_word()
+    o, l = vk().chunk_attn_block_sparse(q, k, v, torch.from_numpy(c.persist_idx).to(DEV), idx, c.window_blk0,
+                                        c.n_win_blk, scale=c.scale, err=err, qblk_order=order)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, idx.cpu().numpy(), c.window_blk0,
+                                           c.block, c.scale)
+    assert_bf16_close(o, ro, "sparse O (grouped order)")
+    assert_lse_close(l, rl, "sparse LSE (grouped order)")
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_block_sparse_random_query_block_order(seed):
+    c = _small_sparse(seed=86 + seed, qf=3)
+    sel = W.random_selection(20 + seed, c.B * c.H, c.n_qblk, c.n_win_blk, 4)
+    rng = np.random.default_rng(90 + seed)
+    perm = np.stack([rng.permutation(c.n_qblk) for _ in range(c.B * c.H)]).astype(np.int32)
+    err = err_word()
+    o, l = vk().chunk_attn_block_sparse(c.q.to(DEV), c.k.to(DEV), c.v.to(DEV),
+                                        torch.from_numpy(c.persist_idx).to(DEV), torch.from_numpy(sel).to(DEV),
+                                        c.window_blk0, c.n_win_blk, scale=c.scale, err=err,
+                                        qblk_order=torch.from_numpy(perm).to(DEV))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel, c.window_blk0, c.block, c.scale)
+    assert_bf16_close(o, ro, "sparse O (random order)")
+    assert_lse_close(l, rl, "sparse LSE (random order)")
+
+
+@pytest.mark.parametrize("frac", [W.SPARSE_TOPK_FRACTIONS[0], W.SPARSE_TOPK_FRACTIONS[2]])
+def test_full_sparse_config_grouped_sampled(frac):
+    c = W.cfg_sparse()
+    K = W.topk_for_fraction(frac, c.n_win_blk)
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    idx, _, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
+    err = err_word()
+    o, l = vk().chunk_attn_block_sparse(q, k, v, torch.from_numpy(c.persist_idx).to(DEV), idx,
+                                        c.window_blk0, c.n_win_blk, scale=c.scale, err=err, qblk_order=order)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    sel = idx.cpu().numpy()
+    heads, qblocks = [0, 5, 11], [0, 1, 36, 70, 71]
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel, c.window_blk0, c.block, c.scale,
+                                           heads=heads, qblocks=qblocks)
+    rows = [r for j in qblocks for r in range(j * 64, j * 64 + 64)]
+    assert_bf16_close(to_np(o)[:, rows][:, :, heads], ro[:, rows][:, :, heads], f"grouped sparse K={K}")
+    assert_lse_close(to_np(l)[:, heads][:, :, rows], rl[:, heads][:, :, rows], f"grouped sparse LSE K={K}")
+
+
+def test_sparse_bad_query_block_order_sets_error_word():
+    c = _small_sparse(seed=88)
+    sel = W.random_selection(5, c.B * c.H, c.n_qblk, c.n_win_blk, 3)
+    perm = np.tile(np.arange(c.n_qblk, dtype=np.int32), (c.B * c.H, 1))
+    perm[1, 2] = c.n_qblk + 3  # not a query block
+    err = err_word()
+    vk().chunk_attn_block_sparse(c.q.to(DEV), c.k.to(DEV), c.v.to(DEV), torch.from_numpy(c.persist_idx).to(DEV),
+                                 torch.from_numpy(sel).to(DEV), c.window_blk0, c.n_win_blk, scale=c.scale, err=err,
+                                 qblk_order=torch.from_numpy(perm).to(DEV))
+    torch.cuda.synchronize()
+    assert int(err.item()) == vk().DEVERR_BAD_INDEX
+
+
 # ---------------------------------------------------------------------------
 # mode 3: ragged per-head cache
 # ---------------------------------------------------------------------------
