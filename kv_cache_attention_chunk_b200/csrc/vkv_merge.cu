@@ -24,7 +24,10 @@ struct MergeParams {
   long long n_chunks;  // B * Lq * H * (d / 8)
 };
 
-constexpr int kMergePos = 8;  // consecutive (b, i) query positions per thread
+#ifndef VKV_MERGE_POS
+#define VKV_MERGE_POS 4
+#endif
+constexpr int kMergePos = VKV_MERGE_POS;  // consecutive (b, i) query positions per thread
 
 // grid: x = ceil(B * Lq / kMergePos) position groups, y = column blocks of at
 // most 256 threads (H * d/8 columns split as evenly as whole warps allow).

@@ -6,9 +6,9 @@
 // Two kernels on the caller's stream:
 //   pool_kernel     mean of every 64-row block of Q and of the window part of K,
 //                   in fp32, written to the caller's workspace.  One CTA of 256
-//                   threads per (block, batch, group of 256/d heads): the group's
+//                   threads per (block, batch, group of 512/d heads): the group's
 //                   contiguous slice of each row is read with 16-byte loads,
-//                   8 rows per thread in flight; row groups are combined in
+//                   16 rows per thread in flight; row groups are combined in
 //                   shared memory.  HBM-bound.
 //   select_kernel   one CTA per (batch*head, 8 query blocks): the pooled keys
 //                   are copied to shared memory 160 blocks at a time (cp.async),
@@ -53,17 +53,23 @@ struct PoolParams {
   float* kbar;  // [B*H][n_win][d]
 };
 
-// Heads per pooling CTA: a contiguous 512-byte slice of each row (2 heads at
-// d = 128, 4 at d = 64), 8 rows per thread in flight.
+// Heads per pooling CTA: a contiguous 1024-byte slice of each row (4 heads at
+// d = 128, 8 at d = 64), 16 rows per thread in flight.
+#ifndef VKV_POOL_SLICE
+#define VKV_POOL_SLICE 1024
+#endif
 template <int D>
-__host__ __device__ constexpr int pool_heads() { return 256 / D; }
+__host__ __device__ constexpr int pool_heads() { return VKV_POOL_SLICE / (2 * D) > 0 ? VKV_POOL_SLICE / (2 * D) : 1; }
 
 // grid: x = block index over n_qblk + n_win, y = b * ceil(H / kPoolHeads) + head group;
 // 256 threads.  Thread (g, c): column c = (head, 16-byte chunk) of the head
 // group's slice, rows g*RPG .. g*RPG + RPG - 1 of the 64-row block; the row
 // groups are combined in shared memory.
 template <int D>
-__global__ void __launch_bounds__(256, 4) pool_kernel(const PoolParams p) {
+#ifndef VKV_POOL_MINB
+#define VKV_POOL_MINB 2
+#endif
+__global__ void __launch_bounds__(256, VKV_POOL_MINB) pool_kernel(const PoolParams p) {
   constexpr int kPoolHeads = pool_heads<D>();
   constexpr int CPR = D / 8;                  // 16-byte chunks per head row
   constexpr int COLS = kPoolHeads * CPR;      // columns of the slice
@@ -179,6 +185,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) select_kernel(const SelParams 
   const int j = j0 + warp;
   const bool active = warp < nq;
   VKV_SEL_STAMP(0);
+  griddep_launch_dependents();  // the (small) order kernel may be scheduled alongside
   griddep_wait();  // the pooling kernel before this one on the stream has completed
   VKV_SEL_STAMP(1);
   const float* qsrc = p.qbar + ((size_t)s * p.n_qblk + j0) * D;
@@ -304,6 +311,7 @@ constexpr int kOrderMaxQblk = 4096;  // signatures of one (batch, head) in share
 
 __global__ void __launch_bounds__(256) order_kernel(const OrderParams p) {
   extern __shared__ unsigned long long sig[];
+  griddep_wait();  // the selection kernel before this one on the stream has completed
   const int s = blockIdx.x;
   const int* rows = p.sel + (size_t)s * p.n_qblk * p.topk;
   for (int j = threadIdx.x; j < p.n_qblk; j += blockDim.x) {
@@ -333,8 +341,18 @@ bool launch_order(const int* sel, int* order, int BH, int n_qblk, int topk, cuda
   op.order = order;
   op.n_qblk = n_qblk;
   op.topk = topk;
-  order_kernel<<<BH, 256, (size_t)n_qblk * sizeof(unsigned long long), st>>>(op);
-  return cudaGetLastError() == cudaSuccess;
+  // programmatic dependent launch: set-up overlaps the selection kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = (size_t)n_qblk * sizeof(unsigned long long);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, order_kernel, op) == cudaSuccess;
 }
 
 // Instantiation by head dimension and by window size (candidates per lane).
