@@ -21,6 +21,7 @@ of the same workload); under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -351,6 +352,26 @@ def extras(dev, peaks):
                          "target": "t(K)/t(144) = visited fraction: slope 1, intercept 0"}
     out["sparse"] = sp
     del q, k, v
+    # head-aware compaction of a dense cache into the ragged one (config-4 shape and policies)
+    ft, hist, cur, recent = 1560, 60, 3, 2
+    rules = [(vkv.HEAD_ANCHOR, 8)] * 4 + [(vkv.HEAD_WAVE, p) for p in (2, 3, 4, 5)] + [(vkv.HEAD_VEIL, 8)] * 4
+    g = torch.Generator(device=dev).manual_seed(12)
+    kd = torch.randn((1, (hist + cur) * ft, 12, 128), generator=g, device=dev).to(torch.bfloat16)
+    vd = torch.randn((1, (hist + cur) * ft, 12, 128), generator=g, device=dev).to(torch.bfloat16)
+    kc, vc, cuc, cuh = vkv.compact_cache(kd, vd, rules, ft, hist, cur, recent)
+    a = vkv.vkv_compact_args()
+    a.B, a.H, a.d, a.frame_tokens, a.hist_frames, a.cur_frames, a.recent_frames = 1, 12, 128, ft, hist, cur, recent
+    a.k_src, a.v_src = vkv.tensor_desc(kd), vkv.tensor_desc(vd)
+    rr = (vkv.vkv_head_rule * 12)(*[vkv.vkv_head_rule(int(pp), int(x)) for pp, x in rules])
+    a.rules = ctypes.cast(rr, ctypes.POINTER(vkv.vkv_head_rule))
+    a.k_out, a.v_out, a.out_rows, a.cu_seqlens = kc.data_ptr(), vc.data_ptr(), kc.shape[0], cuc.data_ptr()
+    ms = statistics.median(timed(lambda: vkv.vkv_compact_cache(a, st.cuda_stream), 30, st, flush))
+    rows = int(cuh[-1])
+    merged_rows = 4 * 4 * ft  # four veil heads, four merged pairs each
+    nbytes = 2 * (rows + merged_rows) * 128 * 2 + 2 * rows * 128 * 2
+    out["compaction_cfg4"] = {"ms": ms, "gbs": nbytes / ms / 1e6, "bytes": nbytes,
+                              "frac_hbm": nbytes / ms / 1e6 / peaks["hbm_gbs"]}
+    del kd, vd, kc, vc
     # ragged per-head cache
     c = W.cfg_ragged()
     q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)

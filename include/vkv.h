@@ -242,6 +242,68 @@ vkv_status vkv_block_select(const vkv_select_args* args, vkv_stream_t stream);
 vkv_status vkv_block_select_noalloc(const vkv_select_args* args, vkv_stream_t stream);
 
 /*
+ * Head-aware cache compaction (Pyramid Forcing summary, methodology section 2
+ * "head-aware pyramid KV cache policies" and section 3 "flattened sequences
+ * with boundary indices"): every (batch, head) keeps its own subset of the
+ * frames of a dense cache, and the kept frames of all heads are packed into
+ * one flattened ragged cache with boundary offsets, in one launch.
+ *
+ * Source frames: 0 .. hist_frames-1 are history (frame 0 is the sink), then
+ * cur_frames frames of the current chunk; frame f is cache rows
+ * [f*frame_tokens, (f+1)*frame_tokens).  Every head keeps, in this order:
+ * the sink, its policy's middle frames (chosen from [1, hist_frames -
+ * recent_frames - 1]), the last recent_frames history frames, and the current
+ * frames.  Middle frames by policy:
+ *   FULL    every middle frame;
+ *   ANCHOR  `param` frames evenly spaced over the middle range, both ends
+ *           included (frame lo + floor(i * (hi - lo) / (param - 1)));
+ *   WAVE    middle frames f with (hist_frames - f) % param == 0 (period
+ *           `param`, aligned to the current chunk);
+ *   VEIL    the last `param` (even) middle frames, merged in adjacent pairs:
+ *           a pair is stored once, as the fp32 mean of its two bf16 frames
+ *           rounded to nearest-even bf16.
+ */
+typedef enum {
+  VKV_HEAD_FULL = 0,
+  VKV_HEAD_ANCHOR = 1,
+  VKV_HEAD_WAVE = 2,
+  VKV_HEAD_VEIL = 3
+} vkv_head_policy;
+
+typedef struct {
+  int32_t policy; /* vkv_head_policy */
+  int32_t param;  /* ANCHOR: frames kept (1..middle); WAVE: period >= 1; VEIL: frames merged (even, <= middle) */
+} vkv_head_rule;
+
+#define VKV_COMPACT_MAX_SEQS 512      /* B*H */
+#define VKV_COMPACT_MAX_PIECES 1024   /* stored frames (or merged pairs) over all sequences */
+
+typedef struct {
+  int32_t B, H, d;          /* d in {64, 128}                                        */
+  int32_t frame_tokens;     /* rows per frame                                         */
+  int32_t hist_frames;      /* history frames (>= 1 + recent_frames)                  */
+  int32_t cur_frames;       /* current-chunk frames after the history (>= 0)          */
+  int32_t recent_frames;    /* history frames every head keeps before the chunk (>= 0) */
+  vkv_tensor k_src;         /* [B, (hist_frames + cur_frames) * frame_tokens, H, d]   */
+  vkv_tensor v_src;         /* same layout as k_src                                   */
+  const vkv_head_rule* rules; /* HOST [H]: the rule of head h (same for every batch)  */
+  void* k_out;              /* DEVICE bf16 [rows, d], rows contiguous, sequence s = b*H + h at rows [cu[s], cu[s+1]) */
+  void* v_out;              /* same                                                   */
+  int64_t out_rows;         /* capacity of k_out / v_out in rows                      */
+  int32_t* cu_seqlens;      /* DEVICE int32 [B*H + 1], written by the launch          */
+  int32_t* cu_seqlens_host; /* optional HOST int32 [B*H + 1], filled before the call returns */
+} vkv_compact_args;
+
+/* Rows the compacted cache needs (>= 0), or -(vkv_status) for invalid arguments.
+ * Reads only the sizes and `rules`; no device work. */
+int64_t vkv_compact_rows(const vkv_compact_args* args);
+
+/* Writes k_out, v_out and cu_seqlens on `stream` (one kernel launch).  Returns
+ * VKV_ERR_RANGE when out_rows is too small, VKV_ERR_UNSUPPORTED beyond
+ * VKV_COMPACT_MAX_SEQS sequences or VKV_COMPACT_MAX_PIECES stored frames. */
+vkv_status vkv_compact_cache(const vkv_compact_args* args, vkv_stream_t stream);
+
+/*
  * vkv_lse_merge -- exact recombination of two partial attentions over disjoint
  * key sets (ISPA summary, section 2 step 1 and contribution 2):
  *   M = max(lse_a, lse_b),  w_x = exp(lse_x - M),
@@ -261,7 +323,8 @@ const char* vkv_status_string(vkv_status s);
 int32_t vkv_version(void);
 
 /* sizeof() of the ABI structs, for bindings to check their layout:
- * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment; -1 otherwise. */
+ * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment,
+ * 4 vkv_compact_args, 5 vkv_head_rule; -1 otherwise. */
 int32_t vkv_abi_sizeof(int32_t which);
 
 #ifdef __cplusplus

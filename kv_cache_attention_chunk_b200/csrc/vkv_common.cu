@@ -88,7 +88,7 @@ extern "C" const char* vkv_status_string(vkv_status s) {
   return "unknown status";
 }
 
-extern "C" int32_t vkv_version(void) { return 101; }
+extern "C" int32_t vkv_version(void) { return 200; }
 
 extern "C" int32_t vkv_abi_sizeof(int32_t which) {
   switch (which) {
@@ -96,6 +96,8 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
     case 1: return (int32_t)sizeof(vkv_select_args);
     case 2: return (int32_t)sizeof(vkv_tensor);
     case 3: return (int32_t)sizeof(vkv_segment);
+    case 4: return (int32_t)sizeof(vkv_compact_args);
+    case 5: return (int32_t)sizeof(vkv_head_rule);
   }
   return -1;
 }

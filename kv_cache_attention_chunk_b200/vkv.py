@@ -75,6 +75,23 @@ class vkv_select_args(ctypes.Structure):
     ]
 
 
+class vkv_head_rule(ctypes.Structure):
+    _fields_ = [("policy", c_int32), ("param", c_int32)]
+
+
+class vkv_compact_args(ctypes.Structure):
+    _fields_ = [
+        ("B", c_int32), ("H", c_int32), ("d", c_int32), ("frame_tokens", c_int32),
+        ("hist_frames", c_int32), ("cur_frames", c_int32), ("recent_frames", c_int32),
+        ("k_src", vkv_tensor), ("v_src", vkv_tensor),
+        ("rules", POINTER(vkv_head_rule)),
+        ("k_out", c_void_p), ("v_out", c_void_p), ("out_rows", c_int64),
+        ("cu_seqlens", c_void_p), ("cu_seqlens_host", POINTER(c_int32)),
+    ]
+
+
+HEAD_FULL, HEAD_ANCHOR, HEAD_WAVE, HEAD_VEIL = 0, 1, 2, 3
+
 _lib = None
 
 
@@ -104,7 +121,12 @@ def lib() -> ctypes.CDLL:
     L.vkv_version.restype = c_int32
     L.vkv_abi_sizeof.argtypes = [c_int32]
     L.vkv_abi_sizeof.restype = c_int32
-    for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment)):
+    L.vkv_compact_rows.argtypes = [POINTER(vkv_compact_args)]
+    L.vkv_compact_rows.restype = c_int64
+    L.vkv_compact_cache.argtypes = [POINTER(vkv_compact_args), c_void_p]
+    L.vkv_compact_cache.restype = c_int32
+    for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
+                            vkv_head_rule)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
             raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
                                f"binding {ctypes.sizeof(st)} B")
@@ -130,6 +152,14 @@ def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
 def vkv_block_select_noalloc(args: vkv_select_args, stream: int | None) -> int:
     """vkv_block_select with the library's own fixed scratch array (no workspace argument)."""
     return int(lib().vkv_block_select_noalloc(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_compact_rows(args: vkv_compact_args) -> int:
+    return int(lib().vkv_compact_rows(ctypes.byref(args)))
+
+
+def vkv_compact_cache(args: vkv_compact_args, stream: int | None) -> int:
+    return int(lib().vkv_compact_cache(ctypes.byref(args), c_void_p(stream or 0)))
 
 
 def vkv_block_select_workspace_size(B, H, Lq, n_win_blk, block, d) -> int:
@@ -316,3 +346,33 @@ def lse_merge(o_a, lse_a, o_b, lse_b, stream=None, out=None):
     _check(vkv_lse_merge(tensor_desc(o_a), lse_a.data_ptr(), tensor_desc(o_b), lse_b.data_ptr(),
                          tensor_desc(o), l.data_ptr(), B, H, Lq, d, _stream(stream)), "vkv_lse_merge")
     return o, l
+
+
+def compact_cache(k, v, rules, frame_tokens, hist_frames, cur_frames, recent_frames, stream=None):
+    """Head-aware compaction of a dense cache into a flattened ragged cache.
+
+    k, v: device bf16 [B, L, H, d] with L = (hist_frames + cur_frames) * frame_tokens;
+    rules: one (policy, param) per head (HEAD_FULL / HEAD_ANCHOR / HEAD_WAVE / HEAD_VEIL).
+    Returns (k_flat [rows, d], v_flat, cu_seqlens on the device, cu_seqlens on the host).
+    """
+    B, L, H, d = k.shape
+    a = vkv_compact_args()
+    a.B, a.H, a.d = B, H, d
+    a.frame_tokens, a.hist_frames, a.cur_frames, a.recent_frames = (int(frame_tokens), int(hist_frames),
+                                                                     int(cur_frames), int(recent_frames))
+    a.k_src = tensor_desc(k)
+    a.v_src = tensor_desc(v)
+    rr = (vkv_head_rule * H)(*[vkv_head_rule(int(p), int(x)) for p, x in rules])
+    a.rules = ctypes.cast(rr, POINTER(vkv_head_rule))
+    rows = vkv_compact_rows(a)
+    if rows < 0:
+        raise VkvError(-rows, "vkv_compact_rows")
+    k_out = torch.empty((rows, d), dtype=k.dtype, device=k.device)
+    v_out = torch.empty((rows, d), dtype=v.dtype, device=v.device)
+    cu_dev = torch.empty(B * H + 1, dtype=torch.int32, device=k.device)
+    cu_host = np.zeros(B * H + 1, dtype=np.int32)
+    a.k_out, a.v_out, a.out_rows = k_out.data_ptr(), v_out.data_ptr(), rows
+    a.cu_seqlens = cu_dev.data_ptr()
+    a.cu_seqlens_host = cu_host.ctypes.data_as(POINTER(c_int32))
+    _check(vkv_compact_cache(a, _stream(stream)), "vkv_compact_cache")
+    return k_out, v_out, cu_dev, cu_host

@@ -218,3 +218,32 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(vkv, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         vkv.lib()
+
+
+def test_compact_rows_of_the_pyramid_policies():
+    """Host planning of the head-aware compaction: per-head frame lists of the config-4 readings."""
+    from kv_cache_attention_chunk_b200 import vkv
+    a = vkv.vkv_compact_args()
+    a.B, a.H, a.d, a.frame_tokens, a.hist_frames, a.cur_frames, a.recent_frames = 1, 12, 128, 1560, 60, 3, 2
+    rules = [(vkv.HEAD_ANCHOR, 8)] * 4 + [(vkv.HEAD_WAVE, p) for p in (2, 3, 4, 5)] + [(vkv.HEAD_VEIL, 8)] * 4
+    rr = (vkv.vkv_head_rule * 12)(*[vkv.vkv_head_rule(p, x) for p, x in rules])
+    a.rules = ctypes.cast(rr, ctypes.POINTER(vkv.vkv_head_rule))
+    assert vkv.vkv_compact_rows(a) == 299520
+    a.B = 2
+    assert vkv.vkv_compact_rows(a) == 2 * 299520
+    rr[9] = vkv.vkv_head_rule(vkv.HEAD_VEIL, 3)  # odd merge count
+    assert vkv.vkv_compact_rows(a) == -2  # -VKV_ERR_SHAPE
+
+
+def test_compact_cache_rejects_small_output_without_a_gpu():
+    from kv_cache_attention_chunk_b200 import vkv
+    a = vkv.vkv_compact_args()
+    a.B, a.H, a.d, a.frame_tokens, a.hist_frames, a.cur_frames, a.recent_frames = 1, 1, 64, 16, 4, 1, 1
+    rr = (vkv.vkv_head_rule * 1)(vkv.vkv_head_rule(vkv.HEAD_FULL, 0))
+    a.rules = ctypes.cast(rr, ctypes.POINTER(vkv.vkv_head_rule))
+    assert vkv.vkv_compact_rows(a) == 5 * 16
+    a.k_src = vkv.vkv_tensor(64, 64, 64, 64)
+    a.v_src = vkv.vkv_tensor(64, 64, 64, 64)
+    a.k_out, a.v_out, a.cu_seqlens = 64, 64, 64
+    a.out_rows = 79
+    assert vkv.vkv_compact_cache(a, None) == 4  # VKV_ERR_RANGE: checked before any device work
