@@ -212,11 +212,27 @@ typedef struct {
    * vkv_chunk_attn as qblk_order.  Not part of the pages' method: it only
    * groups work. */
   int32_t* out_order;
+  /* optional DEVICE fp32 [B*H][n_win_blk][d] (NULL = pool from k): the window
+   * blocks' means as written by vkv_block_pool for blocks [window_blk0,
+   * window_blk0 + n_win_blk), kept by the caller as blocks enter the cache
+   * (Sparse Forcing summary, section 2 component 2: one representative per
+   * block).  Then only the query blocks are pooled and `k` is not read. */
+  const float* kbar;
 } vkv_select_args;
 
 size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,
                                        int32_t block, int32_t d);
 vkv_status vkv_block_select(const vkv_select_args* args, vkv_stream_t stream);
+
+/*
+ * vkv_block_pool -- the representative (fp32 mean of the rows) of each of the
+ * 64-row blocks [blk0, blk0 + n_blk) of x [B, L, H, d] (Sparse Forcing summary,
+ * section 2 component 2), written to out [B*H][n_blk][d] (DEVICE fp32, caller
+ * owned).  The same arithmetic as vkv_block_select's own pooling, so a
+ * selection from cached representatives equals one that pools them itself.
+ */
+vkv_status vkv_block_pool(vkv_tensor x, int32_t B, int32_t L, int32_t H, int32_t d, int32_t blk0,
+                          int32_t n_blk, float* out, vkv_stream_t stream);
 
 /*
  * vkv_block_select_noalloc -- vkv_block_select for callers that cannot allocate.

@@ -20,6 +20,7 @@
 //                   Launched as a programmatic dependent of the pooling kernel,
 //                   so its launch overlaps the pooling kernel's last CTAs.
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "vkv_internal.h"
@@ -415,23 +416,29 @@ extern "C" size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t 
   return (bytes + 255) & ~(size_t)255;
 }
 
-extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t stream) {
+namespace vkv {
+namespace {
+
+// Argument checks shared by both selection entry points (workspace excluded).
+vkv_status check_select_args(const vkv_select_args* a) {
   if (!a) return VKV_ERR_NULL;
   if (a->d != 64 && a->d != 128) return VKV_ERR_UNSUPPORTED;
   if (a->block != 64) return VKV_ERR_UNSUPPORTED;
   if (a->B <= 0 || a->H <= 0 || a->Lq <= 0 || a->Lkv <= 0) return VKV_ERR_SHAPE;
   if (a->n_win_blk < 1 || a->n_win_blk > 1024 || a->topk < 1 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
   if (a->window_blk0 < 0 || (long long)(a->window_blk0 + a->n_win_blk) * a->block > a->Lkv) return VKV_ERR_RANGE;
-  if (!a->q.ptr || !a->k.ptr || !a->out_idx) return VKV_ERR_NULL;
-  if (!tensor_aligned(a->q) || !tensor_aligned(a->k)) return VKV_ERR_ALIGN;
-  const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
-  if (!a->workspace || a->workspace_bytes < need) return VKV_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
+  if (!a->q.ptr || (!a->k.ptr && !a->kbar) || !a->out_idx) return VKV_ERR_NULL;
+  if (!tensor_aligned(a->q) || (!a->kbar && !tensor_aligned(a->k))) return VKV_ERR_ALIGN;
+  if (a->kbar && (reinterpret_cast<uintptr_t>(a->kbar) & 15u)) return VKV_ERR_ALIGN;
   if ((long long)a->B * a->H > 65535) return VKV_ERR_UNSUPPORTED;
   if (a->out_order && (a->Lq + a->block - 1) / a->block > kOrderMaxQblk) return VKV_ERR_UNSUPPORTED;
-  int dev = 0;
-  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return VKV_OK;
+}
+
+// Pooling (query blocks, and the window blocks unless cached), scoring and
+// top-K, and the optional query-block order, on `st`; `scratch` holds the
+// pooled vectors.
+vkv_status run_select(const vkv_select_args* a, float* scratch, cudaStream_t st) {
   const int BH = a->B * a->H;
   const int n_qblk = (a->Lq + 63) / 64;
   PoolParams pp;
@@ -446,10 +453,11 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   pp.n_qblk = n_qblk;
   pp.n_win = a->n_win_blk;
   pp.win_row0 = a->window_blk0 * a->block;
-  pp.qbar = reinterpret_cast<float*>(a->workspace);
+  pp.qbar = scratch;
   pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
   const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
-  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + ph - 1) / ph));
+  // with cached window representatives only the query blocks are pooled
+  const dim3 pg(n_qblk + (a->kbar ? 0 : a->n_win_blk), a->B * ((a->H + ph - 1) / ph));
   if (a->d == 128)
     pool_kernel<128><<<pg, 256, 0, st>>>(pp);
   else
@@ -457,7 +465,7 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   SelParams sp;
   sp.qbar = pp.qbar;
-  sp.kbar = pp.kbar;
+  sp.kbar = a->kbar ? a->kbar : pp.kbar;
   sp.BH = BH;
   sp.n_qblk = n_qblk;
   sp.n_win = a->n_win_blk;
@@ -469,6 +477,54 @@ extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t st
   if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   if (a->out_order && !launch_order(a->out_idx, a->out_order, BH, n_qblk, a->topk, st)) return VKV_ERR_CUDA;
+  return VKV_OK;
+}
+
+}  // namespace
+}  // namespace vkv
+
+extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t stream) {
+  const vkv_status chk = check_select_args(a);
+  if (chk != VKV_OK) return chk;
+  const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
+  if (!a->workspace || a->workspace_bytes < need) return VKV_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
+  return run_select(a, reinterpret_cast<float*>(a->workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" vkv_status vkv_block_pool(vkv_tensor x, int32_t B, int32_t L, int32_t H, int32_t d, int32_t blk0,
+                                     int32_t n_blk, float* out, vkv_stream_t stream) {
+  if (!x.ptr || !out) return VKV_ERR_NULL;
+  if (d != 64 && d != 128) return VKV_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || L <= 0 || n_blk <= 0 || blk0 < 0) return VKV_ERR_SHAPE;
+  if ((long long)(blk0 + n_blk) * 64 > L) return VKV_ERR_RANGE;
+  if (!tensor_aligned(x) || (reinterpret_cast<uintptr_t>(out) & 15u)) return VKV_ERR_ALIGN;
+  if ((long long)B * H > 65535) return VKV_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
+  // the window-block path of the selection's pooling kernel, with no query blocks
+  PoolParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.k = reinterpret_cast<const __nv_bfloat16*>(x.ptr);
+  pp.k_sb = x.sb; pp.k_st = x.st; pp.k_sh = x.sh;
+  pp.B = B;
+  pp.H = H;
+  pp.d = d;
+  pp.Lq = 0;
+  pp.n_qblk = 0;
+  pp.n_win = n_blk;
+  pp.win_row0 = blk0 * 64;
+  pp.kbar = out;
+  const int ph = d == 128 ? pool_heads<128>() : pool_heads<64>();
+  const dim3 pg(n_blk, B * ((H + ph - 1) / ph));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
+  else
+    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }
 
@@ -519,59 +575,13 @@ void* noalloc_scratch(int dev) {
 }  // namespace vkv
 
 extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_stream_t stream) {
-  if (!a) return VKV_ERR_NULL;
-  if (a->d != 64 && a->d != 128) return VKV_ERR_UNSUPPORTED;
-  if (a->block != 64) return VKV_ERR_UNSUPPORTED;
-  if (a->B <= 0 || a->H <= 0 || a->Lq <= 0 || a->Lkv <= 0) return VKV_ERR_SHAPE;
-  if (a->n_win_blk < 1 || a->n_win_blk > 1024 || a->topk < 1 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
-  if (a->window_blk0 < 0 || (long long)(a->window_blk0 + a->n_win_blk) * a->block > a->Lkv) return VKV_ERR_RANGE;
-  if (!a->q.ptr || !a->k.ptr || !a->out_idx) return VKV_ERR_NULL;
-  if (!tensor_aligned(a->q) || !tensor_aligned(a->k)) return VKV_ERR_ALIGN;
-  if ((long long)a->B * a->H > 65535) return VKV_ERR_UNSUPPORTED;
-  if (a->out_order && (a->Lq + a->block - 1) / a->block > kOrderMaxQblk) return VKV_ERR_UNSUPPORTED;
+  const vkv_status chk = check_select_args(a);
+  if (chk != VKV_OK) return chk;
   const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
   if (need > kNoallocScratchBytes) return VKV_ERR_WORKSPACE;  // larger than the fixed scratch array
   int dev = 0;
   if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
   void* scratch = noalloc_scratch(dev);
   if (!scratch) return VKV_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = a->B * a->H;
-  const int n_qblk = (a->Lq + 63) / 64;
-  PoolParams pp;
-  pp.q = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
-  pp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
-  pp.q_sb = a->q.sb; pp.q_st = a->q.st; pp.q_sh = a->q.sh;
-  pp.k_sb = a->k.sb; pp.k_st = a->k.st; pp.k_sh = a->k.sh;
-  pp.B = a->B;
-  pp.H = a->H;
-  pp.d = a->d;
-  pp.Lq = a->Lq;
-  pp.n_qblk = n_qblk;
-  pp.n_win = a->n_win_blk;
-  pp.win_row0 = a->window_blk0 * a->block;
-  pp.qbar = reinterpret_cast<float*>(scratch);
-  pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
-  dim3 pg(n_qblk + a->n_win_blk, a->B * ((a->H + ph - 1) / ph));
-  if (a->d == 128)
-    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
-  else
-    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
-  SelParams sp;
-  sp.qbar = pp.qbar;
-  sp.kbar = pp.kbar;
-  sp.BH = BH;
-  sp.n_qblk = n_qblk;
-  sp.n_win = a->n_win_blk;
-  sp.topk = a->topk;
-  sp.out_idx = a->out_idx;
-  sp.out_scores = a->out_scores;
-  const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
-  const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
-  if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
-  if (a->out_order && !launch_order(a->out_idx, a->out_order, BH, n_qblk, a->topk, st)) return VKV_ERR_CUDA;
-  return VKV_OK;
+  return run_select(a, reinterpret_cast<float*>(scratch), reinterpret_cast<cudaStream_t>(stream));
 }

@@ -72,6 +72,7 @@ class vkv_select_args(ctypes.Structure):
         ("workspace", c_void_p), ("workspace_bytes", c_size_t),
         ("err_word", c_void_p),
         ("out_order", c_void_p),
+        ("kbar", c_void_p),
     ]
 
 
@@ -121,6 +122,9 @@ def lib() -> ctypes.CDLL:
     L.vkv_version.restype = c_int32
     L.vkv_abi_sizeof.argtypes = [c_int32]
     L.vkv_abi_sizeof.restype = c_int32
+    L.vkv_block_pool.argtypes = [vkv_tensor, c_int32, c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p,
+                                 c_void_p]
+    L.vkv_block_pool.restype = c_int32
     L.vkv_compact_rows.argtypes = [POINTER(vkv_compact_args)]
     L.vkv_compact_rows.restype = c_int64
     L.vkv_compact_cache.argtypes = [POINTER(vkv_compact_args), c_void_p]
@@ -152,6 +156,10 @@ def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
 def vkv_block_select_noalloc(args: vkv_select_args, stream: int | None) -> int:
     """vkv_block_select with the library's own fixed scratch array (no workspace argument)."""
     return int(lib().vkv_block_select_noalloc(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_block_pool(x: vkv_tensor, B, L, H, d, blk0, n_blk, out, stream: int | None) -> int:
+    return int(lib().vkv_block_pool(x, B, L, H, d, blk0, n_blk, c_void_p(out), c_void_p(stream or 0)))
 
 
 def vkv_compact_rows(args: vkv_compact_args) -> int:
@@ -303,11 +311,13 @@ def chunk_attn_ragged(q, k_flat, v_flat, cu_seqlens, cu_seqlens_host=None, scale
 
 
 def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=False, err=None, stream=None,
-                 out_idx=None, order=False, out_order=None):
+                 out_idx=None, order=False, out_order=None, kbar=None):
     """Top-K window blocks per 64-query block; returns (idx [B*H, nQblk, topk], scores or None).
 
     With order=True (or an out_order tensor) also returns the query-block order
     [B*H, nQblk] that groups blocks with similar selections: (idx, scores, order).
+    kbar (optional device fp32 [B*H, n_win_blk, d], from block_pool) supplies the
+    window blocks' representatives, so only the query blocks are pooled.
     """
     B, Lq, H, d = q.shape
     n_qblk = -(-Lq // 64)
@@ -330,6 +340,9 @@ def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=Fals
     a.workspace = workspace.data_ptr()
     a.workspace_bytes = workspace.numel() * workspace.element_size()
     a.err_word = err.data_ptr() if err is not None else None
+    if kbar is not None:
+        kbar = kbar.contiguous()
+        a.kbar = kbar.data_ptr()
     if order and out_order is None:
         out_order = torch.empty((B * H, n_qblk), dtype=torch.int32, device=q.device)
     if out_order is not None:
@@ -338,6 +351,15 @@ def block_select(q, k, window_blk0, n_win_blk, topk, workspace=None, scores=Fals
     if out_order is not None:
         return idx, sc, out_order
     return idx, sc
+
+
+def block_pool(x, blk0, n_blk, stream=None, out=None):
+    """fp32 mean of each 64-row block [blk0, blk0 + n_blk) of x [B, L, H, d] -> [B*H, n_blk, d]."""
+    B, L, H, d = x.shape
+    o = out if out is not None else torch.empty((B * H, n_blk, d), dtype=torch.float32, device=x.device)
+    _check(vkv_block_pool(tensor_desc(x), B, L, H, d, int(blk0), int(n_blk), o.data_ptr(), _stream(stream)),
+           "vkv_block_pool")
+    return o
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, stream=None, out=None):

@@ -363,6 +363,35 @@ def test_sparse_bad_query_block_order_sets_error_word():
     assert int(err.item()) == vk().DEVERR_BAD_INDEX
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_block_pool_matches_oracle(d):
+    c = _small_sparse(seed=89, d=d)
+    k = c.k.to(DEV)
+    blk0, n = 3, 20  # the cache holds 7 frames x 4 blocks
+    kb = vk().block_pool(k, blk0, n)
+    torch.cuda.synchronize()
+    kk = oracle.to64(c.k)
+    ref = np.stack([oracle.pool_blocks(kk[b, blk0 * 64:(blk0 + n) * 64, h], 64)
+                    for b in range(c.B) for h in range(c.H)])
+    assert np.abs(to_np(kb) - ref).max() < 1e-5
+
+
+@pytest.mark.parametrize("topk", [3, 9])
+def test_block_select_with_cached_representatives(topk):
+    c = W.cfg_sparse()
+    q, k = c.q.to(DEV), c.k.to(DEV)
+    idx, sc, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, topk, scores=True, order=True)
+    kbar = vk().block_pool(k, c.window_blk0, c.n_win_blk)
+    # the cached path must not need k: pass a tensor of the right shape filled with garbage
+    junk = torch.full_like(k, float("nan"))
+    idx2, sc2, order2 = vk().block_select(q, junk, c.window_blk0, c.n_win_blk, topk, scores=True, order=True,
+                                          kbar=kbar)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(sc, sc2)
+    assert torch.equal(order, order2)
+
+
 # ---------------------------------------------------------------------------
 # mode 3: ragged per-head cache
 # ---------------------------------------------------------------------------
