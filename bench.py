@@ -351,6 +351,14 @@ def extras(dev, peaks):
     ms_cached = statistics.median(timed(lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws,
                                                                  out_idx=idx, out_order=order, kbar=kbar),
                                         30, st, flush))
+    # persistent-memory update: the oldest window frame (24 blocks) leaves the window
+    pidx, _ = vkv.persist_update(q, k, pers, c.window_blk0, 24)
+    pws = torch.empty(vkv.vkv_persist_update_workspace_size(1, 12, c.Lq, pers.shape[1], 24, 64, 128),
+                      dtype=torch.uint8, device=dev)
+    ms_pu = statistics.median(timed(lambda: vkv.persist_update(q, k, pers, c.window_blk0, 24, out_idx=pidx,
+                                                               workspace=pws), 30, st, flush))
+    pu_bytes = (c.Lq + (pers.shape[1] + 24) * 64) * 12 * 128 * 2
+    sp["persist_update"] = {"ms": ms_pu, "gbs": pu_bytes / ms_pu / 1e6, "candidates": pers.shape[1] + 24}
     q_bytes = c.Lq * 12 * 128 * 2
     sp["select_cached_representatives"] = {"K": K, "select_ms": ms_cached, "q_read_gbs": q_bytes / ms_cached / 1e6,
                                            "window_pool_ms": ms_pool}

@@ -258,6 +258,43 @@ vkv_status vkv_block_pool(vkv_tensor x, int32_t B, int32_t L, int32_t H, int32_t
 vkv_status vkv_block_select_noalloc(const vkv_select_args* args, vkv_stream_t stream);
 
 /*
+ * vkv_persist_update -- persistent-memory management (Sparse Forcing summary,
+ * section 2 component 1 "Structured Memory Decomposition": the blocks evicted
+ * from the local window are candidates, and the top C by coarse score are
+ * kept in, or replace blocks of, the persistent memory).
+ *
+ * Per (batch b, head h): the candidates are the current persistent blocks
+ * persist_idx[b*H+h][0..C) and the evicted blocks [evict_blk0, evict_blk0 +
+ * n_evict); each is scored by <qbar, kbar_c>, where qbar is the mean of the
+ * chunk's Lq query rows and kbar_c the mean of block c's rows (no softmax
+ * scale: a positive factor does not change the ranking).  The C highest
+ * scores are kept (equal scores: the lower block id first) and written to
+ * out_idx [B*H][C] in ascending block order.  out_scores (optional, fp32
+ * [B*H][C + n_evict]) receives the candidates' scores, persistent ones first.
+ * A persistent id outside [0, Lkv/block) or inside the evicted range raises
+ * VKV_DEVERR_BAD_INDEX (that candidate is dropped).
+ */
+typedef struct {
+  int32_t B, H, d, block;    /* d in {64, 128}; block = 64                         */
+  int32_t Lq, Lkv;           /* query rows; cache rows                             */
+  vkv_tensor q;              /* [B, Lq, H, d]                                      */
+  vkv_tensor k;              /* [B, Lkv, H, d]                                     */
+  const int32_t* persist_idx;/* DEVICE int32 [B*H][n_persist], absolute block ids  */
+  int32_t n_persist;         /* C, 1..1024                                         */
+  int32_t evict_blk0;        /* first evicted block                                */
+  int32_t n_evict;           /* evicted blocks, 0..1024 (C + n_evict <= 2048)      */
+  int32_t* out_idx;          /* DEVICE int32 [B*H][n_persist]                      */
+  float* out_scores;         /* optional DEVICE fp32 [B*H][n_persist + n_evict]    */
+  void* workspace;           /* DEVICE, >= vkv_persist_update_workspace_size(), 256-byte aligned */
+  size_t workspace_bytes;
+  int32_t* err_word;         /* optional DEVICE int32                              */
+} vkv_persist_args;
+
+size_t vkv_persist_update_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_persist,
+                                         int32_t n_evict, int32_t block, int32_t d);
+vkv_status vkv_persist_update(const vkv_persist_args* args, vkv_stream_t stream);
+
+/*
  * Head-aware cache compaction (Pyramid Forcing summary, methodology section 2
  * "head-aware pyramid KV cache policies" and section 3 "flattened sequences
  * with boundary indices"): every (batch, head) keeps its own subset of the
@@ -340,7 +377,7 @@ int32_t vkv_version(void);
 
 /* sizeof() of the ABI structs, for bindings to check their layout:
  * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment,
- * 4 vkv_compact_args, 5 vkv_head_rule; -1 otherwise. */
+ * 4 vkv_compact_args, 5 vkv_head_rule, 6 vkv_persist_args; -1 otherwise. */
 int32_t vkv_abi_sizeof(int32_t which);
 
 #ifdef __cplusplus

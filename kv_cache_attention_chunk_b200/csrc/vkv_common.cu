@@ -98,6 +98,7 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
     case 3: return (int32_t)sizeof(vkv_segment);
     case 4: return (int32_t)sizeof(vkv_compact_args);
     case 5: return (int32_t)sizeof(vkv_head_rule);
+    case 6: return (int32_t)sizeof(vkv_persist_args);
   }
   return -1;
 }

@@ -93,6 +93,19 @@ class vkv_compact_args(ctypes.Structure):
 
 HEAD_FULL, HEAD_ANCHOR, HEAD_WAVE, HEAD_VEIL = 0, 1, 2, 3
 
+
+class vkv_persist_args(ctypes.Structure):
+    _fields_ = [
+        ("B", c_int32), ("H", c_int32), ("d", c_int32), ("block", c_int32),
+        ("Lq", c_int32), ("Lkv", c_int32),
+        ("q", vkv_tensor), ("k", vkv_tensor),
+        ("persist_idx", c_void_p), ("n_persist", c_int32),
+        ("evict_blk0", c_int32), ("n_evict", c_int32),
+        ("out_idx", c_void_p), ("out_scores", c_void_p),
+        ("workspace", c_void_p), ("workspace_bytes", c_size_t),
+        ("err_word", c_void_p),
+    ]
+
 _lib = None
 
 
@@ -129,8 +142,12 @@ def lib() -> ctypes.CDLL:
     L.vkv_compact_rows.restype = c_int64
     L.vkv_compact_cache.argtypes = [POINTER(vkv_compact_args), c_void_p]
     L.vkv_compact_cache.restype = c_int32
+    L.vkv_persist_update_workspace_size.argtypes = [c_int32] * 7
+    L.vkv_persist_update_workspace_size.restype = c_size_t
+    L.vkv_persist_update.argtypes = [POINTER(vkv_persist_args), c_void_p]
+    L.vkv_persist_update.restype = c_int32
     for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
-                            vkv_head_rule)):
+                            vkv_head_rule, vkv_persist_args)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
             raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
                                f"binding {ctypes.sizeof(st)} B")
@@ -160,6 +177,14 @@ def vkv_block_select_noalloc(args: vkv_select_args, stream: int | None) -> int:
 
 def vkv_block_pool(x: vkv_tensor, B, L, H, d, blk0, n_blk, out, stream: int | None) -> int:
     return int(lib().vkv_block_pool(x, B, L, H, d, blk0, n_blk, c_void_p(out), c_void_p(stream or 0)))
+
+
+def vkv_persist_update_workspace_size(B, H, Lq, n_persist, n_evict, block, d) -> int:
+    return int(lib().vkv_persist_update_workspace_size(B, H, Lq, n_persist, n_evict, block, d))
+
+
+def vkv_persist_update(args: vkv_persist_args, stream: int | None) -> int:
+    return int(lib().vkv_persist_update(ctypes.byref(args), c_void_p(stream or 0)))
 
 
 def vkv_compact_rows(args: vkv_compact_args) -> int:
@@ -398,3 +423,33 @@ def compact_cache(k, v, rules, frame_tokens, hist_frames, cur_frames, recent_fra
     a.cu_seqlens_host = cu_host.ctypes.data_as(POINTER(c_int32))
     _check(vkv_compact_cache(a, _stream(stream)), "vkv_compact_cache")
     return k_out, v_out, cu_dev, cu_host
+
+
+def persist_update(q, k, persist_idx, evict_blk0, n_evict, scores=False, err=None, stream=None, out_idx=None,
+                   workspace=None):
+    """Top-C of (persistent blocks + evicted window blocks) by <mean query, block mean>.
+
+    q [B, Lq, H, d], k [B, Lkv, H, d] device bf16; persist_idx device int32 [B*H, C].
+    Returns (new persistent ids [B*H, C] ascending, candidate scores [B*H, C + n_evict] or None).
+    """
+    B, Lq, H, d = q.shape
+    persist_idx = persist_idx.contiguous()
+    C = persist_idx.shape[-1]
+    a = vkv_persist_args()
+    a.B, a.H, a.d, a.block, a.Lq, a.Lkv = B, H, d, 64, Lq, k.shape[1]
+    a.q, a.k = tensor_desc(q), tensor_desc(k)
+    a.persist_idx, a.n_persist = persist_idx.data_ptr(), C
+    a.evict_blk0, a.n_evict = int(evict_blk0), int(n_evict)
+    idx = out_idx if out_idx is not None else torch.empty((B * H, C), dtype=torch.int32, device=q.device)
+    a.out_idx = idx.data_ptr()
+    sc = None
+    if scores:
+        sc = torch.empty((B * H, C + int(n_evict)), dtype=torch.float32, device=q.device)
+        a.out_scores = sc.data_ptr()
+    need = vkv_persist_update_workspace_size(B, H, Lq, C, int(n_evict), 64, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.err_word = err.data_ptr() if err is not None else None
+    _check(vkv_persist_update(a, _stream(stream)), "vkv_persist_update")
+    return idx, sc

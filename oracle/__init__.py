@@ -26,3 +26,4 @@ from .attention import (  # noqa: F401
     visited_flops_sparse,
 )
 from .compaction import compact_cache, head_frames, merge_frames  # noqa: F401
+from .memory import persist_update  # noqa: F401
