@@ -347,3 +347,50 @@ def make_merge_inputs(seed: int, B: int, Lq: int, H: int, d: int, neg_inf_frac: 
         la[rng.random(la.shape) < neg_inf_frac] = -np.inf
         lb[rng.random(lb.shape) < neg_inf_frac] = -np.inf
     return oa, torch.from_numpy(la), ob, torch.from_numpy(lb)
+
+
+# ---------------------------------------------------------------------------
+# Latent (VideoMLA) cache: one head-shared [c_t ; k^R_t] row per token
+# ---------------------------------------------------------------------------
+@dataclass
+class LatentCase:
+    name: str
+    B: int
+    H: int
+    d_c: int
+    d_rope: int
+    q: torch.Tensor   # [B, Lq, H, d_c + d_rope] bf16, absorbed and rotated queries
+    kv: torch.Tensor  # [B, Lkv, d_c + d_rope] bf16, cached rows [c ; k_R]
+    scale: float
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def Lq(self) -> int:
+        return self.q.shape[1]
+
+    @property
+    def Lkv(self) -> int:
+        return self.kv.shape[1]
+
+
+def make_latent(name: str = "latent", seed: int = 5, B: int = 1, H: int = 12, Lq: int = 4680,
+                Lkv: int = 32760, d_c: int = 192, d_rope: int = 32, d_head: int = 128,
+                q_std: float = 1.0) -> LatentCase:
+    """N(0, q_std^2) queries and N(0, 1) cached rows, both bf16.
+
+    Defaults: the Wan-1.3B shape (12 heads of width 128, 1560 tokens per latent
+    frame) with a 3-frame query chunk over a 21-latent-frame cache, and the
+    default latent budget d_c = 192, d_rope = 32 (VideoMLA technical summary,
+    "Methodology", memory reduction).  Scale 1/sqrt(d_head).
+    """
+    rng = np.random.default_rng(seed)
+    dq = d_c + d_rope
+    q = _bf16(rng.standard_normal((B, Lq, H, dq), dtype=np.float32) * np.float32(q_std))
+    kv = _bf16(rng.standard_normal((B, Lkv, dq), dtype=np.float32))
+    return LatentCase(name, B, H, d_c, d_rope, q, kv, 1.0 / float(np.sqrt(d_head)),
+                      dict(seed=seed, q_std=q_std))
+
+
+def cfg_latent() -> LatentCase:
+    """VideoMLA-shaped chunk on Wan-1.3B: H=12, Q 3 frames (4680), cache 21 frames (32 760)."""
+    return make_latent()

@@ -27,3 +27,4 @@ from .attention import (  # noqa: F401
 )
 from .compaction import compact_cache, head_frames, merge_frames  # noqa: F401
 from .memory import persist_update  # noqa: F401
+from .mla import latent_attention, visited_flops_latent  # noqa: F401
