@@ -369,6 +369,37 @@ vkv_status vkv_lse_merge(vkv_tensor o_a, const float* lse_a, vkv_tensor o_b, con
                          vkv_tensor o_out, float* lse_out, int32_t B, int32_t H, int32_t Lq,
                          int32_t d, vkv_stream_t stream);
 
+/*
+ * vkv_latent_attn -- latent (multi-head latent) attention over a head-shared
+ * cache (VideoMLA technical summary, "Methodology": each cached token keeps one
+ * content latent c_t of width d_c and one rotary key k^R_t of width d_rope,
+ * shared by all heads; each head rebuilds its keys and values from them with
+ * its own up-projections).  With the key up-projection absorbed into the query
+ * (qa_h = [(W^K_h)^T q^nope_h ; q^R_h]) and the value up-projection left to
+ * the output projection, for each (batch b, head h, query row i):
+ *   s_t = scale * <qa_{b,i,h}, [c_{b,t} ; k^R_{b,t}]>,
+ *   o_{b,i,h} = sum_t softmax(s)_t c_{b,t}     (latent output, width d_c),
+ *   LSE_{b,h,i} = ln sum_t exp(s_t).
+ * Every head reads the same cache rows.  No position math happens here: q and
+ * k^R arrive rotated.  An empty cache (Lkv = 0) gives o = 0 and LSE = -inf.
+ */
+typedef struct {
+  int32_t B, H, Lq, Lkv; /* B, H, Lq >= 1; Lkv >= 0                                 */
+  int32_t d_c;     /* latent width: 128 or 192                                     */
+  int32_t d_rope;  /* rotary key width: 32                                         */
+  float scale;     /* softmax scale, > 0                                           */
+  vkv_tensor q;    /* [B, Lq, H, d_c + d_rope]: absorbed, rotated queries          */
+  vkv_tensor kv;   /* [B, Lkv, d_c (+ d_rope)]: cached rows [c ; k^R]; sb, st read, sh ignored;
+                      may be NULL when Lkv = 0                                     */
+  vkv_tensor kr;   /* optional [B, Lkv, d_rope] rotary keys stored apart (sb, st read);
+                      ptr NULL = columns [d_c, d_c + d_rope) of kv                */
+  vkv_tensor o;    /* [B, Lq, H, d_c] bf16 latent output                           */
+  float* lse;      /* optional fp32 [B, H, Lq] contiguous (NULL = skip)            */
+  int32_t* err_word; /* optional DEVICE int32; a pipeline timeout sets VKV_DEVERR_TIMEOUT */
+} vkv_latent_args;
+
+vkv_status vkv_latent_attn(const vkv_latent_args* args, vkv_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* vkv_status_string(vkv_status s);
 
@@ -377,7 +408,8 @@ int32_t vkv_version(void);
 
 /* sizeof() of the ABI structs, for bindings to check their layout:
  * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment,
- * 4 vkv_compact_args, 5 vkv_head_rule, 6 vkv_persist_args; -1 otherwise. */
+ * 4 vkv_compact_args, 5 vkv_head_rule, 6 vkv_persist_args, 7 vkv_latent_args;
+ * -1 otherwise. */
 int32_t vkv_abi_sizeof(int32_t which);
 
 #ifdef __cplusplus

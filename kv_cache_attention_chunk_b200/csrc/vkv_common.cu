@@ -54,15 +54,17 @@ int device_sm_count(int* dev_out) {
 }
 
 bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
-                         const uint64_t strides_bytes[3], const uint32_t box[4]) {
+                         const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes) {
   std::call_once(g_encode_once, init_encode);
   if (!g_encode) return false;
   cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
   cuuint32_t bd[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t es[4] = {1, 1, 1, 1};
+  if (swizzle_bytes != 128 && swizzle_bytes != 64) return false;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bd, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -99,6 +101,7 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
     case 4: return (int32_t)sizeof(vkv_compact_args);
     case 5: return (int32_t)sizeof(vkv_head_rule);
     case 6: return (int32_t)sizeof(vkv_persist_args);
+    case 7: return (int32_t)sizeof(vkv_latent_args);
   }
   return -1;
 }

@@ -6,9 +6,11 @@ on a non-OK status.  There is no fallback: if libvkv.so is missing or no
 sm_100 device is present the calls raise.
 
 Raw entry points with the C names: ``vkv_chunk_attn``, ``vkv_block_select``,
-``vkv_block_select_workspace_size``, ``vkv_lse_merge``, ``vkv_status_string``.
+``vkv_block_select_workspace_size``, ``vkv_lse_merge``, ``vkv_latent_attn``,
+``vkv_status_string`` (and the other entry points of the header).
 Convenience wrappers that allocate outputs with torch: ``chunk_attn_segments``,
-``chunk_attn_block_sparse``, ``chunk_attn_ragged``, ``block_select``, ``lse_merge``.
+``chunk_attn_block_sparse``, ``chunk_attn_ragged``, ``block_select``, ``lse_merge``,
+``latent_attn`` and the others below.
 """
 from __future__ import annotations
 
@@ -106,6 +108,14 @@ class vkv_persist_args(ctypes.Structure):
         ("err_word", c_void_p),
     ]
 
+class vkv_latent_args(ctypes.Structure):
+    _fields_ = [
+        ("B", c_int32), ("H", c_int32), ("Lq", c_int32), ("Lkv", c_int32),
+        ("d_c", c_int32), ("d_rope", c_int32), ("scale", c_float),
+        ("q", vkv_tensor), ("kv", vkv_tensor), ("kr", vkv_tensor), ("o", vkv_tensor),
+        ("lse", c_void_p), ("err_word", c_void_p),
+    ]
+
 _lib = None
 
 
@@ -146,8 +156,10 @@ def lib() -> ctypes.CDLL:
     L.vkv_persist_update_workspace_size.restype = c_size_t
     L.vkv_persist_update.argtypes = [POINTER(vkv_persist_args), c_void_p]
     L.vkv_persist_update.restype = c_int32
+    L.vkv_latent_attn.argtypes = [POINTER(vkv_latent_args), c_void_p]
+    L.vkv_latent_attn.restype = c_int32
     for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
-                            vkv_head_rule, vkv_persist_args)):
+                            vkv_head_rule, vkv_persist_args, vkv_latent_args)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
             raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
                                f"binding {ctypes.sizeof(st)} B")
@@ -185,6 +197,10 @@ def vkv_persist_update_workspace_size(B, H, Lq, n_persist, n_evict, block, d) ->
 
 def vkv_persist_update(args: vkv_persist_args, stream: int | None) -> int:
     return int(lib().vkv_persist_update(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_latent_attn(args: vkv_latent_args, stream: int | None) -> int:
+    return int(lib().vkv_latent_attn(ctypes.byref(args), c_void_p(stream or 0)))
 
 
 def vkv_compact_rows(args: vkv_compact_args) -> int:
@@ -453,3 +469,39 @@ def persist_update(q, k, persist_idx, evict_blk0, n_evict, scores=False, err=Non
     a.err_word = err.data_ptr() if err is not None else None
     _check(vkv_persist_update(a, _stream(stream)), "vkv_persist_update")
     return idx, sc
+
+
+def latent_desc(x: torch.Tensor) -> vkv_tensor:
+    """[B, L, w] bf16 cache rows with contiguous w -> vkv_tensor (sh unused)."""
+    if x.dim() != 3 or x.dtype != torch.bfloat16 or x.stride(2) != 1:
+        raise ValueError("expected a bf16 [B, L, w] tensor with contiguous w")
+    return vkv_tensor(x.data_ptr(), x.stride(0), x.stride(1), 0)
+
+
+def latent_attn(q, kv, d_c, scale=None, kr=None, err=None, stream=None, out=None, lse=True):
+    """Latent attention over a head-shared cache (vkv_latent_attn).
+
+    q [B, Lq, H, d_c + d_rope] absorbed queries; kv [B, Lkv, d_c (+ d_rope)] cached rows
+    [c ; k_R]; kr optional [B, Lkv, d_rope] when the rotary keys are stored apart.
+    Returns (latent output [B, Lq, H, d_c] bf16, LSE [B, H, Lq] fp32 or None).
+    """
+    B, Lq, H, dq = q.shape
+    d_rope = dq - d_c
+    a = vkv_latent_args()
+    a.B, a.H, a.Lq, a.Lkv, a.d_c, a.d_rope = B, H, Lq, kv.shape[1], d_c, d_rope
+    a.scale = float(scale if scale is not None else 1.0 / np.sqrt(dq))
+    a.q = tensor_desc(q)
+    if kv.shape[1] > 0:  # an empty cache is passed as a NULL pointer
+        a.kv = latent_desc(kv)
+        if kr is not None:
+            a.kr = latent_desc(kr)
+    if out is None:
+        o = torch.empty((B, Lq, H, d_c), dtype=torch.bfloat16, device=q.device)
+        l = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device) if lse else None
+    else:
+        o, l = out
+    a.o = tensor_desc(o)
+    a.lse = l.data_ptr() if l is not None else None
+    a.err_word = err.data_ptr() if err is not None else None
+    _check(vkv_latent_attn(a, _stream(stream)), "vkv_latent_attn")
+    return o, l

@@ -247,3 +247,35 @@ def test_compact_cache_rejects_small_output_without_a_gpu():
     a.k_out, a.v_out, a.cu_seqlens = 64, 64, 64
     a.out_rows = 79
     assert vkv.vkv_compact_cache(a, None) == 4  # VKV_ERR_RANGE: checked before any device work
+
+
+def latent_args(**kw):
+    a = vkv.vkv_latent_args()
+    a.B, a.H, a.Lq, a.Lkv, a.d_c, a.d_rope, a.scale = 1, 12, 4680, 32760, 192, 32, 0.088
+    a.q = T(sb=4680 * 12 * 224, st=12 * 224, sh=224)
+    a.kv = T(sb=32760 * 224, st=224, sh=0)
+    a.o = T(sb=4680 * 12 * 192, st=12 * 192, sh=192)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d_c", 64, 5), ("d_c", 256, 5), ("d_rope", 64, 5), ("d_rope", 0, 5),
+    ("B", 0, 2), ("H", 0, 2), ("Lq", 0, 2), ("Lkv", -1, 2), ("scale", 0.0, 2), ("scale", float("inf"), 2),
+])
+def test_latent_bad_sizes(field, value, status):
+    assert vkv.vkv_latent_attn(latent_args(**{field: value}), None) == status
+
+
+def test_latent_null_and_alignment():
+    assert vkv.lib().vkv_latent_attn(None, None) == 1
+    assert vkv.vkv_latent_attn(latent_args(q=T(ptr=0)), None) == 1
+    assert vkv.vkv_latent_attn(latent_args(kv=T(ptr=0, st=224)), None) == 1
+    assert vkv.vkv_latent_attn(latent_args(q=T(ptr=FAKE + 2, sb=4680 * 12 * 224, st=12 * 224, sh=224)), None) == 3
+    assert vkv.vkv_latent_attn(latent_args(kv=T(st=228, sb=32760 * 228)), None) == 3
+    assert vkv.vkv_latent_attn(latent_args(kr=T(ptr=FAKE + 4, st=32, sb=32760 * 32)), None) == 3
+    # an empty cache needs no cache pointer
+    if not torch.cuda.is_available():
+        assert vkv.vkv_latent_attn(latent_args(Lkv=0, kv=T(ptr=0)), None) == 6
+        assert vkv.vkv_latent_attn(latent_args(), None) == 6
