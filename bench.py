@@ -403,6 +403,20 @@ def extras(dev, peaks):
                                  20, st))
     fl = oracle.visited_flops_ragged(1, 12, c.Lq, 128, c.cu_seqlens)
     out["ragged"] = {"ms": ms, "tflops": fl / ms / 1e9}
+    del q, k, v, o
+    # latent (VideoMLA) attention: the Wan-1.3B 3-frame chunk over a 21-frame head-shared cache
+    lat = {}
+    for d_c in (192, 128):
+        c = W.make_latent(d_c=d_c)
+        q, kv = c.q.to(dev), c.kv.to(dev)
+        o = vkv.latent_attn(q, kv, d_c, scale=c.scale)
+        ms = statistics.median(timed(lambda: vkv.latent_attn(q, kv, d_c, scale=c.scale, out=o), 20, st, flush))
+        fl = oracle.visited_flops_latent(c.B, c.H, c.Lq, c.Lkv, d_c, c.d_rope)
+        lat[f"d_c{d_c}"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_bf16": fl / ms / 1e9 / peaks["bf16_tflops"],
+                            "cache_bytes_per_layer": kv.numel() * 2,
+                            "dense_cache_bytes_per_layer": 2 * c.H * 128 * c.Lkv * 2}
+        del q, kv, o
+    out["latent_wan13b"] = lat
     return out
 
 
@@ -555,6 +569,11 @@ def run_profile(args):
         cu = torch.from_numpy(c.cu_seqlens).to(dev)
         o = vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale)
         fn = lambda: vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale, out=o)  # noqa: E731
+    elif args.profile == "latent":
+        c = W.cfg_latent()
+        q, kv = c.q.to(dev), c.kv.to(dev)
+        o = vkv.latent_attn(q, kv, c.d_c, scale=c.scale)
+        fn = lambda: vkv.latent_attn(q, kv, c.d_c, scale=c.scale, out=o)  # noqa: E731
     else:
         raise SystemExit(f"unknown profile case {args.profile}")
     for _ in range(args.warmup):
@@ -569,7 +588,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
                     help="run one small case for an ncu capture: wan13b, wan14b, merge, select, sparse9, "
-                         "sparse144, ragged")
+                         "sparse144, ragged, latent")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)

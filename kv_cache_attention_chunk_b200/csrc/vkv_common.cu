@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "vkv_internal.h"
+#include "vkv_tmap.h"
 
 namespace vkv {
 
@@ -54,7 +55,12 @@ int device_sm_count(int* dev_out) {
 }
 
 bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
-                         const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes) {
+                         const uint64_t strides_bytes[3], const uint32_t box[4]) {
+  return encode_tmap_bf16_4d_swizzle(tm, ptr, dims, strides_bytes, box, 128);
+}
+
+bool encode_tmap_bf16_4d_swizzle(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
+                                 const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes) {
   std::call_once(g_encode_once, init_encode);
   if (!g_encode) return false;
   cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};

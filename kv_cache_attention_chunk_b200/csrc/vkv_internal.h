@@ -56,9 +56,8 @@ struct AttnParams {
 
 // Host helpers (vkv_common.cu).
 int device_sm_count(int* dev_out);                // -1 when no usable sm_100 device
-// swizzle_bytes: 128 (box rows of 128 B) or 64 (box rows of 64 B).
 bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
-                         const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes = 128);
+                         const uint64_t strides_bytes[3], const uint32_t box[4]);
 bool tensor_aligned(const vkv_tensor& t);
 
 }  // namespace vkv

@@ -41,6 +41,7 @@
 //          the next tile's first PV (which overwrites O) waits o_free.
 #include "vkv_internal.h"
 #include "vkv_ptx.cuh"
+#include "vkv_tmap.h"
 
 #include <algorithm>
 #include <cmath>
@@ -90,6 +91,18 @@ struct LatParams {
   int B, H, Lq, Lkv, n_qt, n_tiles;
   float scale_log2;
 };
+
+// Shared-memory matrix descriptor of a K-major operand with 64-byte swizzle
+// (sm_100 layout code 4): rows of 64 B (32 bf16 along K), 8-row groups 512 B
+// apart; the two 16-element K slices of a row start at +0 and +32 B.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused by this layout): 16 B
+  d |= (uint64_t)(512 >> 4) << 32;   // stride byte offset: 8-row group pitch
+  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+  d |= (uint64_t)4 << 61;            // swizzle: 64 B
+  return d;
+}
 
 constexpr float kLn2f = 0.6931471805599453f;
 
@@ -442,7 +455,7 @@ bool encode_lat(CUtensorMap* tm, const void* ptr, long long sb, long long st, lo
   const uint64_t bsb = (B == 1) ? bst * (uint64_t)L : (uint64_t)sb * 2;
   const uint64_t strides[3] = {bsh, bst, bsb};
   const uint32_t box[4] = {(uint32_t)box_w, 1, 128, 1};
-  return encode_tmap_bf16_4d(tm, ptr, dims, strides, box, swz);
+  return encode_tmap_bf16_4d_swizzle(tm, ptr, dims, strides, box, swz);
 }
 
 template <int DC>

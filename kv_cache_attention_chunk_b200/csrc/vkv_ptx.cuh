@@ -229,17 +229,6 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// K-major operand with 64-byte swizzle: rows of 64 B (32 bf16 along K), 8-row
-// groups 512 B apart; the 32-byte K slices of one row are at +0 and +32.
-__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1 << 16;              // leading byte offset (unused by this layout): 16 B
-  d |= (uint64_t)(512 >> 4) << 32;     // stride byte offset: 8-row group pitch
-  d |= (uint64_t)1 << 46;              // descriptor version for sm_100
-  d |= (uint64_t)4 << 61;              // swizzle: 64 B
-  return d;
-}
-
 // MN-major operand: each K index is a 128 B row holding 64 consecutive MN
 // elements; 8-row K groups are 1024 B apart; 64-wide MN chunks `mn_chunk_bytes` apart.
 __device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t mn_chunk_bytes) {
