@@ -104,6 +104,33 @@ __device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
   return d;
 }
 
+// Part of the exponentials can run on the FMA pipe instead of MUFU (one MUFU
+// ex2 per score and one softmax warp per SM sub-partition make MUFU the
+// longest part of a step): kLatExpEmu of every 16 columns.  2^x = 2^r q(f),
+// r = round(x) by the 1.5 * 2^23 trick, f = x - r in [-1/2, 1/2], q a cubic
+// fitted to 2^f by relative-error minimax (max relative error 7.5e-5, far below
+// the 2^-9 rounding of P to bf16); 2^r enters the exponent field as an integer
+// add.  Arguments below -126 give at most 2^-126 (masked scores are -inf).
+#ifndef VKV_LAT_EXP_EMU
+#define VKV_LAT_EXP_EMU 0
+#endif
+constexpr int kLatExpEmu = VKV_LAT_EXP_EMU;
+
+__device__ __forceinline__ void lat_exp2_pair(float x0, float x1, float& e0, float& e1) {
+  const uint64_t xc = pack2f(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = pack2f(12582912.f, 12582912.f);
+  const uint64_t t = add2f(xc, magic);
+  const uint64_t f = sub2f(xc, sub2f(t, magic));
+  uint64_t q = fma2f(pack2f(0.0551716685f, 0.0551716685f), f, pack2f(0.242611140f, 0.242611140f));
+  q = fma2f(q, f, pack2f(0.693260968f, 0.693260968f));
+  q = fma2f(q, f, pack2f(0.999928057f, 0.999928057f));
+  float q0, q1, t0, t1;
+  unpack2f(q, q0, q1);
+  unpack2f(t, t0, t1);
+  e0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(q0));
+  e1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(q1));
+}
+
 constexpr float kLn2f = 0.6931471805599453f;
 
 __device__ __forceinline__ bool lat_all(bool v) { return __all_sync(0xFFFFFFFFu, v); }
@@ -375,7 +402,14 @@ __global__ void __launch_bounds__(256, 1) latent_attn_kernel(const __grid_consta
               unpack2f(fma2f(pack2f(__uint_as_float(sr[c0 + i]), __uint_as_float(sr[c0 + i + 1])), sl2x2, nmu2),
                        a[i], a[i + 1]);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) e[i] = ex2_approx(a[i]);
+            for (int i = 0; i < 16; i += 2) {
+              if (i >= 16 - kLatExpEmu) {
+                lat_exp2_pair(a[i], a[i + 1], e[i], e[i + 1]);
+              } else {
+                e[i] = ex2_approx(a[i]);
+                e[i + 1] = ex2_approx(a[i + 1]);
+              }
+            }
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
               acc2[(i >> 1) & 3] = add2f(acc2[(i >> 1) & 3], pack2f(e[i], e[i + 1]));
