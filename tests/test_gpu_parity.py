@@ -138,6 +138,21 @@ def test_full_size_dense_configs_sampled(cfg):
     assert np.isfinite(to_np(res["o_merged"])).all()
 
 
+@pytest.mark.parametrize("H,q_tokens", [(160, 300), (300, 100)])
+def test_many_heads_odd_tile_count(H, q_tokens):
+    """Many heads with an odd number of query tiles (one-tile units beside pairs,
+    more units than SMs): every output of every head matches the oracle."""
+    c = W.make_dual_branch("m", 90 + H, H=H, d=128, frame_tokens=100, q_frames=3, hist_frames=2,
+                           q_tokens=q_tokens)
+    res = run_segments(c)
+    ref = oracle.segment_attention(c.q, c.k, c.v, c.branches, c.scale)
+    for i in range(2):
+        assert_bf16_close(res["o"][i], ref["branch_o"][i], f"H{H} O{i}")
+        assert_lse_close(res["lse"][i], ref["branch_lse"][i], f"H{H} LSE{i}")
+    assert_bf16_close(res["o_merged"], ref["dense_o"], f"H{H} merged")
+    assert_lse_close(res["lse_merged"], ref["dense_lse"], f"H{H} merged LSE")
+
+
 # ---------------------------------------------------------------------------
 # standalone LSE merge
 # ---------------------------------------------------------------------------
