@@ -112,13 +112,21 @@ ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx
 
 
 def kernel_source_hash() -> str:
-    """Hash of the attention kernel's sources (ties recorded ncu counters to a kernel version)."""
+    """Hash of the attention kernel's code (ties recorded ncu counters to a kernel version).
+
+    Comments and whitespace are left out, so an edit of the prose alone keeps the record.
+    """
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_attention_chunk_b200", "csrc")
     for name in ATTN_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as fh:
-            h.update(name.encode() + fh.read())
+        with open(os.path.join(csrc, name)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        src = " ".join(src.split())
+        h.update(name.encode() + src.encode())
     return h.hexdigest()[:16]
 
 

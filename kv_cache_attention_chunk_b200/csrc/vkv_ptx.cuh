@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers, TMA tensor loads (no multicast), tcgen05 MMA / tensor memory,
+// mbarriers, TMA tensor loads into this CTA only, tcgen05 MMA / tensor memory,
 // and a few special registers.  Every wait on an mbarrier is bounded in time.
 #pragma once
 
@@ -131,7 +131,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ----------------------------------------------------------------------------
-// TMA (tensor memory accelerator) tiled loads, no multicast
+// TMA (tensor memory accelerator) tiled loads, each into this CTA's shared memory only
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
@@ -146,7 +146,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
-// Untiled bulk copy global -> shared (no multicast), completion counted in
+// Untiled bulk copy global -> this CTA's shared memory, completion counted in
 // bytes on `bar`; both addresses 16-byte aligned, `bytes` a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
