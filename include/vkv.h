@@ -400,6 +400,17 @@ typedef struct {
 
 vkv_status vkv_latent_attn(const vkv_latent_args* args, vkv_stream_t stream);
 
+/*
+ * vkv_debug_withhold_copy -- test aid for the bounded pipeline waits.  The next
+ * n_calls launches of vkv_chunk_attn or vkv_latent_attn (in any thread) run with
+ * the first cache-tile copy of every CTA withheld: the wait for it runs out
+ * after its time limit (1 s), the kernel stops its work, lets the copies it did
+ * issue land, releases its resources and writes VKV_DEVERR_TIMEOUT to err_word;
+ * the outputs of that launch are incomplete and the device stays usable.
+ * n_calls = 0 disarms it.  Returns VKV_ERR_SHAPE for n_calls < 0.
+ */
+vkv_status vkv_debug_withhold_copy(int32_t n_calls);
+
 /* Human-readable name of a status code (static storage). */
 const char* vkv_status_string(vkv_status s);
 

@@ -227,6 +227,7 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   P->d = d;
   P->scale_log2 = a->scale * 1.4426950408889634f;
   P->err = a->err_word;
+  P->withhold_first_copy = take_withhold_request() ? 1 : 0;
 
   int nb = 1;
   std::vector<double> pc(n_seq), oc(n_seq);

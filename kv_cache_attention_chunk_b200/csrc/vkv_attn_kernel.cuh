@@ -520,6 +520,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               const uint32_t slot = item % C::NSLOT, use = item / C::NSLOT;
               if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
               if (!ok) break;
+              if (item == 0 && p.withhold_first_copy) {
+                ++item;  // test aid: this copy never arrives, so the wait for it runs out
+                continue;
+              }
               VKV_STAMP(20480 + (int)item);
               mbar_arrive_expect_tx(b_full0 + 8 * slot, (uint32_t)C::KV_BYTES);
               const CUtensorMap* tm = kv ? &p.tm_v : &p.tm_k;

@@ -3,6 +3,7 @@
 // without a GPU driver), status strings.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "vkv_internal.h"
@@ -75,6 +76,18 @@ bool encode_tmap_bf16_4d_swizzle(CUtensorMap* tm, const void* ptr, const uint64_
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+std::atomic<int> g_withhold{0};
+}  // namespace
+
+bool take_withhold_request() {
+  int n = g_withhold.load();
+  while (n > 0) {
+    if (g_withhold.compare_exchange_weak(n, n - 1)) return true;
+  }
+  return false;
+}
+
 bool tensor_aligned(const vkv_tensor& t) {
   return (reinterpret_cast<uintptr_t>(t.ptr) & 15u) == 0 && (t.sb % 8) == 0 && (t.st % 8) == 0 &&
          (t.sh % 8) == 0;
@@ -110,4 +123,10 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
     case 7: return (int32_t)sizeof(vkv_latent_args);
   }
   return -1;
+}
+
+extern "C" vkv_status vkv_debug_withhold_copy(int32_t n_calls) {
+  if (n_calls < 0) return VKV_ERR_SHAPE;
+  vkv::g_withhold.store(n_calls);
+  return VKV_OK;
 }

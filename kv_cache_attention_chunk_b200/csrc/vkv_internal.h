@@ -48,6 +48,7 @@ struct AttnParams {
   long long om_sb, om_st, om_sh;
   float* lsem;
   int* err;
+  int withhold_first_copy;  // test aid: the producer skips its first K/V copy (see vkv_debug_withhold_copy)
   // schedule: CTA c runs units[cta_begin[c] .. cta_begin[c+1])
   int n_ctas;
   int cta_begin[kMaxCtas + 1];
@@ -59,5 +60,8 @@ int device_sm_count(int* dev_out);                // -1 when no usable sm_100 de
 bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
                          const uint64_t strides_bytes[3], const uint32_t box[4]);
 bool tensor_aligned(const vkv_tensor& t);
+// Test aid (vkv_common.cu): true when the calling launch should withhold its first
+// cache-tile copy (consumes one of the calls armed by vkv_debug_withhold_copy).
+bool take_withhold_request();
 
 }  // namespace vkv

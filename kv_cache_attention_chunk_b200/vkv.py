@@ -158,6 +158,8 @@ def lib() -> ctypes.CDLL:
     L.vkv_persist_update.restype = c_int32
     L.vkv_latent_attn.argtypes = [POINTER(vkv_latent_args), c_void_p]
     L.vkv_latent_attn.restype = c_int32
+    L.vkv_debug_withhold_copy.argtypes = [c_int32]
+    L.vkv_debug_withhold_copy.restype = c_int32
     for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
                             vkv_head_rule, vkv_persist_args, vkv_latent_args)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
@@ -201,6 +203,11 @@ def vkv_persist_update(args: vkv_persist_args, stream: int | None) -> int:
 
 def vkv_latent_attn(args: vkv_latent_args, stream: int | None) -> int:
     return int(lib().vkv_latent_attn(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_debug_withhold_copy(n_calls: int) -> int:
+    """Test aid: the next n_calls attention launches withhold their first cache-tile copy."""
+    return int(lib().vkv_debug_withhold_copy(int(n_calls)))
 
 
 def vkv_compact_rows(args: vkv_compact_args) -> int:

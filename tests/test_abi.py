@@ -279,3 +279,9 @@ def test_latent_null_and_alignment():
     if not torch.cuda.is_available():
         assert vkv.vkv_latent_attn(latent_args(Lkv=0, kv=T(ptr=0)), None) == 6
         assert vkv.vkv_latent_attn(latent_args(), None) == 6
+
+
+def test_withhold_copy_arming():
+    assert vkv.vkv_debug_withhold_copy(-1) == 2
+    assert vkv.vkv_debug_withhold_copy(1) == 0
+    assert vkv.vkv_debug_withhold_copy(0) == 0

@@ -139,3 +139,20 @@ def test_full_size_sampled():
     assert_bf16_close(to_np(o)[:, rows], o_ref[:, rows], "full size")
     assert_lse_close(to_np(lse)[:, :, rows], l_ref[:, :, rows], "full size lse")
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+def test_stalled_pipeline_reports_timeout_and_device_stays_usable():
+    """A withheld cache-tile copy makes the bounded wait run out: VKV_DEVERR_TIMEOUT,
+    then a normal call on the same context matches the oracle."""
+    v = vk()
+    case = W.make_latent("t", seed=8, B=1, H=2, Lq=200, Lkv=400)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert v.vkv_debug_withhold_copy(1) == 0
+    try:
+        v.latent_attn(case.q.to(DEV), case.kv.to(DEV), case.d_c, scale=case.scale, err=err)
+        torch.cuda.synchronize()
+    finally:
+        v.vkv_debug_withhold_copy(0)
+    assert int(err.item()) == v.DEVERR_TIMEOUT
+    o, lse = _run(case)
+    _check_full(case, o, lse, "after a timeout")

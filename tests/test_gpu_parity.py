@@ -153,6 +153,24 @@ def test_many_heads_odd_tile_count(H, q_tokens):
     assert_lse_close(res["lse_merged"], ref["dense_lse"], f"H{H} merged LSE")
 
 
+def test_stalled_pipeline_reports_timeout_and_device_stays_usable():
+    """A cache-tile copy that never arrives (withheld on purpose): the bounded wait
+    for it runs out, the call reports VKV_DEVERR_TIMEOUT and the next call on the
+    same context is correct."""
+    v = vk()
+    c = W.cfg_tiny()
+    q, k, vv = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    err = err_word()
+    assert v.vkv_debug_withhold_copy(1) == 0
+    try:
+        v.chunk_attn_segments(q, k, vv, c.branches, scale=c.scale, err=err)
+        torch.cuda.synchronize()
+    finally:
+        v.vkv_debug_withhold_copy(0)
+    assert int(err.item()) == v.DEVERR_TIMEOUT
+    check_segments_full(c, run_segments(c))
+
+
 # ---------------------------------------------------------------------------
 # standalone LSE merge
 # ---------------------------------------------------------------------------
