@@ -105,6 +105,12 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
   };
   std::vector<long long> cands = {0};
   for (int k = 1; k <= 32; ++k) cands.push_back((long long)k * n_sm / 8);
+  // and the splits that leave exactly k * n_sm units (k units per SM when the costs are equal)
+  const long long n_odd = (T & 1) ? n_seq : 0;
+  for (int k = 1; k <= 16; ++k) {
+    const long long c = (long long)k * n_sm - n_pairs - n_odd;
+    if (c > 0 && c < n_pairs) cands.push_back(c);
+  }
   cands.push_back(n_pairs);
   double best = 1e300;
   long long best_split = 0;
