@@ -151,14 +151,17 @@ std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T,
   return plan;
 }
 
-bool set_smem_attr(int dev, int D) {
+bool set_smem_attr(int dev, int D, bool sparse) {
   static std::mutex mu;
-  static unsigned long long done[2] = {0, 0};
+  static unsigned long long done[4] = {0, 0, 0, 0};
   std::lock_guard<std::mutex> lk(mu);
-  const int k = (D == 128) ? 0 : 1;
+  const int k = ((D == 128) ? 0 : 1) + (sparse ? 2 : 0);
   if (done[k] & (1ull << dev)) return true;
-  const void* fn = (D == 128) ? reinterpret_cast<const void*>(chunk_attn_kernel<128>)
-                              : reinterpret_cast<const void*>(chunk_attn_kernel<64>);
+  const void* fn =
+      (D == 128) ? (sparse ? reinterpret_cast<const void*>(chunk_attn_kernel<128, true>)
+                           : reinterpret_cast<const void*>(chunk_attn_kernel<128, false>))
+                 : (sparse ? reinterpret_cast<const void*>(chunk_attn_kernel<64, true>)
+                           : reinterpret_cast<const void*>(chunk_attn_kernel<64, false>));
   const int smem = (D == 128) ? AttnCfg<128>::SMEM_BYTES : AttnCfg<64>::SMEM_BYTES;
   cudaFuncAttributes fa;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
@@ -369,12 +372,20 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     if (!encode_bhld(&P->tm_k, a->k, B, Lkv, H, d, 64) || !encode_bhld(&P->tm_v, a->v, B, Lkv, H, d, 64))
       return VKV_ERR_CUDA;
   }
-  if (!set_smem_attr(dev, d)) return VKV_ERR_CUDA;
+  const bool sp = mode == VKV_MODE_BLOCK_SPARSE;
+  if (!set_smem_attr(dev, d, sp)) return VKV_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 128)
-    chunk_attn_kernel<128><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
-  else
-    chunk_attn_kernel<64><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
+  if (d == 128) {
+    if (sp)
+      chunk_attn_kernel<128, true><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
+    else
+      chunk_attn_kernel<128, false><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
+  } else {
+    if (sp)
+      chunk_attn_kernel<64, true><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
+    else
+      chunk_attn_kernel<64, false><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
+  }
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   return VKV_OK;
 }

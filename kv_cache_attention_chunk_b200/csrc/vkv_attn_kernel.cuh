@@ -66,13 +66,12 @@ struct Ctl {
   uint64_t empty[kMaxSlots];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t list_ready, list_free, drain;
+  uint64_t list_ready[2], list_free[2], drain;  // one pair per block-list buffer
   uint32_t tmem_base;
   int abort_flag;
-  int list_count;
-  int pad_;
+  int list_count[2];
   uint32_t bitmap[4][32];
-  uint32_t list[kMaxListEntries];
+  uint32_t list[kMaxListEntries];  // block-list buffer 0 (buffer 1: the ring's last K/V slot)
 };
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
 
@@ -87,14 +86,16 @@ struct TileDesc {
 // Walks the key-tile stream of one unit; every role runs its own copy.
 struct TileIter {
   const AttnParams* p;
-  const Ctl* ctl;
+  const uint32_t* list;  // BLOCK_SPARSE: the unit's block list and its length
+  int count;
   int k, off;        // SEGMENTS: flat segment index, row offset inside it
   int rstart, rlen;  // RAGGED: this sequence's rows
   int j;
 
-  __device__ __forceinline__ void init(const AttnParams* pp, const Ctl* c, int rs, int rl) {
+  __device__ __forceinline__ void init(const AttnParams* pp, const uint32_t* lst, int cnt, int rs, int rl) {
     p = pp;
-    ctl = c;
+    list = lst;
+    count = cnt;
     k = 0;
     off = 0;
     rstart = rs;
@@ -105,9 +106,9 @@ struct TileIter {
   __device__ __forceinline__ TileDesc next() {
     TileDesc t;
     if (p->mode == VKV_MODE_BLOCK_SPARSE) {
-      const int n = ctl->list_count;
-      const uint32_t e0 = ctl->list[2 * j];
-      const uint32_t e1 = (2 * j + 1 < n) ? ctl->list[2 * j + 1] : (e0 & 0xFFFFFFu);
+      const int n = count;
+      const uint32_t e0 = list[2 * j];
+      const uint32_t e1 = (2 * j + 1 < n) ? list[2 * j + 1] : (e0 & 0xFFFFFFu);
       t.rowA = (int)(e0 & 0xFFFFFFu) * 64;
       t.rowB = (int)(e1 & 0xFFFFFFu) * 64;
       t.limA = 64;
@@ -200,17 +201,18 @@ __device__ __forceinline__ void ragged_range(const AttnParams& p, int s, int& st
   }
 }
 
-__device__ __forceinline__ int unit_steps(const AttnParams& p, const Ctl* ctl, int rlen) {
+__device__ __forceinline__ int unit_steps(const AttnParams& p, int list_count, int rlen) {
   if (p.mode == VKV_MODE_SEGMENTS) return p.total_steps;
   if (p.mode == VKV_MODE_RAGGED) return (rlen + 127) >> 7;
-  return (ctl->list_count + 1) >> 1;
+  return (list_count + 1) >> 1;
 }
 
 // Build the unit's block list (BLOCK_SPARSE): persistent blocks (visible to
 // every query block of the unit) followed by the union of the window blocks
 // selected by the unit's query blocks, ascending, each tagged with the query
 // blocks that selected it.  Executed by all 32 lanes of one warp.
-__device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, const UnitInfo& u) {
+__device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, const UnitInfo& u,
+                                                 uint32_t* list, int* list_count) {
   const uint32_t lane = lane_id();
   const int qb0 = u.tile0 * 2;
   const int nqb = min(2 * u.ntiles, p.n_qblk - qb0);
@@ -245,7 +247,7 @@ __device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, 
       if (!ok) set_err(p, VKV_DEVERR_BAD_INDEX);
     }
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, ok);
-    if (ok) ctl->list[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)blk | (all_mask << 24);
+    if (ok) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)blk | (all_mask << 24);
     base += __popc(bal);
   }
   // window union: lane L owns window blocks [32L, 32L + 32)
@@ -271,9 +273,9 @@ __device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, 
     uint32_t qm = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) qm |= ((m[i] >> bit) & 1u) << i;
-    ctl->list[pos++] = (uint32_t)(p.window_blk0 + (int)lane * 32 + bit) | (qm << 24);
+    list[pos++] = (uint32_t)(p.window_blk0 + (int)lane * 32 + bit) | (qm << 24);
   }
-  if (lane == 0) ctl->list_count = base + total;
+  if (lane == 0) *list_count = base + total;
   __threadfence_block();
   __syncwarp();
 }
@@ -401,9 +403,13 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xFFFFFFFFu, v); }
 
-template <int D>
+// SP: the block-sparse instantiation.  It keeps two block lists, so the next
+// unit's list and its first copies are ready before the current unit ends; the
+// second list lives in the last K/V slot, which its ring then leaves out.
+template <int D, bool SP>
 __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constant__ AttnParams p) {
   using C = AttnCfg<D>;
+  constexpr uint32_t NS = SP ? (uint32_t)C::NSLOT - 1u : (uint32_t)C::NSLOT;  // ring slots
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -421,8 +427,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   const uint32_t b_sfull0 = smem_u32(&ctl->s_full[0]);
   const uint32_t b_pfull0 = smem_u32(&ctl->p_full[0]);
   const uint32_t b_odone0 = smem_u32(&ctl->o_done[0]);
-  const uint32_t b_lready = smem_u32(&ctl->list_ready);
-  const uint32_t b_lfree = smem_u32(&ctl->list_free);
+  const uint32_t b_lready0 = smem_u32(&ctl->list_ready[0]);
+  const uint32_t b_lfree0 = smem_u32(&ctl->list_free[0]);
   const uint32_t b_drain = smem_u32(&ctl->drain);
 
   if (threadIdx.x == 0) {
@@ -437,11 +443,14 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       mbar_init(b_pfull0 + 8 * t, 4);
       mbar_init(b_odone0 + 8 * t, 1);
     }
-    mbar_init(b_lready, 1);
-    mbar_init(b_lfree, 9);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_lready0 + 8 * b, 1);
+      mbar_init(b_lfree0 + 8 * b, 9);
+    }
     mbar_init(b_drain, 1);
     ctl->abort_flag = 0;
-    ctl->list_count = 0;
+    ctl->list_count[0] = 0;
+    ctl->list_count[1] = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -461,6 +470,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   const int u_end = p.cta_begin[blockIdx.x + 1];
   const bool sparse = p.mode == VKV_MODE_BLOCK_SPARSE;
   const bool ragged = p.mode == VKV_MODE_RAGGED;
+  uint32_t* const list1 = reinterpret_cast<uint32_t*>(smem + C::OFF_KV + (C::NSLOT - 1) * C::KV_BYTES);
+  auto list_buf = [&](int b) { return (SP && b) ? list1 : ctl->list; };
 
   if (warp < 4) {
     setmaxnreg_dec<kRegsProducer>();
@@ -471,19 +482,23 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
         const UnitInfo u = decode_unit(p, p.units[ui]);
         int rs = 0, rl = 0;
+        const int lb = SP ? (int)(ucnt & 1u) : 0;
         if (sparse) {
-          if (ucnt > 0) {
+          // wait for the unit that used this list buffer before (one unit back with a
+          // single buffer, two with two) to release it
+          const uint32_t back = SP ? 2u : 1u;
+          if (ucnt >= back) {
             bool w = true;
-            if (lane == 0) w = mbar_wait(b_lfree, (ucnt - 1) & 1, abort_flag, p.err);
+            if (lane == 0) w = mbar_wait(b_lfree0 + 8 * lb, ((ucnt - back) / back) & 1, abort_flag, p.err);
             ok = __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
             if (!ok) break;
           }
-          build_block_list(p, ctl, u);
-          if (lane == 0) mbar_arrive(b_lready);
+          build_block_list(p, ctl, u, list_buf(lb), &ctl->list_count[lb]);
+          if (lane == 0) mbar_arrive(b_lready0 + 8 * lb);
         } else if (ragged) {
           ragged_range(p, u.s, rs, rl, lane == 0);
         }
-        const int nsteps = unit_steps(p, ctl, rl);
+        const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
         if (nsteps == 0) continue;
         if (lane == 0) {
           if (qcnt > 0) ok = mbar_wait(b_qempty, (qcnt - 1) & 1, abort_flag, p.err);
@@ -511,13 +526,13 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             ++qcnt;
           }
           TileIter it;
-          it.init(&p, ctl, rs, rl);
+          it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
           const int kvh = ragged ? 0 : u.h;
           const int kvb = ragged ? 0 : u.b;
           for (int j = 0; j < nsteps && ok; ++j) {
             const TileDesc td = it.next();
             for (int kv = 0; kv < 2; ++kv) {
-              const uint32_t slot = item % C::NSLOT, use = item / C::NSLOT;
+              const uint32_t slot = item % NS, use = item / NS;
               if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
               if (!ok) break;
               if (item == 0 && p.withhold_first_copy) {
@@ -543,8 +558,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       }
       if (!ok && lane == 0) {
         // let copies already issued land before the CTA exits
-        for (uint32_t i = (item > (uint32_t)C::NSLOT ? item - C::NSLOT : 0); i < item; ++i)
-          mbar_wait_drain(b_full0 + 8 * (i % C::NSLOT), (i / C::NSLOT) & 1);
+        for (uint32_t i = (item > NS ? item - NS : 0); i < item; ++i)
+          mbar_wait_drain(b_full0 + 8 * (i % NS), (i / NS) & 1);
         if (qcnt > 0) mbar_wait_drain(b_qfull, (qcnt - 1) & 1);
       }
       __syncwarp();
@@ -559,7 +574,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         uint32_t pv_cnt[2] = {0, 0};
         bool ok = true;
         auto wait_item = [&](uint32_t it_) {
-          return mbar_wait(b_full0 + 8 * (it_ % C::NSLOT), (it_ / C::NSLOT) & 1, abort_flag, p.err);
+          return mbar_wait(b_full0 + 8 * (it_ % NS), (it_ / NS) & 1, abort_flag, p.err);
         };
         auto issue_qk = [&](int t, uint32_t kslot) {
           const uint32_t d_tm = tmem + (uint32_t)(t * 128);
@@ -575,17 +590,19 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
           const UnitInfo u = decode_unit(p, p.units[ui]);
           int rs = 0, rl = 0;
+          const int lb = SP ? (int)(ucnt & 1u) : 0;
+          const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);  // this buffer's use parity
           if (sparse) {
-            ok = mbar_wait(b_lready, ucnt & 1, abort_flag, p.err);
+            ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
             if (!ok) break;
           } else if (ragged) {
             ragged_range(p, u.s, rs, rl, false);
           }
-          const int nsteps = unit_steps(p, ctl, rl);
-          if (sparse) mbar_arrive(b_lfree);  // only the step count was needed
+          const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
+          if (sparse) mbar_arrive(b_lfree0 + 8 * lb);  // only the step count was needed
           if (nsteps == 0) continue;
           TileIter it;
-          it.init(&p, ctl, rs, rl);
+          it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
           ok = mbar_wait(b_qfull, qcnt & 1, abort_flag, p.err);
           ++qcnt;
           if (!ok) break;
@@ -593,8 +610,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ok = wait_item(item);
           if (!ok) break;
           tc_fence_after();
-          for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % C::NSLOT);
-          mma_commit(b_empty0 + 8 * (item % C::NSLOT));
+          for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % NS);
+          mma_commit(b_empty0 + 8 * (item % NS));
           if (nsteps == 1) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
             const bool first = (sparse || ragged) ? (j == 0) : it.next().first;
@@ -614,7 +631,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               {
                 const uint32_t d_tm = tmem + C::TM_O + (uint32_t)(t * D);
                 const uint32_t pa = tmem + (uint32_t)(t * 128);
-                const uint32_t vb = sKV + (vit % C::NSLOT) * C::KV_BYTES;
+                const uint32_t vb = sKV + (vit % NS) * C::KV_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                   mma_bf16_ts(d_tm, pa + 8 * kk, sdesc_mn_sw128(vb + kk * 2048, C::ATOM), IDESC_PV,
@@ -631,14 +648,14 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
                   k_ready = true;
                   VKV_STAMP(trm + 3 + 4 * t);
                 }
-                issue_qk(t, knext % C::NSLOT);
+                issue_qk(t, knext % NS);
                 VKV_STAMP(trm + 4 + 4 * t);
               }
             }
             if (!ok) break;
-            mma_commit(b_empty0 + 8 * (vit % C::NSLOT));
+            mma_commit(b_empty0 + 8 * (vit % NS));
             if (has_next) {
-              mma_commit(b_empty0 + 8 * (knext % C::NSLOT));
+              mma_commit(b_empty0 + 8 * (knext % NS));
               if (j + 2 == nsteps) mma_commit(b_qempty);
             }
           }
@@ -667,13 +684,15 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
       const UnitInfo u = decode_unit(p, p.units[ui]);
       int rs = 0, rl = 0;
+      const int lb = SP ? (int)(ucnt & 1u) : 0;
       if (sparse) {
-        ok = warp_all(mbar_wait(b_lready, ucnt & 1, abort_flag, p.err));
+        const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);
+        ok = warp_all(mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err));
         if (!ok) break;
       } else if (ragged) {
         ragged_range(p, u.s, rs, rl, false);
       }
-      const int nsteps = unit_steps(p, ctl, rl);
+      const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
       const bool active = t < u.ntiles;
       int qrow = (u.tile0 + t) * 128 + r;
       if (sparse) {
@@ -687,7 +706,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       int cur_branch = -1, prev_branch = -1;
       if (active && nsteps > 0) {
         TileIter it;
-        it.init(&p, ctl, rs, rl);
+        it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
         for (int j = 0; j < nsteps; ++j) {
           const TileDesc td = it.next();
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
@@ -930,7 +949,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       }
       if (sparse) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(b_lfree);
+        if (lane == 0) mbar_arrive(b_lfree0 + 8 * lb);
       }
     }
   }
