@@ -424,6 +424,16 @@ def extras(dev, peaks):
                             "cache_bytes_per_layer": kv.numel() * 2,
                             "dense_cache_bytes_per_layer": 2 * c.H * 128 * c.Lkv * 2}
         del q, kv, o
+    # a batch of 8 chunks, each over its own 21-frame latent cache (the batch size the
+    # smaller cache makes room for)
+    c = W.make_latent(B=8)
+    q, kv = c.q.to(dev), c.kv.to(dev)
+    o = vkv.latent_attn(q, kv, c.d_c, scale=c.scale)
+    ms = statistics.median(timed(lambda: vkv.latent_attn(q, kv, c.d_c, scale=c.scale, out=o), 10, st, flush))
+    fl = oracle.visited_flops_latent(c.B, c.H, c.Lq, c.Lkv, c.d_c, c.d_rope)
+    lat["d_c192_batch8"] = {"ms": ms, "tflops": fl / ms / 1e9, "frac_bf16": fl / ms / 1e9 / peaks["bf16_tflops"],
+                            "ms_per_chunk": ms / c.B}
+    del q, kv, o
     out["latent_wan13b"] = lat
     return out
 

@@ -45,6 +45,7 @@ def _check_full(case, o, lse, what):
     (192, 1, 1, 5, 1, 1.0),         # a single cached row
     (128, 2, 3, 300, 1000, 1.0),    # the smaller latent budget
     (192, 1, 40, 512, 600, 2.0),    # more query tiles than SMs: several tiles per CTA
+    (192, 4, 12, 300, 700, 1.0),    # a batch of chunks, each over its own cache
 ])
 def test_latent_matches_oracle(d_c, B, H, Lq, Lkv, q_std):
     case = W.make_latent("t", seed=11 + Lq, B=B, H=H, Lq=Lq, Lkv=Lkv, d_c=d_c, q_std=q_std)
