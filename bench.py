@@ -621,6 +621,19 @@ def run_profile(args):
         cu = torch.from_numpy(c.cu_seqlens).to(dev)
         o = vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale)
         fn = lambda: vkv.chunk_attn_ragged(q, k, v, cu, c.cu_seqlens, scale=c.scale, out=o)  # noqa: E731
+    elif args.profile == "compaction":
+        ft, hist, cur, recent = 1560, 60, 3, 2
+        rules = [(vkv.HEAD_ANCHOR, 8)] * 4 + [(vkv.HEAD_WAVE, p) for p in (2, 3, 4, 5)] + [(vkv.HEAD_VEIL, 8)] * 4
+        g = torch.Generator(device=dev).manual_seed(12)
+        kd = torch.randn((1, (hist + cur) * ft, 12, 128), generator=g, device=dev).to(torch.bfloat16)
+        vd = torch.randn((1, (hist + cur) * ft, 12, 128), generator=g, device=dev).to(torch.bfloat16)
+        fn = lambda: vkv.compact_cache(kd, vd, rules, ft, hist, cur, recent)  # noqa: E731
+    elif args.profile == "persist":
+        c = W.cfg_sparse()
+        q, k = c.q.to(dev), c.k.to(dev)
+        pers = torch.from_numpy(c.persist_idx).to(dev)
+        pidx, _ = vkv.persist_update(q, k, pers, c.window_blk0, 24)
+        fn = lambda: vkv.persist_update(q, k, pers, c.window_blk0, 24, out_idx=pidx)  # noqa: E731
     elif args.profile == "latent":
         c = W.cfg_latent()
         q, kv = c.q.to(dev), c.kv.to(dev)
@@ -640,7 +653,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
                     help="run one small case for an ncu capture: wan13b, wan14b, merge, select, sparse9, "
-                         "sparse144, ragged, latent")
+                         "sparse144, ragged, latent, compaction, persist")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)

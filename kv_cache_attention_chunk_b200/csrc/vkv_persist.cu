@@ -4,15 +4,17 @@
 // or replace blocks of, the persistent memory; component 2: one representative
 // per block for the coarse score).
 //
-// Three launches on the caller's stream:
+// Three launches on the caller's stream, the last two as programmatic dependent
+// launches (each starts while the one before it drains):
 //   pool_kernel          means of the chunk's 64-row query blocks (shared with
 //                        block selection) -> workspace;
 //   cand_pool_kernel     means of the candidate blocks (current persistent
 //                        blocks, then the evicted range) -> workspace, with a
 //                        validity flag per candidate;
 //   persist_pick_kernel  one CTA per (batch, head): the chunk's mean query from
-//                        the block means (weighted by block rows), one score
-//                        per candidate, rank of each candidate among the valid
+//                        the block means (weighted by block rows; all threads,
+//                        partial sums in shared memory), one score per
+//                        candidate (a warp each), rank of each candidate among the valid
 //                        ones (higher score first, then the lower block id),
 //                        the C best written in ascending block order.
 // Candidate counts are small (C + evicted <= 2048), so ranking by counting is
@@ -60,13 +62,18 @@ __global__ void __launch_bounds__(256) cand_pool_kernel(const CandParams p) {
     ok = true;
   }
   if (threadIdx.x == 0) p.valid[(size_t)s * n_cand + i] = ok ? 1 : 0;
-  if (!ok) return;
+  if (!ok) {
+    griddep_wait();
+    return;
+  }
   const int b = s / p.H, h = s - (s / p.H) * p.H;
   const int c = threadIdx.x % CPR, g = threadIdx.x / CPR;
   const __nv_bfloat16* base = p.k + b * p.k_sb + h * p.k_sh + (long long)blk * 64 * p.k_st;
   uint4 v[RPG];
 #pragma unroll
   for (int r = 0; r < RPG; ++r) v[r] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)(g * RPG + r) * p.k_st) + c);
+  // the pick kernel may be scheduled now; it waits for this grid's completion
+  griddep_launch_dependents();
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -89,6 +96,9 @@ __global__ void __launch_bounds__(256) cand_pool_kernel(const CandParams p) {
     for (int gg = 0; gg < GROUPS; ++gg) sum += part[gg][x];
     dst[x] = sum * (1.f / 64.f);
   }
+  // this grid reads nothing the query pooling writes and may run beside it; it ends
+  // only after that grid has, so the pick kernel's wait on this grid covers both
+  griddep_wait();
 }
 
 struct PickParams {
@@ -109,37 +119,61 @@ __global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
   __shared__ int ids[kMaxCand];
   __shared__ unsigned char ok[kMaxCand];
   __shared__ unsigned char keep[kMaxCand];
+  constexpr int C4 = D / 4;          // 16-byte column chunks of a row
+  constexpr int G = 256 / C4;        // row groups
+  __shared__ float part[G][D];
   const int s = blockIdx.x;
   const int n_cand = p.C + p.n_evict;
-  // mean query of the chunk: block means weighted by their rows (the last block may be short)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();  // both pooling grids before this one on the stream have completed
+  // mean query of the chunk: block means weighted by their rows (the last block may
+  // be short).  Thread (g, c) sums chunk c of query blocks g, g + G, ... (independent
+  // loads, several in flight), then the G partial sums are added in shared memory.
+  {
+    const int c = threadIdx.x % C4, g = threadIdx.x / C4;
+    const float4* qb = reinterpret_cast<const float4*>(p.qbar + (size_t)s * p.n_qblk * D) + c;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int j = g; j < p.n_qblk; j += G) {
+      const float w = (float)min(64, p.Lq - j * 64);
+      const float4 v = __ldg(qb + (size_t)j * C4);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    part[g][4 * c + 0] = acc.x;
+    part[g][4 * c + 1] = acc.y;
+    part[g][4 * c + 2] = acc.z;
+    part[g][4 * c + 3] = acc.w;
+  }
+  __syncthreads();
   for (int x = threadIdx.x; x < D; x += blockDim.x) {
     float acc = 0.f;
-    for (int j = 0; j < p.n_qblk; ++j) {
-      const int rows = min(64, p.Lq - j * 64);
-      acc += (float)rows * p.qbar[((size_t)s * p.n_qblk + j) * D + x];
-    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc += part[g][x];
     qm[x] = acc / (float)p.Lq;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-    ids[i] = i < p.C ? __ldg(p.persist_idx + (size_t)s * p.C + i) : p.evict_blk0 + (i - p.C);
-    ok[i] = p.valid[(size_t)s * n_cand + i];
+  // one warp per candidate: lane l takes columns l, l + 32, ... of the block mean
+  for (int i = warp; i < n_cand; i += blockDim.x >> 5) {
+    const bool valid = p.valid[(size_t)s * n_cand + i] != 0;
     float v = -INFINITY;
-    if (ok[i]) {
+    if (valid) {
       const float* kr = p.kbar + ((size_t)s * n_cand + i) * D;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-      for (int x = 0; x < D; x += 4) {
-        a0 = fmaf(qm[x], kr[x], a0);
-        a1 = fmaf(qm[x + 1], kr[x + 1], a1);
-        a2 = fmaf(qm[x + 2], kr[x + 2], a2);
-        a3 = fmaf(qm[x + 3], kr[x + 3], a3);
-      }
-      v = (a0 + a1) + (a2 + a3);
-      v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);  // NaN ranks last; -0 ties with +0
+      float a = 0.f;
+#pragma unroll
+      for (int x = lane; x < D; x += 32) a = fmaf(qm[x], __ldg(kr + x), a);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+      v = (a != a) ? -INFINITY : (a == 0.f ? 0.f : a);  // NaN ranks last; -0 ties with +0
     }
-    sc[i] = v;
-    if (p.out_scores) p.out_scores[(size_t)s * n_cand + i] = ok[i] ? v : -INFINITY;
+    if (lane == 0) {
+      ids[i] = i < p.C ? __ldg(p.persist_idx + (size_t)s * p.C + i) : p.evict_blk0 + (i - p.C);
+      ok[i] = valid ? 1 : 0;
+      sc[i] = v;
+      if (p.out_scores) p.out_scores[(size_t)s * n_cand + i] = valid ? v : -INFINITY;
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
@@ -168,6 +202,25 @@ __global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Programmatic dependent launch of a 256-thread kernel with one parameter struct:
+// the grid may start while the one before it on the stream is still running, and
+// orders itself with griddep_wait.
+template <class P>
+bool launch_dependent(const void* fn, dim3 grid, cudaStream_t st, P* params) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[1] = {params};
+  return cudaLaunchKernelExC(&cfg, fn, args) == cudaSuccess;
+}
 
 }  // namespace
 }  // namespace vkv
@@ -239,12 +292,9 @@ extern "C" vkv_status vkv_persist_update(const vkv_persist_args* a, vkv_stream_t
   cp.kbar = kbar;
   cp.valid = valid;
   cp.err = a->err_word;
-  const dim3 cg(n_cand, BH);
-  if (a->d == 128)
-    cand_pool_kernel<128><<<cg, 256, 0, st>>>(cp);
-  else
-    cand_pool_kernel<64><<<cg, 256, 0, st>>>(cp);
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  if (!launch_dependent(a->d == 128 ? (const void*)cand_pool_kernel<128> : (const void*)cand_pool_kernel<64>,
+                        dim3(n_cand, BH), st, &cp))
+    return VKV_ERR_CUDA;
   // 3. scores and the top C
   PickParams kp;
   kp.qbar = qbar;
@@ -258,10 +308,8 @@ extern "C" vkv_status vkv_persist_update(const vkv_persist_args* a, vkv_stream_t
   kp.Lq = a->Lq;
   kp.out_idx = a->out_idx;
   kp.out_scores = a->out_scores;
-  if (a->d == 128)
-    persist_pick_kernel<128><<<BH, 256, 0, st>>>(kp);
-  else
-    persist_pick_kernel<64><<<BH, 256, 0, st>>>(kp);
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  if (!launch_dependent(a->d == 128 ? (const void*)persist_pick_kernel<128> : (const void*)persist_pick_kernel<64>,
+                        dim3(BH), st, &kp))
+    return VKV_ERR_CUDA;
   return VKV_OK;
 }
