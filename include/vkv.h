@@ -160,6 +160,21 @@ typedef struct {
    * [0, ceil(Lq/block)) raises VKV_DEVERR_BAD_INDEX; a repeated entry leaves
    * some query block unwritten (not checked). */
   const int32_t* qblk_order;
+
+  /* Optional DEVICE scratch for key-axis splitting (SEGMENTS and RAGGED with
+   * cu_seqlens_host).  NULL: every unit of work is one or two whole query tiles
+   * over all of its keys, and the schedule balances whole units over the SMs.
+   * Otherwise at least vkv_chunk_attn_workspace_size() bytes, 256-byte aligned,
+   * owned by the caller (VKV_ERR_WORKSPACE when smaller): the schedule may then
+   * cut some units into pieces over disjoint key ranges that run on different
+   * SMs; each piece leaves its partial output and LSE in the workspace and the
+   * last piece of a unit to finish combines them exactly (the same LSE merge as
+   * the two branches) and writes the outputs.  Results equal those of an
+   * unsplit run up to fp32 rounding.  Its contents need no initialisation (the
+   * call clears its counters on `stream` first) and are dead after the call;
+   * calls that overlap on the GPU must not share one. */
+  void* workspace;
+  size_t workspace_bytes;
 } vkv_attn_args;
 
 /*
@@ -169,10 +184,42 @@ typedef struct {
  *   s_j = scale * <q_i, k_j>,  O_i = sum_j softmax(s)_j v_j,  LSE_i = ln sum_j exp(s_j).
  * Rows of the cache up to 127 past the end of a segment (SEGMENTS, RAGGED) are
  * read but masked; where they lie inside the cache they must hold finite values.
+ * Limits: B*H < 2^18 and Lq <= 4096 * 128 (else VKV_ERR_UNSUPPORTED).
  * Sources: ISPA summary section 2 step 1; Sparse Forcing summary section 2
  * component 3; Pyramid Forcing summary methodology section 3.
  */
 vkv_status vkv_chunk_attn(const vkv_attn_args* args, vkv_stream_t stream);
+
+/*
+ * Bytes of `workspace` that vkv_chunk_attn can use for these arguments (0 when
+ * its schedule does not split any unit; always 0 for BLOCK_SPARSE and for
+ * RAGGED without cu_seqlens_host).  Reads only the host-side fields (mode,
+ * shapes, segments, cu_seqlens_host); returns 0 for arguments that
+ * vkv_chunk_attn would refuse.  The size depends on the shapes and on the
+ * number of SMs of the current device.
+ */
+size_t vkv_chunk_attn_workspace_size(const vkv_attn_args* args);
+
+/*
+ * vkv_debug_schedule -- test aid (host only, no device needed): the work
+ * schedule vkv_chunk_attn would run for `args` on a device with `n_sm` SMs
+ * (1..160), with key-axis splitting allowed when `split` is non-zero.  Reads
+ * the same host-side fields as vkv_chunk_attn_workspace_size.  Output arrays
+ * are HOST and caller-owned (NULL = skip): cta_begin / cta_piece0 [n_sm + 1],
+ * units [6144], pieces [2 * 384] (uint32 pairs).  Unit code: bits [0, 12)
+ * first 128-row query tile, bit 12 piece, bit 13 two tiles, bits [14, 32)
+ * sequence b*H + h.  Piece pair: first word = first key step | end step << 16,
+ * second = first workspace slot of its unit | piece index << 16 | piece
+ * count << 24; the pieces of CTA c start at cta_piece0[c], in unit order.
+ */
+typedef struct {
+  int32_t n_ctas, n_units, n_pieces, n_slots;
+  int32_t* cta_begin;
+  int32_t* cta_piece0;
+  uint32_t* units;
+  uint32_t* pieces;
+} vkv_schedule;
+vkv_status vkv_debug_schedule(const vkv_attn_args* args, int32_t n_sm, int32_t split, vkv_schedule* out);
 
 /*
  * Block selection for VKV_MODE_BLOCK_SPARSE (Sparse Forcing summary, section 2

@@ -24,6 +24,10 @@ struct Plan {
   int n_ctas = 0;
   std::vector<int> cta_begin;
   std::vector<uint32_t> units;
+  // key-axis pieces (empty when no unit is split)
+  std::vector<int> cta_piece0;
+  std::vector<uint2> pieces;
+  int n_slots = 0;
 };
 
 struct Cand {
@@ -69,17 +73,164 @@ double lpt(std::vector<Cand>& units, int g, Plan* out) {
       out->units.insert(out->units.end(), per[c].begin(), per[c].end());
     }
     out->cta_begin[g] = (int)out->units.size();
+    out->cta_piece0.assign(g + 1, 0);
+    out->pieces.clear();
+    out->n_slots = 0;
   }
   return mk;
 }
+
+constexpr uint32_t kPieceBit = 1u << 12;
 
 inline uint32_t unit_code(int s, int tile0, bool two) {
   return ((uint32_t)s << 14) | (two ? (1u << 13) : 0u) | (uint32_t)tile0;
 }
 
+// Fixed cost of a unit (Q load, first product, epilogue) and of a piece (the
+// same plus its partial in the workspace and a share of the combine), in key
+// steps; pieces are at least kMinPieceSteps long.
+constexpr double kUnitOverhead = 2.0;
+constexpr double kPieceOverhead = 4.0;
+constexpr int kMinPieceSteps = 16;
+
+// Schedule with key-axis pieces: longest-first onto the least loaded CTA, as for
+// whole units, but against a capacity T = slack * (total cost / CTAs).  A unit
+// that does not fit the least loaded CTA is cut: the piece that fills that CTA
+// up to T stays there, and the rest of its key steps goes back into the queue
+// as an item of its own (cut again if needed, at most kMaxPiecesPerUnit pieces).
+// The best of a few slacks is kept.  steps[s] is the key-step count of sequence s.
+bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
+                const std::vector<int>& steps, int n_sm, Plan* out, double* mk_out) {
+  struct Item {
+    double cost;
+    uint32_t code;
+    int S;       // steps of the whole unit
+    int j0, j1;  // steps still to place
+    double rate;
+    int k;       // pieces already cut from this unit
+    int unit;    // index of the unit (for its piece list)
+  };
+  auto cmp = [](const Item& a, const Item& b) {
+    if (a.cost != b.cost) return a.cost < b.cost;  // max-heap on cost
+    return a.unit > b.unit;                        // then the earlier unit
+  };
+  std::vector<Item> base;
+  for (int s = 0; s < n_seq; ++s) {
+    for (int i = 0; i < T / 2; ++i)
+      base.push_back({pair_cost[s], unit_code(s, 2 * i, true), steps[s], 0, steps[s], 1.0, 0, 0});
+    if (T & 1)
+      base.push_back({one_cost[s], unit_code(s, T - 1, false), steps[s], 0, steps[s], 0.0, 0, 0});
+  }
+  if (base.empty() || (long long)base.size() > kMaxUnits) return false;
+  double tot = 0, lb_piece = 0;
+  for (size_t i = 0; i < base.size(); ++i) {
+    base[i].unit = (int)i;
+    base[i].rate = base[i].cost / (base[i].S + kUnitOverhead);
+    tot += base[i].cost;
+    // no CTA can finish before a unit cut into the most pieces allowed
+    lb_piece = std::max(lb_piece, base[i].rate * ((double)base[i].S / kMaxPiecesPerUnit + kPieceOverhead));
+  }
+  const int g = n_sm;
+  const double lb = std::max(tot / g, lb_piece);
+  const double slacks[] = {1.0, 1.01, 1.015, 1.02, 1.03, 1.05, 1.07, 1.1, 1.2, 1.4};
+  double best = 1e300;
+  using E = std::pair<double, int>;
+  for (double slack : slacks) {
+    const double cap = lb * slack;
+    std::priority_queue<Item, std::vector<Item>, decltype(cmp)> q(cmp, base);
+    std::priority_queue<E, std::vector<E>, std::greater<E>> heap;
+    for (int c = 0; c < g; ++c) heap.push({0.0, c});
+    // per CTA: (unit index, j0, j1) in placement order; j1 < 0 marks a whole unit
+    std::vector<std::vector<std::pair<int, std::pair<int, int>>>> lists(g);
+    std::vector<int> n_cut(base.size(), 0);
+    while (!q.empty()) {
+      Item it = q.top();
+      q.pop();
+      E e = heap.top();
+      heap.pop();
+      const bool whole_unit = it.k == 0;
+      int n = it.j1 - it.j0;
+      if (e.first + it.cost > cap && it.k < kMaxPiecesPerUnit - 1 && it.S <= 0xFFFF) {
+        const int fit = (int)((cap - e.first) / it.rate - kPieceOverhead);
+        if (fit >= kMinPieceSteps && n - fit >= kMinPieceSteps) n = fit;
+      }
+      if (n == it.j1 - it.j0) {
+        // the rest of the unit in one go
+        e.first += it.cost;
+        lists[e.second].push_back({it.unit, {whole_unit ? 0 : it.j0, whole_unit ? -1 : it.j1}});
+        if (!whole_unit) ++n_cut[it.unit];
+      } else {
+        e.first += it.rate * (n + kPieceOverhead);
+        lists[e.second].push_back({it.unit, {it.j0, it.j0 + n}});
+        ++n_cut[it.unit];
+        Item rest = it;
+        rest.j0 = it.j0 + n;
+        rest.k = it.k + 1;
+        rest.cost = it.rate * (rest.j1 - rest.j0 + kPieceOverhead);
+        q.push(rest);
+      }
+      heap.push(e);
+    }
+    double mk = 0;
+    while (!heap.empty()) {
+      mk = std::max(mk, heap.top().first);
+      heap.pop();
+    }
+    // slots: the pieces of a unit get consecutive slots, numbered in j0 order
+    std::vector<int> slot0(base.size(), -1);
+    int n_slots = 0, n_pieces = 0, n_units = 0;
+    for (size_t i = 0; i < base.size(); ++i)
+      if (n_cut[i] > 0) {
+        slot0[i] = n_slots;
+        n_slots += n_cut[i];
+        n_pieces += n_cut[i];
+      }
+    for (int c = 0; c < g; ++c) n_units += (int)lists[c].size();
+    if (n_pieces > kMaxPieces || n_units > kMaxUnits || n_slots > 0xFFFF) continue;
+    if (!(mk < best)) continue;
+    best = mk;
+    // piece index of a cut = its rank among the unit's cuts by j0
+    std::vector<std::vector<int>> starts(base.size());
+    for (int c = 0; c < g; ++c)
+      for (const auto& e : lists[c])
+        if (e.second.second >= 0) starts[e.first].push_back(e.second.first);
+    for (auto& v : starts) std::sort(v.begin(), v.end());
+    out->n_ctas = g;
+    out->cta_begin.assign(g + 1, 0);
+    out->cta_piece0.assign(g + 1, 0);
+    out->units.clear();
+    out->pieces.clear();
+    for (int c = 0; c < g; ++c) {
+      out->cta_begin[c] = (int)out->units.size();
+      out->cta_piece0[c] = (int)out->pieces.size();
+      for (const auto& e : lists[c]) {
+        const Item& b = base[e.first];
+        if (e.second.second < 0) {
+          out->units.push_back(b.code);
+          continue;
+        }
+        const auto& v = starts[e.first];
+        const int idx = (int)(std::lower_bound(v.begin(), v.end(), e.second.first) - v.begin());
+        out->units.push_back(b.code | kPieceBit);
+        out->pieces.push_back(make_uint2((uint32_t)e.second.first | ((uint32_t)e.second.second << 16),
+                                         (uint32_t)slot0[e.first] | ((uint32_t)idx << 16) |
+                                             ((uint32_t)n_cut[e.first] << 24)));
+      }
+    }
+    out->cta_begin[g] = (int)out->units.size();
+    out->cta_piece0[g] = (int)out->pieces.size();
+    out->n_slots = n_slots;
+  }
+  if (best >= 1e299) return false;
+  *mk_out = best;
+  return true;
+}
+
 // pair_cost[s] / single_cost[s]: estimated cost of a 2-tile / 1-tile unit of sequence s.
+// steps (empty: unknown) gives each sequence's key steps; with it the schedule
+// may split units along the key axis when that shortens it by 3 % or more.
 bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
-               const std::vector<double>& one_cost, int n_sm, Plan* plan) {
+               const std::vector<double>& one_cost, const std::vector<int>& steps, int n_sm, Plan* plan) {
   // sequences by decreasing pair cost: their pairs are split first
   std::vector<int> order(n_seq);
   for (int s = 0; s < n_seq; ++s) order[s] = s;
@@ -126,6 +277,15 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
       best_split = c;
     }
   }
+  if (!steps.empty()) {
+    Plan sp;
+    double mk_split = 1e300;
+    // the whole-unit makespan in the same cost terms (a split plan always uses n_sm CTAs)
+    if (split_plan(n_seq, T, pair_cost, one_cost, steps, n_sm, &sp, &mk_split) && mk_split < 0.97 * best) {
+      *plan = std::move(sp);
+      return true;
+    }
+  }
   if (best >= 1e299) return false;
   build(best_split, u);
   const int g = (int)std::min<long long>(n_sm, (long long)u.size());
@@ -136,15 +296,15 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
 std::mutex g_plan_mu;
 std::map<std::string, std::shared_ptr<Plan>> g_plans;
 
-std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T,
-                               const std::vector<double>& pc, const std::vector<double>& oc, int n_sm) {
+std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const std::vector<double>& pc,
+                               const std::vector<double>& oc, const std::vector<int>& steps, int n_sm) {
   {
     std::lock_guard<std::mutex> lk(g_plan_mu);
     auto it = g_plans.find(key);
     if (it != g_plans.end()) return it->second;
   }
   auto plan = std::make_shared<Plan>();
-  if (!make_plan(n_seq, T, pc, oc, n_sm, plan.get())) return nullptr;
+  if (!make_plan(n_seq, T, pc, oc, steps, n_sm, plan.get())) return nullptr;
   std::lock_guard<std::mutex> lk(g_plan_mu);
   if (g_plans.size() > 256) g_plans.clear();
   g_plans[key] = plan;
@@ -208,9 +368,28 @@ bool out_ok(const vkv_tensor& t) {
 
 }  // namespace vkv
 
-using namespace vkv;
+namespace vkv {
+namespace {
 
-extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream) {
+// Bytes of the piece workspace: counters, LSEs, partial outputs (all 256-aligned).
+struct WsLayout {
+  size_t cnt_off, l_off, o_off, bytes;
+};
+
+WsLayout ws_layout(int n_slots, int nbr, int d) {
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  WsLayout w;
+  w.cnt_off = 0;
+  w.l_off = al((size_t)n_slots * 8 * sizeof(int));
+  w.o_off = w.l_off + al((size_t)n_slots * 2 * nbr * 128 * sizeof(float));
+  w.bytes = n_slots > 0 ? w.o_off + (size_t)n_slots * 2 * nbr * 128 * d * sizeof(float) : 0;
+  return w;
+}
+
+// Checks the arguments and builds the kernel parameters and the schedule.
+// check_ptrs = false (workspace size query): only the host-side fields are read.
+vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, AttnParams* P,
+                      std::shared_ptr<Plan>* plan_out, int* dev_out, int n_sm_override = 0) {
   if (!a) return VKV_ERR_NULL;
   const int mode = a->mode;
   if (mode != VKV_MODE_SEGMENTS && mode != VKV_MODE_BLOCK_SPARSE && mode != VKV_MODE_RAGGED)
@@ -221,13 +400,14 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   const int B = a->B, H = a->H, Lq = a->Lq, Lkv = a->Lkv, d = a->d;
   const long long n_seq = (long long)B * H;
   const int T = (Lq + 127) / 128;
-  if (n_seq >= (1ll << 18) || T > 8192) return VKV_ERR_UNSUPPORTED;
-  if (!a->q.ptr || !a->k.ptr || !a->v.ptr) return VKV_ERR_NULL;
-  if (!tensor_aligned(a->q) || !tensor_aligned(a->k) || !tensor_aligned(a->v)) return VKV_ERR_ALIGN;
-  if (!dims_ok_for_tma(a->q, B, Lq, H, d)) return VKV_ERR_SHAPE;
+  if (n_seq >= (1ll << 18) || T > 4096) return VKV_ERR_UNSUPPORTED;
+  if (check_ptrs) {
+    if (!a->q.ptr || !a->k.ptr || !a->v.ptr) return VKV_ERR_NULL;
+    if (!tensor_aligned(a->q) || !tensor_aligned(a->k) || !tensor_aligned(a->v)) return VKV_ERR_ALIGN;
+    if (!dims_ok_for_tma(a->q, B, Lq, H, d)) return VKV_ERR_SHAPE;
+  }
 
-  auto P = std::make_unique<AttnParams>();
-  std::memset(P.get(), 0, sizeof(AttnParams));
+  std::memset(P, 0, sizeof(AttnParams));
   P->mode = mode;
   P->B = B;
   P->H = H;
@@ -236,16 +416,17 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   P->d = d;
   P->scale_log2 = a->scale * 1.4426950408889634f;
   P->err = a->err_word;
-  P->withhold_first_copy = take_withhold_request() ? 1 : 0;
 
   int nb = 1;
   std::vector<double> pc(n_seq), oc(n_seq);
+  std::vector<int> steps;  // per sequence, when the schedule may split units
   const double c1 = single_tile_cost();
   std::string key;
   if (mode == VKV_MODE_SEGMENTS) {
     nb = a->n_branches;
     if (nb < 1 || nb > 2) return VKV_ERR_SHAPE;
-    if (Lkv <= 0 || !dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d))
+    if (Lkv <= 0) return VKV_ERR_SHAPE;
+    if (check_ptrs && (!dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d)))
       return VKV_ERR_SHAPE;
     P->n_branches = nb;
     int nf = 0, total = 0;
@@ -254,7 +435,7 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
       if (ns < 0 || ns > VKV_MAX_SEGMENTS) return VKV_ERR_SHAPE;
       if (ns > 0 && !a->segs[br]) return VKV_ERR_NULL;
       bool first = true;
-      int steps = 0;
+      int stp = 0;
       for (int i = 0; i < ns; ++i) {
         const vkv_segment sg = a->segs[br][i];
         if (sg.start < 0 || sg.len < 0 || (long long)sg.start + sg.len > Lkv) return VKV_ERR_RANGE;
@@ -263,13 +444,13 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
         P->flat_len[nf] = sg.len;
         P->flat_branch[nf] = br;
         P->flat_first[nf] = first ? 1 : 0;
-        P->flat_step0[nf] = total + steps;
+        P->flat_step0[nf] = total + stp;
         first = false;
-        steps += (sg.len + 127) / 128;
+        stp += (sg.len + 127) / 128;
         ++nf;
       }
-      P->branch_steps[br] = steps;
-      total += steps;
+      P->branch_steps[br] = stp;
+      total += stp;
     }
     P->n_flat = nf;
     P->total_steps = total;
@@ -277,16 +458,19 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
       pc[s] = total + 2.0;
       oc[s] = c1 * (total + 2.0);
     }
+    if (want_split) steps.assign(n_seq, total);
     key = "S" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(total);
   } else if (mode == VKV_MODE_BLOCK_SPARSE) {
     if (a->block != 64) return VKV_ERR_UNSUPPORTED;
-    if (Lkv <= 0 || !dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d))
+    if (Lkv <= 0) return VKV_ERR_SHAPE;
+    if (check_ptrs && (!dims_ok_for_tma(a->k, B, Lkv, H, d) || !dims_ok_for_tma(a->v, B, Lkv, H, d)))
       return VKV_ERR_SHAPE;
     if (a->n_persist < 0 || a->topk < 0 || a->n_win_blk < 0 || a->window_blk0 < 0) return VKV_ERR_SHAPE;
     if (a->n_win_blk > 1024 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
     if ((long long)(a->window_blk0 + a->n_win_blk) * 64 > Lkv) return VKV_ERR_RANGE;
     if (a->n_persist + std::min(a->n_win_blk, 4 * a->topk) > kMaxListEntries) return VKV_ERR_UNSUPPORTED;
-    if ((a->n_persist > 0 && !a->persist_idx) || (a->topk > 0 && !a->sel_idx)) return VKV_ERR_NULL;
+    if (check_ptrs && ((a->n_persist > 0 && !a->persist_idx) || (a->topk > 0 && !a->sel_idx)))
+      return VKV_ERR_NULL;
     P->n_persist = a->n_persist;
     P->topk = a->topk;
     P->window_blk0 = a->window_blk0;
@@ -310,19 +494,22 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
           std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n");
   } else {
-    if (!a->cu_seqlens) return VKV_ERR_NULL;
-    if (Lkv <= 0 || a->k.st <= 0 || a->v.st <= 0 || (a->k.st % 8) || (a->v.st % 8)) return VKV_ERR_SHAPE;
+    if (check_ptrs && !a->cu_seqlens) return VKV_ERR_NULL;
+    if (Lkv <= 0) return VKV_ERR_SHAPE;
+    if (check_ptrs && (a->k.st <= 0 || a->v.st <= 0 || (a->k.st % 8) || (a->v.st % 8))) return VKV_ERR_SHAPE;
     if (a->cu_seqlens_host) {
       const int32_t* cu = a->cu_seqlens_host;
       if (cu[0] < 0) return VKV_ERR_RANGE;
       for (long long s = 0; s < n_seq; ++s)
         if (cu[s + 1] < cu[s] || cu[s + 1] > Lkv) return VKV_ERR_RANGE;
       key = "R" + std::to_string(n_seq) + "/" + std::to_string(T);
+      if (want_split) steps.resize(n_seq);
       for (long long s = 0; s < n_seq; ++s) {
-        const int steps = (cu[s + 1] - cu[s] + 127) / 128;
-        pc[s] = steps + 2.0;
-        oc[s] = c1 * (steps + 2.0);
-        key += "," + std::to_string(steps);
+        const int stp = (cu[s + 1] - cu[s] + 127) / 128;
+        pc[s] = stp + 2.0;
+        oc[s] = c1 * (stp + 2.0);
+        if (want_split) steps[s] = stp;
+        key += "," + std::to_string(stp);
       }
     } else {
       for (long long s = 0; s < n_seq; ++s) {
@@ -333,36 +520,107 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     }
     P->cu_seqlens = a->cu_seqlens;
   }
-  const int nout = (mode == VKV_MODE_SEGMENTS) ? nb : 1;
-  for (int br = 0; br < nout; ++br) {
-    if (!a->lse[br]) return VKV_ERR_NULL;
-    if (!out_ok(a->o[br])) return a->o[br].ptr ? VKV_ERR_ALIGN : VKV_ERR_NULL;
-    P->o[br] = reinterpret_cast<__nv_bfloat16*>(a->o[br].ptr);
-    P->o_sb[br] = a->o[br].sb;
-    P->o_st[br] = a->o[br].st;
-    P->o_sh[br] = a->o[br].sh;
-    P->lse[br] = a->lse[br];
-  }
-  if (mode == VKV_MODE_SEGMENTS && nb == 2 && a->o_merged.ptr) {
-    if (!a->lse_merged) return VKV_ERR_NULL;
-    if (!out_ok(a->o_merged)) return VKV_ERR_ALIGN;
-    P->om = reinterpret_cast<__nv_bfloat16*>(a->o_merged.ptr);
-    P->om_sb = a->o_merged.sb;
-    P->om_st = a->o_merged.st;
-    P->om_sh = a->o_merged.sh;
-    P->lsem = a->lse_merged;
+  if (check_ptrs) {
+    const int nout = (mode == VKV_MODE_SEGMENTS) ? nb : 1;
+    for (int br = 0; br < nout; ++br) {
+      if (!a->lse[br]) return VKV_ERR_NULL;
+      if (!out_ok(a->o[br])) return a->o[br].ptr ? VKV_ERR_ALIGN : VKV_ERR_NULL;
+      P->o[br] = reinterpret_cast<__nv_bfloat16*>(a->o[br].ptr);
+      P->o_sb[br] = a->o[br].sb;
+      P->o_st[br] = a->o[br].st;
+      P->o_sh[br] = a->o[br].sh;
+      P->lse[br] = a->lse[br];
+    }
+    if (mode == VKV_MODE_SEGMENTS && nb == 2 && a->o_merged.ptr) {
+      if (!a->lse_merged) return VKV_ERR_NULL;
+      if (!out_ok(a->o_merged)) return VKV_ERR_ALIGN;
+      P->om = reinterpret_cast<__nv_bfloat16*>(a->o_merged.ptr);
+      P->om_sb = a->o_merged.sb;
+      P->om_st = a->o_merged.st;
+      P->om_sh = a->o_merged.sh;
+      P->lsem = a->lse_merged;
+    }
   }
 
   int dev = 0;
-  const int n_sm = device_sm_count(&dev);
+  const int n_sm = n_sm_override > 0 ? n_sm_override : device_sm_count(&dev);
   if (n_sm <= 0) return VKV_ERR_CUDA;
   const int g_max = std::min(n_sm, kMaxCtas);
-  key += "@" + std::to_string(g_max) + ":" + std::to_string(c1);
-  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, g_max);
+  key += "@" + std::to_string(g_max) + ":" + std::to_string(c1) + (steps.empty() ? "" : "/split");
+  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, g_max);
   if (!plan) return VKV_ERR_UNSUPPORTED;
   P->n_ctas = plan->n_ctas;
   std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);
+  std::copy(plan->cta_piece0.begin(), plan->cta_piece0.end(), P->cta_piece0);
+  std::copy(plan->pieces.begin(), plan->pieces.end(), P->pieces);
   std::copy(plan->units.begin(), plan->units.end(), P->units);
+  *plan_out = plan;
+  *dev_out = dev;
+  return VKV_OK;
+}
+
+}  // namespace
+}  // namespace vkv
+
+using namespace vkv;
+
+extern "C" size_t vkv_chunk_attn_workspace_size(const vkv_attn_args* a) {
+  if (!a || (a->mode != VKV_MODE_SEGMENTS && a->mode != VKV_MODE_RAGGED)) return 0;
+  auto P = std::make_unique<AttnParams>();
+  std::shared_ptr<Plan> plan;
+  int dev = 0;
+  if (attn_setup(a, false, true, P.get(), &plan, &dev) != VKV_OK) return 0;
+  const int nbr = a->mode == VKV_MODE_RAGGED ? 1 : a->n_branches;
+  return ws_layout(plan->n_slots, nbr, a->d).bytes;
+}
+
+extern "C" vkv_status vkv_debug_schedule(const vkv_attn_args* a, int32_t n_sm, int32_t split,
+                                         vkv_schedule* out) {
+  if (!a || !out || n_sm <= 0 || n_sm > kMaxCtas) return VKV_ERR_SHAPE;
+  auto P = std::make_unique<AttnParams>();
+  std::shared_ptr<Plan> plan;
+  int dev = 0;
+  const vkv_status stt =
+      attn_setup(a, false, split != 0 && a->mode != VKV_MODE_BLOCK_SPARSE, P.get(), &plan, &dev, n_sm);
+  if (stt != VKV_OK) return stt;
+  out->n_ctas = plan->n_ctas;
+  out->n_units = (int32_t)plan->units.size();
+  out->n_pieces = (int32_t)plan->pieces.size();
+  out->n_slots = plan->n_slots;
+  if (out->cta_begin) std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), out->cta_begin);
+  if (out->cta_piece0) std::copy(plan->cta_piece0.begin(), plan->cta_piece0.end(), out->cta_piece0);
+  if (out->units) std::copy(plan->units.begin(), plan->units.end(), out->units);
+  if (out->pieces)
+    for (size_t i = 0; i < plan->pieces.size(); ++i) {
+      out->pieces[2 * i] = plan->pieces[i].x;
+      out->pieces[2 * i + 1] = plan->pieces[i].y;
+    }
+  return VKV_OK;
+}
+
+extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream) {
+  if (!a) return VKV_ERR_NULL;
+  const bool want_split = a->workspace != nullptr && a->mode != VKV_MODE_BLOCK_SPARSE;
+  auto P = std::make_unique<AttnParams>();
+  std::shared_ptr<Plan> plan;
+  int dev = 0;
+  const vkv_status stt = attn_setup(a, true, want_split, P.get(), &plan, &dev);
+  if (stt != VKV_OK) return stt;
+  P->withhold_first_copy = take_withhold_request() ? 1 : 0;
+  const int mode = a->mode, B = a->B, H = a->H, Lq = a->Lq, Lkv = a->Lkv, d = a->d;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (plan->n_slots > 0) {
+    const int nbr = mode == VKV_MODE_RAGGED ? 1 : a->n_branches;
+    const WsLayout w = ws_layout(plan->n_slots, nbr, d);
+    if (a->workspace_bytes < w.bytes) return VKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(a->workspace) & 255) return VKV_ERR_ALIGN;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(a->workspace);
+    P->ws_cnt = reinterpret_cast<int*>(ws + w.cnt_off);
+    P->ws_l = reinterpret_cast<float*>(ws + w.l_off);
+    P->ws_o = reinterpret_cast<float*>(ws + w.o_off);
+    if (cudaMemsetAsync(P->ws_cnt, 0, (size_t)plan->n_slots * 8 * sizeof(int), st) != cudaSuccess)
+      return VKV_ERR_CUDA;
+  }
 
   // BLOCK_SPARSE loads a query tile as two 64-row blocks (a unit's blocks follow qblk_order)
   if (!encode_bhld(&P->tm_q, a->q, B, Lq, H, d, mode == VKV_MODE_BLOCK_SPARSE ? 64 : 128)) return VKV_ERR_CUDA;
@@ -374,7 +632,6 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   }
   const bool sp = mode == VKV_MODE_BLOCK_SPARSE;
   if (!set_smem_attr(dev, d, sp)) return VKV_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) {
     if (sp)
       chunk_attn_kernel<128, true><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);

@@ -103,6 +103,20 @@ struct TileIter {
     j = 0;
   }
 
+  // Start the walk at key-tile step j0 (a piece of a split unit); SEGMENTS and
+  // RAGGED only, with j0 below the unit's step count.
+  __device__ __forceinline__ void seek(int j0) {
+    if (p->mode == VKV_MODE_SEGMENTS) {
+      int kk = 0;
+      while (kk + 1 < p->n_flat && p->flat_step0[kk + 1] <= j0) ++kk;
+      k = kk;
+      off = (j0 - p->flat_step0[kk]) * 128;
+    } else {
+      off = j0 * 128;
+    }
+    j = j0;
+  }
+
   __device__ __forceinline__ TileDesc next() {
     TileDesc t;
     if (p->mode == VKV_MODE_BLOCK_SPARSE) {
@@ -156,11 +170,48 @@ struct UnitInfo {
   int b, h;
   int tile0;   // first 128-row query tile
   int ntiles;  // 1 or 2
+  bool piece;  // covers only the key steps of its piece entry
 };
+
+struct PieceInfo {
+  int j0, j1;  // key-tile steps [j0, j1) of the unit's stream
+  int slot0;   // the unit's first workspace slot (its counters live there)
+  int idx, n;  // this piece's index and the unit's piece count
+};
+
+__device__ __forceinline__ PieceInfo piece_info(const AttnParams& p, int k) {
+  const uint2 e = p.pieces[k];
+  PieceInfo r;
+  r.j0 = (int)(e.x & 0xFFFFu);
+  r.j1 = (int)(e.x >> 16);
+  r.slot0 = (int)(e.y & 0xFFFFu);
+  r.idx = (int)((e.y >> 16) & 0xFFu);
+  r.n = (int)(e.y >> 24);
+  return r;
+}
+
+// Steps of this unit entry: all `full` steps of the unit's stream, or the part
+// [j0, j1) of a piece.  RAGGED lengths are read on the device and may differ
+// from the host copy the pieces were cut from: the range is clamped to `full`,
+// and the unit's last piece runs to `full`, so the pieces always cover the
+// device's key range.  Advances the CTA's piece cursor; every role walks the
+// same unit list.
+__device__ __forceinline__ int entry_steps(const AttnParams& p, const UnitInfo& u, int full, int& piece_k,
+                                           PieceInfo& pi) {
+  if (!u.piece) {
+    pi.j0 = 0;
+    pi.n = 0;
+    return full;
+  }
+  pi = piece_info(p, piece_k++);
+  const int j1 = (pi.idx == pi.n - 1) ? full : min(pi.j1, full);
+  return max(0, j1 - pi.j0);
+}
 
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, uint32_t code) {
   UnitInfo u;
-  u.tile0 = (int)(code & 0x1FFFu);
+  u.tile0 = (int)(code & 0xFFFu);
+  u.piece = ((code >> 12) & 1u) != 0;
   u.ntiles = ((code >> 13) & 1u) ? 2 : 1;
   u.s = (int)(code >> 14);
   u.b = u.s / p.H;
@@ -391,6 +442,117 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float&
 
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Key-axis pieces.  A piece of a split unit leaves, per branch it reached, O / l
+// (fp32) and its LSE (log2 units) in its workspace slot; the last piece of the
+// unit to arrive combines them (the LSE merge, the same as between branches).
+__device__ __forceinline__ size_t piece_row(const AttnParams& p, int slot, int t, int br, int r) {
+  const int nbr = p.mode == VKV_MODE_RAGGED ? 1 : p.n_branches;
+  return ((size_t)(slot * 2 + t) * nbr + br) * 128 + r;
+}
+
+// One branch of this piece: O from TMEM divided by l, and m + log2 l.  All
+// lanes of the warp take part (tcgen05.ld); rows past Lq store nothing.
+template <int D>
+__device__ __forceinline__ void piece_store(const AttnParams& p, const PieceInfo& pi, int t, int br, int r,
+                                            bool row_ok, uint32_t tO, float m, float l) {
+  const size_t row = piece_row(p, pi.slot0 + pi.idx, t, br, r);
+  const bool has = l > 0.f;
+  const float inv = has ? 1.f / l : 0.f;
+  float* dst = p.ws_o + row * D;
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tO + c0, v);
+    tmem_ld_wait();
+    reg_fence<32>(v);
+    if (row_ok) {
+      float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        d4[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
+                            __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
+    }
+  }
+  if (row_ok) p.ws_l[row] = has ? m + lg2_approx(l) : -INFINITY;
+}
+
+// Row r of tile t of a split unit from all of its pieces: per branch
+// L = log2 sum_i 2^L_i and O = sum_i 2^(L_i - L) O_i, then the outputs exactly
+// as an unsplit unit writes them (branch rows, LSEs, and the merge of two branches).
+template <int D>
+__device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
+                                              int r, int qrow) {
+  const bool ragged = p.mode == VKV_MODE_RAGGED;
+  const int nbr = ragged ? 1 : p.n_branches;
+  const bool do_merge = p.om != nullptr && nbr == 2;
+  float w[2][kMaxPiecesPerUnit];
+  float L[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    float Li[kMaxPiecesPerUnit];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+      Li[i] = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) : -INFINITY;
+      mx = fmaxf(mx, Li[i]);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+      w[br][i] = (Li[i] == -INFINITY) ? 0.f : ex2_approx(Li[i] - mx);
+      den += w[br][i];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) w[br][i] *= inv;
+    L[br] = den > 0.f ? mx + lg2_approx(den) : -INFINITY;
+  }
+  const float M = fmaxf(L[0], L[1]);
+  const float Ms = (M == -INFINITY) ? 0.f : M;
+  const float e0 = (L[0] == -INFINITY) ? 0.f : ex2_approx(L[0] - Ms);
+  const float e1 = (L[1] == -INFINITY) ? 0.f : ex2_approx(L[1] - Ms);
+  const float den = e0 + e1;
+  const float cb[2] = {den > 0.f ? e0 / den : 0.f, den > 0.f ? e1 / den : 0.f};
+  __nv_bfloat16* mrow = do_merge ? p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh : nullptr;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float g[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) g[e] = 0.f;
+#pragma unroll
+    for (int br = 0; br < 2; ++br) {
+      if (br >= nbr) continue;
+      float f[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) f[e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+        if (w[br][i] > 0.f) {
+          const float4* src =
+              reinterpret_cast<const float4*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D + c0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 x = __ldcg(src + q);
+            f[4 * q] = fmaf(w[br][i], x.x, f[4 * q]);
+            f[4 * q + 1] = fmaf(w[br][i], x.y, f[4 * q + 1]);
+            f[4 * q + 2] = fmaf(w[br][i], x.z, f[4 * q + 2]);
+            f[4 * q + 3] = fmaf(w[br][i], x.w, f[4 * q + 3]);
+          }
+        }
+      }
+      __nv_bfloat16* orow = p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
+      store_row32(orow + c0, f);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) g[e] = fmaf(cb[br], f[e], g[e]);
+    }
+    if (do_merge) store_row32(mrow + c0, g);
+  }
+  for (int br = 0; br < nbr; ++br)
+    p.lse[br][(size_t)u.s * p.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
+  if (do_merge)
+    p.lsem[(size_t)u.s * p.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
+}
+
 // Register split between the producer/MMA warpgroup and the two softmax
 // warpgroups.  setmaxnreg.inc only succeeds if the total stays within what the
 // CTA was launched with (384 threads x 168 registers); the host checks the
@@ -478,6 +640,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     if (warp == 0) {
       // ------------------------------------------------------------ producer
       uint32_t item = 0, qcnt = 0, ucnt = 0;
+      int piece_k = p.cta_piece0[blockIdx.x];
       bool ok = true;
       for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
         const UnitInfo u = decode_unit(p, p.units[ui]);
@@ -498,7 +661,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         } else if (ragged) {
           ragged_range(p, u.s, rs, rl, lane == 0);
         }
-        const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
+        PieceInfo pi;
+        const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
         if (nsteps == 0) continue;
         if (lane == 0) {
           if (qcnt > 0) ok = mbar_wait(b_qempty, (qcnt - 1) & 1, abort_flag, p.err);
@@ -527,6 +691,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           }
           TileIter it;
           it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
+          if (u.piece) it.seek(pi.j0);
           const int kvh = ragged ? 0 : u.h;
           const int kvb = ragged ? 0 : u.b;
           for (int j = 0; j < nsteps && ok; ++j) {
@@ -572,6 +737,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
         uint32_t item = 0, qcnt = 0, ucnt = 0;
         uint32_t pv_cnt[2] = {0, 0};
+        int piece_k = p.cta_piece0[blockIdx.x];
         bool ok = true;
         auto wait_item = [&](uint32_t it_) {
           return mbar_wait(b_full0 + 8 * (it_ % NS), (it_ / NS) & 1, abort_flag, p.err);
@@ -598,11 +764,13 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           } else if (ragged) {
             ragged_range(p, u.s, rs, rl, false);
           }
-          const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
+          PieceInfo pi;
+          const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
           if (sparse) mbar_arrive(b_lfree0 + 8 * lb);  // only the step count was needed
           if (nsteps == 0) continue;
           TileIter it;
           it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
+          if (u.piece) it.seek(pi.j0);
           ok = mbar_wait(b_qfull, qcnt & 1, abort_flag, p.err);
           ++qcnt;
           if (!ok) break;
@@ -614,7 +782,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           mma_commit(b_empty0 + 8 * (item % NS));
           if (nsteps == 1) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
-            const bool first = (sparse || ragged) ? (j == 0) : it.next().first;
+            // a piece may start inside a branch: its first step starts the accumulator too
+            const bool first = (sparse || ragged) ? (j == 0) : (it.next().first || j == 0);
             const uint32_t vit = item + 2 * j + 1;
             const uint32_t knext = item + 2 * j + 2;
             const bool has_next = j + 1 < nsteps;
@@ -680,6 +849,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     const uint32_t b_pfull = b_pfull0 + 8 * t, b_odone = b_odone0 + 8 * t;
     const float sl2 = p.scale_log2;
     uint32_t sf_cnt = 0, np = 0, ucnt = 0;
+    int piece_k = p.cta_piece0[blockIdx.x];
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
       const UnitInfo u = decode_unit(p, p.units[ui]);
@@ -692,7 +862,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       } else if (ragged) {
         ragged_range(p, u.s, rs, rl, false);
       }
-      const int nsteps = unit_steps(p, ctl->list_count[lb], rl);
+      PieceInfo pi;
+      const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
       const bool active = t < u.ntiles;
       int qrow = (u.tile0 + t) * 128 + r;
       if (sparse) {
@@ -704,9 +875,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       float m = -INFINITY, l = 0.f;            // running state of the current branch
       float m_prev = -INFINITY, l_prev = 0.f;  // state of the branch closed before it
       int cur_branch = -1, prev_branch = -1;
+      uint32_t touched = 0;  // branches this unit entry reached
       if (active && nsteps > 0) {
         TileIter it;
         it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
+        if (u.piece) it.seek(pi.j0);
         for (int j = 0; j < nsteps; ++j) {
           const TileDesc td = it.next();
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
@@ -725,7 +898,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           reg_fence<128>(sr);
           VKV_STAMP(tr < 0 ? -1 : tr + 2);
           bool pending_epi = false;
-          if (td.first) {
+          if (td.first || j == 0) {
             if (cur_branch >= 0) {
               pending_epi = true;
               prev_branch = cur_branch;
@@ -733,6 +906,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               l_prev = l;
             }
             cur_branch = td.branch;
+            touched |= 1u << td.branch;
             m = -INFINITY;
             l = 0.f;
           }
@@ -814,7 +988,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           // O_t += P_t(j-1) V_{j-1}, and a commit covers all earlier MMAs.
           const bool need_o = pending_epi || __any_sync(0xFFFFFFFFu, rescale);
           VKV_STAMP(tr < 0 ? -1 : tr + 4);
-          if (pending_epi) {
+          if (pending_epi && u.piece) {
+            piece_store<D>(p, pi, t, prev_branch, r, row_ok, tO, m_prev, l_prev);
+          } else if (pending_epi) {
             // close the previous branch: O / l and LSE
             const bool has = l_prev > 0.f;
             const float inv = has ? 1.f / l_prev : 0.f;
@@ -864,7 +1040,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ++np;
         }
         if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
-        if (ok) {
+        if (ok && u.piece) {
+          tc_fence_after();
+          piece_store<D>(p, pi, t, cur_branch, r, row_ok, tO, m, l);
+        } else if (ok) {
           tc_fence_after();
           // close the last branch, and merge with the one before it when asked
           const int lb = cur_branch;
@@ -924,7 +1103,24 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           }
         }
       }
-      if (ok && active && row_ok) {
+      if (u.piece && active && ok) {
+        // this piece's rows are in the workspace (LSE -inf for branches it did not
+        // reach); the last piece of the unit to arrive combines every piece
+        const int nbr = ragged ? 1 : p.n_branches;
+        if (row_ok)
+          for (int br = 0; br < nbr; ++br)
+            if (!((touched >> br) & 1u)) p.ws_l[piece_row(p, pi.slot0 + pi.idx, t, br, r)] = -INFINITY;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8 + t * 4 + quarter, 1) == pi.n - 1) ? 1 : 0;
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (last) {
+          __threadfence();
+          if (row_ok) piece_combine<D>(p, u, pi, t, r, qrow);
+        }
+      }
+      if (ok && active && row_ok && !u.piece) {
         // branches without any key tile: O = 0, LSE = -inf
         const int nb = (sparse || ragged) ? 1 : p.n_branches;
         for (int br = 0; br < nb; ++br) {

@@ -15,9 +15,17 @@ constexpr int kMaxCtas = 160;          // >= SMs of a B200 (148)
 constexpr int kMaxListEntries = 288;   // block list of one BLOCK_SPARSE unit
 constexpr int kCtlBytes = 2048;        // control block in shared memory
 constexpr int kMaxFlatSegs = VKV_MAX_BRANCHES * VKV_MAX_SEGMENTS;
+constexpr int kMaxPieces = 384;        // key-axis pieces per launch (kernel parameter space)
+constexpr int kMaxPiecesPerUnit = 8;   // pieces one split unit may be cut into
 
 // Kernel parameters of the attention kernel, passed as __grid_constant__.
-// Unit code: bits [0,13) first query tile, bit 13 two tiles, bits [14,32) sequence b*H+h.
+// Unit code: bits [0,12) first query tile, bit 12 piece (the unit covers only the
+// key steps of its piece entry), bit 13 two tiles, bits [14,32) sequence b*H+h.
+//
+// Piece entry (uint2): x = first step | end step << 16 (key-tile steps of the
+// unit's stream); y = first workspace slot of the unit | piece index << 16 |
+// piece count << 24.  The piece entries of CTA c are pieces[cta_piece0[c] ..],
+// in the order its unit list meets them.
 struct AttnParams {
   CUtensorMap tm_q;  // dims (d, H, Lq, B); box (64, 1, 128 or 64 (BLOCK_SPARSE), 1); 128 B swizzle
   CUtensorMap tm_k;  // dims (d, H, Lkv, B) or (d, 1, rows, 1); box (64, 1, 64, 1)
@@ -49,9 +57,17 @@ struct AttnParams {
   float* lsem;
   int* err;
   int withhold_first_copy;  // test aid: the producer skips its first K/V copy (see vkv_debug_withhold_copy)
+  // key-axis pieces: per workspace slot, the partial outputs (O / l, fp32)
+  // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (log2 units)
+  // [slot][tile][branch][row]; one arrival counter per (unit, tile, row quarter)
+  float* ws_o;
+  float* ws_l;
+  int* ws_cnt;  // [slot][8], zeroed before the launch; a unit uses its first slot's
   // schedule: CTA c runs units[cta_begin[c] .. cta_begin[c+1])
   int n_ctas;
   int cta_begin[kMaxCtas + 1];
+  int cta_piece0[kMaxCtas + 1];
+  uint2 pieces[kMaxPieces];
   uint32_t units[kMaxUnits];
 };
 

@@ -61,6 +61,7 @@ class vkv_attn_args(ctypes.Structure):
         ("o_merged", vkv_tensor), ("lse_merged", c_void_p),
         ("err_word", c_void_p),
         ("qblk_order", c_void_p),
+        ("workspace", c_void_p), ("workspace_bytes", c_size_t),
     ]
 
 
@@ -116,6 +117,14 @@ class vkv_latent_args(ctypes.Structure):
         ("lse", c_void_p), ("err_word", c_void_p),
     ]
 
+class vkv_schedule(ctypes.Structure):
+    _fields_ = [
+        ("n_ctas", c_int32), ("n_units", c_int32), ("n_pieces", c_int32), ("n_slots", c_int32),
+        ("cta_begin", POINTER(c_int32)), ("cta_piece0", POINTER(c_int32)),
+        ("units", POINTER(ctypes.c_uint32)), ("pieces", POINTER(ctypes.c_uint32)),
+    ]
+
+
 _lib = None
 
 
@@ -130,6 +139,10 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     L.vkv_chunk_attn.argtypes = [POINTER(vkv_attn_args), c_void_p]
     L.vkv_chunk_attn.restype = c_int32
+    L.vkv_chunk_attn_workspace_size.argtypes = [POINTER(vkv_attn_args)]
+    L.vkv_chunk_attn_workspace_size.restype = c_size_t
+    L.vkv_debug_schedule.argtypes = [POINTER(vkv_attn_args), c_int32, c_int32, POINTER(vkv_schedule)]
+    L.vkv_debug_schedule.restype = c_int32
     L.vkv_block_select.argtypes = [POINTER(vkv_select_args), c_void_p]
     L.vkv_block_select.restype = c_int32
     L.vkv_block_select_noalloc.argtypes = [POINTER(vkv_select_args), c_void_p]
@@ -178,6 +191,29 @@ def vkv_status_string(status: int) -> str:
 
 def vkv_chunk_attn(args: vkv_attn_args, stream: int | None) -> int:
     return int(lib().vkv_chunk_attn(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_chunk_attn_workspace_size(args: vkv_attn_args) -> int:
+    return int(lib().vkv_chunk_attn_workspace_size(ctypes.byref(args)))
+
+
+def vkv_debug_schedule(args: vkv_attn_args, n_sm: int, split: int, out: vkv_schedule) -> int:
+    return int(lib().vkv_debug_schedule(ctypes.byref(args), int(n_sm), int(split), ctypes.byref(out)))
+
+
+def attn_schedule(args: vkv_attn_args, n_sm: int, split: bool) -> dict:
+    """The work schedule of vkv_chunk_attn for these arguments on `n_sm` SMs (host only):
+    numpy arrays cta_begin, cta_piece0, units (uint32 codes), pieces ([n, 2] uint32) and n_slots."""
+    cb = np.zeros(n_sm + 1, np.int32)
+    cp = np.zeros(n_sm + 1, np.int32)
+    un = np.zeros(6144, np.uint32)
+    pc = np.zeros(2 * 384, np.uint32)
+    out = vkv_schedule(0, 0, 0, 0, cb.ctypes.data_as(POINTER(c_int32)), cp.ctypes.data_as(POINTER(c_int32)),
+                       un.ctypes.data_as(POINTER(ctypes.c_uint32)), pc.ctypes.data_as(POINTER(ctypes.c_uint32)))
+    _check(vkv_debug_schedule(args, n_sm, 1 if split else 0, out), "vkv_debug_schedule")
+    g = out.n_ctas
+    return {"cta_begin": cb[:g + 1].copy(), "cta_piece0": cp[:g + 1].copy(), "units": un[:out.n_units].copy(),
+            "pieces": pc[:2 * out.n_pieces].reshape(-1, 2).copy(), "n_slots": out.n_slots}
 
 
 def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
@@ -274,16 +310,45 @@ def _base_args(mode, q, Lkv, d, scale, k_desc, v_desc, err):
     return a
 
 
+_attn_ws: dict = {}  # (device index, stream handle) -> uint8 device buffer, grown on demand
+
+
+def _attn_workspace(a: vkv_attn_args, q: torch.Tensor, stream_handle: int, split: bool, workspace):
+    """Point the call at a key-axis split workspace: the caller's, or one kept per
+    (device, stream) by this module; none when split is False or the schedule
+    splits nothing.  Returns the buffer (kept alive by the caller until launch)."""
+    if workspace is not None:
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+        return workspace
+    if not split:
+        return None
+    need = vkv_chunk_attn_workspace_size(a)
+    if need == 0:
+        return None
+    key = (q.device.index, stream_handle)
+    buf = _attn_ws.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _attn_ws[key] = buf
+    a.workspace = buf.data_ptr()
+    a.workspace_bytes = buf.numel()
+    return buf
+
+
 def _new_out(q):
     B, Lq, H, d = q.shape
     return (torch.empty((B, Lq, H, d), dtype=torch.bfloat16, device=q.device),
             torch.empty((B, H, Lq), dtype=torch.float32, device=q.device))
 
 
-def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, stream=None, out=None):
+def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, stream=None, out=None,
+                        split=True, workspace=None):
     """Dual-branch (or single-branch) chunk attention over token segments.
 
     branches: list (length 1 or 2) of lists of (start, len) cache-row segments.
+    split: let the schedule cut units along the key axis (a workspace kept by this
+    module; `workspace`, a device uint8 tensor, overrides it).
     Returns dict(o=[...], lse=[...], o_merged, lse_merged).
     """
     nb = len(branches)
@@ -310,7 +375,9 @@ def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, st
     if res.get("o_merged") is not None:
         a.o_merged = tensor_desc(res["o_merged"])
         a.lse_merged = res["lse_merged"].data_ptr()
-    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    sh = _stream(stream)
+    ws = _attn_workspace(a, q, sh, split, workspace)  # noqa: F841 (alive until the launch)
+    _check(vkv_chunk_attn(a, sh), "vkv_chunk_attn")
     return res
 
 
@@ -342,8 +409,12 @@ def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_bl
 
 
 def chunk_attn_ragged(q, k_flat, v_flat, cu_seqlens, cu_seqlens_host=None, scale=None, err=None,
-                      stream=None, out=None):
-    """Ragged per-(batch, head) caches stored flattened with boundary offsets."""
+                      stream=None, out=None, split=True, workspace=None):
+    """Ragged per-(batch, head) caches stored flattened with boundary offsets.
+
+    With cu_seqlens_host the schedule knows each sequence's length and may cut
+    long sequences' units along the key axis (split / workspace as in
+    chunk_attn_segments)."""
     d = q.shape[3]
     a = _base_args(MODE_RAGGED, q, k_flat.shape[0], d, scale, flat_desc(k_flat), flat_desc(v_flat), err)
     a.cu_seqlens = cu_seqlens.data_ptr()
@@ -354,7 +425,9 @@ def chunk_attn_ragged(q, k_flat, v_flat, cu_seqlens, cu_seqlens_host=None, scale
     o, l = out if out is not None else _new_out(q)
     a.o[0] = tensor_desc(o)
     a.lse[0] = l.data_ptr()
-    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    sh = _stream(stream)
+    ws = _attn_workspace(a, q, sh, split, workspace)  # noqa: F841 (alive until the launch)
+    _check(vkv_chunk_attn(a, sh), "vkv_chunk_attn")
     return o, l
 
 
