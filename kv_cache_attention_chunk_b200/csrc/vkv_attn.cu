@@ -132,9 +132,12 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
   }
   const int g = n_sm;
   const double lb = std::max(tot / g, lb_piece);
-  const double slacks[] = {1.0, 1.01, 1.015, 1.02, 1.03, 1.05, 1.07, 1.1, 1.2, 1.4};
   double best = 1e300;
   using E = std::pair<double, int>;
+  // capacities from the lower bound up by 0.25 % steps to +10 %, then a few coarser ones
+  std::vector<double> slacks;
+  for (int i = 0; i <= 40; ++i) slacks.push_back(1.0 + 0.0025 * i);
+  for (double x : {1.15, 1.2, 1.3, 1.4}) slacks.push_back(x);
   for (double slack : slacks) {
     const double cap = lb * slack;
     std::priority_queue<Item, std::vector<Item>, decltype(cmp)> q(cmp, base);
@@ -151,7 +154,9 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
       const bool whole_unit = it.k == 0;
       int n = it.j1 - it.j0;
       if (e.first + it.cost > cap && it.k < kMaxPiecesPerUnit - 1 && it.S <= 0xFFFF) {
-        const int fit = (int)((cap - e.first) / it.rate - kPieceOverhead);
+        int fit = (int)((cap - e.first) / it.rate - kPieceOverhead);
+        // leave at least a minimum piece for the rest rather than overfilling this CTA
+        if (fit >= kMinPieceSteps && n - fit < kMinPieceSteps) fit = n - kMinPieceSteps;
         if (fit >= kMinPieceSteps && n - fit >= kMinPieceSteps) n = fit;
       }
       if (n == it.j1 - it.j0) {
