@@ -125,7 +125,25 @@ __global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
   const int s = blockIdx.x;
   const int n_cand = p.C + p.n_evict;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = 256 / 32;   // warps
+  constexpr int PB = 8;          // candidates a warp holds in registers at once
+  constexpr int PL = D / 32;     // columns per lane
   griddep_wait();  // both pooling grids before this one on the stream have completed
+  // candidate ids and validity into shared memory (independent loads, all at once)
+  for (int i = threadIdx.x; i < n_cand; i += 256) {
+    ids[i] = i < p.C ? __ldg(p.persist_idx + (size_t)s * p.C + i) : p.evict_blk0 + (i - p.C);
+    ok[i] = p.valid[(size_t)s * n_cand + i];
+  }
+  // the block means of this warp's first PB candidates (i = warp + NW * b), loaded
+  // now so that their latency overlaps the mean-query reduction below
+  float kreg[PB][PL];
+#pragma unroll
+  for (int b = 0; b < PB; ++b) {
+    const int i = warp + NW * b;
+    const float* kr = p.kbar + ((size_t)s * n_cand + (i < n_cand ? i : 0)) * D;
+#pragma unroll
+    for (int e = 0; e < PL; ++e) kreg[b][e] = (i < n_cand) ? __ldg(kr + lane + 32 * e) : 0.f;
+  }
   // mean query of the chunk: block means weighted by their rows (the last block may
   // be short).  Thread (g, c) sums chunk c of query blocks g, g + G, ... (independent
   // loads, several in flight), then the G partial sums are added in shared memory.
@@ -156,21 +174,29 @@ __global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
   }
   __syncthreads();
   // one warp per candidate: lane l takes columns l, l + 32, ... of the block mean
-  for (int i = warp; i < n_cand; i += blockDim.x >> 5) {
-    const bool valid = p.valid[(size_t)s * n_cand + i] != 0;
+  // (the first PB candidates of each warp from the registers loaded above)
+  for (int i = warp, b = 0; i < n_cand; i += NW, ++b) {
+    const bool valid = ok[i] != 0;
     float v = -INFINITY;
     if (valid) {
-      const float* kr = p.kbar + ((size_t)s * n_cand + i) * D;
       float a = 0.f;
+      if (b < PB) {
 #pragma unroll
-      for (int x = lane; x < D; x += 32) a = fmaf(qm[x], __ldg(kr + x), a);
+        for (int bb = 0; bb < PB; ++bb)
+          if (bb == b) {
+#pragma unroll
+            for (int e = 0; e < PL; ++e) a = fmaf(qm[lane + 32 * e], kreg[bb][e], a);
+          }
+      } else {
+        const float* kr = p.kbar + ((size_t)s * n_cand + i) * D;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) a = fmaf(qm[lane + 32 * e], __ldg(kr + lane + 32 * e), a);
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
       v = (a != a) ? -INFINITY : (a == 0.f ? 0.f : a);  // NaN ranks last; -0 ties with +0
     }
     if (lane == 0) {
-      ids[i] = i < p.C ? __ldg(p.persist_idx + (size_t)s * p.C + i) : p.evict_blk0 + (i - p.C);
-      ok[i] = valid ? 1 : 0;
       sc[i] = v;
       if (p.out_scores) p.out_scores[(size_t)s * n_cand + i] = valid ? v : -INFINITY;
     }
