@@ -161,15 +161,16 @@ typedef struct {
    * some query block unwritten (not checked). */
   const int32_t* qblk_order;
 
-  /* Optional DEVICE scratch for key-axis splitting (SEGMENTS and RAGGED with
-   * cu_seqlens_host).  NULL: every unit of work is one or two whole query tiles
+  /* Optional DEVICE scratch for key-axis splitting (SEGMENTS, BLOCK_SPARSE, and
+   * RAGGED with cu_seqlens_host).  NULL: every unit of work is one or two whole query tiles
    * over all of its keys, and the schedule balances whole units over the SMs.
    * Otherwise at least vkv_chunk_attn_workspace_size() bytes, 256-byte aligned,
    * owned by the caller (VKV_ERR_WORKSPACE when smaller): the schedule may then
    * cut some units into pieces over disjoint key ranges that run on different
    * SMs; each piece leaves its partial output and LSE in the workspace and the
    * last piece of a unit to finish combines them exactly (the same LSE merge as
-   * the two branches) and writes the outputs.  Results equal those of an
+   * the two branches) and writes the outputs.  (BLOCK_SPARSE units learn their
+   * key count on the device: their pieces are cut as fractions of it.)  Results equal those of an
    * unsplit run up to fp32 rounding.  Its contents need no initialisation (the
    * call clears its counters on `stream` first) and are dead after the call;
    * calls that overlap on the GPU must not share one. */
@@ -192,9 +193,10 @@ vkv_status vkv_chunk_attn(const vkv_attn_args* args, vkv_stream_t stream);
 
 /*
  * Bytes of `workspace` that vkv_chunk_attn can use for these arguments (0 when
- * its schedule does not split any unit; always 0 for BLOCK_SPARSE and for
- * RAGGED without cu_seqlens_host).  Reads only the host-side fields (mode,
- * shapes, segments, cu_seqlens_host); returns 0 for arguments that
+ * its schedule does not split any unit; always 0 for RAGGED without
+ * cu_seqlens_host).  Reads only the host-side fields (mode, shapes, segments,
+ * cu_seqlens_host, the block-sparse counts and whether qblk_order is NULL);
+ * returns 0 for arguments that
  * vkv_chunk_attn would refuse.  The size depends on the shapes and on the
  * number of SMs of the current device.
  */

@@ -88,10 +88,12 @@ inline uint32_t unit_code(int s, int tile0, bool two) {
 
 // Fixed cost of a unit (Q load, first product, epilogue) and of a piece (the
 // same plus its partial in the workspace and a share of the combine), in key
-// steps; pieces are at least kMinPieceSteps long.
+// steps; pieces are at least kMinPieceSteps long (kMinPieceStepsSparse for the
+// short units of BLOCK_SPARSE).
 constexpr double kUnitOverhead = 2.0;
 constexpr double kPieceOverhead = 4.0;
 constexpr int kMinPieceSteps = 16;
+constexpr int kMinPieceStepsSparse = 24;
 
 // Schedule with key-axis pieces: longest-first onto the least loaded CTA, as for
 // whole units, but against a capacity T = slack * (total cost / CTAs).  A unit
@@ -100,7 +102,8 @@ constexpr int kMinPieceSteps = 16;
 // as an item of its own (cut again if needed, at most kMaxPiecesPerUnit pieces).
 // The best of a few slacks is kept.  steps[s] is the key-step count of sequence s.
 bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
-                const std::vector<int>& steps, int n_sm, Plan* out, double* mk_out) {
+                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm, Plan* out,
+                double* mk_out) {
   struct Item {
     double cost;
     uint32_t code;
@@ -119,7 +122,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
     for (int i = 0; i < T / 2; ++i)
       base.push_back({pair_cost[s], unit_code(s, 2 * i, true), steps[s], 0, steps[s], 1.0, 0, 0});
     if (T & 1)
-      base.push_back({one_cost[s], unit_code(s, T - 1, false), steps[s], 0, steps[s], 0.0, 0, 0});
+      base.push_back({one_cost[s], unit_code(s, T - 1, false), steps1[s], 0, steps1[s], 0.0, 0, 0});
   }
   if (base.empty() || (long long)base.size() > kMaxUnits) return false;
   double tot = 0, lb_piece = 0;
@@ -128,7 +131,8 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
     base[i].rate = base[i].cost / (base[i].S + kUnitOverhead);
     tot += base[i].cost;
     // no CTA can finish before a unit cut into the most pieces allowed
-    lb_piece = std::max(lb_piece, base[i].rate * ((double)base[i].S / kMaxPiecesPerUnit + kPieceOverhead));
+    const int most = std::max(1, std::min(kMaxPiecesPerUnit, base[i].S / min_steps));
+    lb_piece = std::max(lb_piece, base[i].rate * ((double)base[i].S / most + kPieceOverhead));
   }
   const int g = n_sm;
   const double lb = std::max(tot / g, lb_piece);
@@ -156,8 +160,8 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
       if (e.first + it.cost > cap && it.k < kMaxPiecesPerUnit - 1 && it.S <= 0xFFFF) {
         int fit = (int)((cap - e.first) / it.rate - kPieceOverhead);
         // leave at least a minimum piece for the rest rather than overfilling this CTA
-        if (fit >= kMinPieceSteps && n - fit < kMinPieceSteps) fit = n - kMinPieceSteps;
-        if (fit >= kMinPieceSteps && n - fit >= kMinPieceSteps) n = fit;
+        if (fit >= min_steps && n - fit < min_steps) fit = n - min_steps;
+        if (fit >= min_steps && n - fit >= min_steps) n = fit;
       }
       if (n == it.j1 - it.j0) {
         // the rest of the unit in one go
@@ -232,10 +236,12 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
 }
 
 // pair_cost[s] / single_cost[s]: estimated cost of a 2-tile / 1-tile unit of sequence s.
-// steps (empty: unknown) gives each sequence's key steps; with it the schedule
-// may split units along the key axis when that shortens it by 3 % or more.
-bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
-               const std::vector<double>& one_cost, const std::vector<int>& steps, int n_sm, Plan* plan) {
+// steps / steps1 (empty: unknown) give the key steps of sequence s's 2-tile /
+// 1-tile units; with them the schedule may split units along the key axis,
+// into pieces of at least min_steps, when that shortens it by 3 % or more.
+bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
+               const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
+               Plan* plan) {
   // sequences by decreasing pair cost: their pairs are split first
   std::vector<int> order(n_seq);
   for (int s = 0; s < n_seq; ++s) order[s] = s;
@@ -286,7 +292,8 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost,
     Plan sp;
     double mk_split = 1e300;
     // the whole-unit makespan in the same cost terms (a split plan always uses n_sm CTAs)
-    if (split_plan(n_seq, T, pair_cost, one_cost, steps, n_sm, &sp, &mk_split) && mk_split < 0.97 * best) {
+    if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, &sp, &mk_split) &&
+        mk_split < 0.97 * best) {
       *plan = std::move(sp);
       return true;
     }
@@ -302,14 +309,15 @@ std::mutex g_plan_mu;
 std::map<std::string, std::shared_ptr<Plan>> g_plans;
 
 std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const std::vector<double>& pc,
-                               const std::vector<double>& oc, const std::vector<int>& steps, int n_sm) {
+                               const std::vector<double>& oc, const std::vector<int>& steps,
+                               const std::vector<int>& steps1, int min_steps, int n_sm) {
   {
     std::lock_guard<std::mutex> lk(g_plan_mu);
     auto it = g_plans.find(key);
     if (it != g_plans.end()) return it->second;
   }
   auto plan = std::make_shared<Plan>();
-  if (!make_plan(n_seq, T, pc, oc, steps, n_sm, plan.get())) return nullptr;
+  if (!make_plan(n_seq, T, pc, oc, steps, steps1, min_steps, n_sm, plan.get())) return nullptr;
   std::lock_guard<std::mutex> lk(g_plan_mu);
   if (g_plans.size() > 256) g_plans.clear();
   g_plans[key] = plan;
@@ -424,7 +432,8 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
 
   int nb = 1;
   std::vector<double> pc(n_seq), oc(n_seq);
-  std::vector<int> steps;  // per sequence, when the schedule may split units
+  std::vector<int> steps, steps1;  // key steps of 2-tile / 1-tile units, when units may be split
+  int min_steps = kMinPieceSteps;
   const double c1 = single_tile_cost();
   std::string key;
   if (mode == VKV_MODE_SEGMENTS) {
@@ -496,6 +505,14 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
       pc[s] = sp;
       oc[s] = c1 * s1;
     }
+    // pieces are cut in these estimated steps and scaled on the device to the
+    // unit's real step count
+    P->sp_est[0] = (int)std::ceil((a->n_persist + u2) * 0.5);
+    P->sp_est[1] = (int)std::ceil((a->n_persist + u4) * 0.5);
+    if (want_split) {
+      steps.assign(n_seq, P->sp_est[1]);
+      steps1.assign(n_seq, P->sp_est[0]);
+    }
     key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
           std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n");
   } else {
@@ -552,7 +569,9 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
   if (n_sm <= 0) return VKV_ERR_CUDA;
   const int g_max = std::min(n_sm, kMaxCtas);
   key += "@" + std::to_string(g_max) + ":" + std::to_string(c1) + (steps.empty() ? "" : "/split");
-  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, g_max);
+  if (mode == VKV_MODE_BLOCK_SPARSE) min_steps = kMinPieceStepsSparse;
+  if (steps1.empty()) steps1 = steps;
+  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, steps1, min_steps, g_max);
   if (!plan) return VKV_ERR_UNSUPPORTED;
   P->n_ctas = plan->n_ctas;
   std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);
@@ -570,12 +589,12 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
 using namespace vkv;
 
 extern "C" size_t vkv_chunk_attn_workspace_size(const vkv_attn_args* a) {
-  if (!a || (a->mode != VKV_MODE_SEGMENTS && a->mode != VKV_MODE_RAGGED)) return 0;
+  if (!a) return 0;
   auto P = std::make_unique<AttnParams>();
   std::shared_ptr<Plan> plan;
   int dev = 0;
   if (attn_setup(a, false, true, P.get(), &plan, &dev) != VKV_OK) return 0;
-  const int nbr = a->mode == VKV_MODE_RAGGED ? 1 : a->n_branches;
+  const int nbr = a->mode == VKV_MODE_SEGMENTS ? a->n_branches : 1;
   return ws_layout(plan->n_slots, nbr, a->d).bytes;
 }
 
@@ -585,8 +604,7 @@ extern "C" vkv_status vkv_debug_schedule(const vkv_attn_args* a, int32_t n_sm, i
   auto P = std::make_unique<AttnParams>();
   std::shared_ptr<Plan> plan;
   int dev = 0;
-  const vkv_status stt =
-      attn_setup(a, false, split != 0 && a->mode != VKV_MODE_BLOCK_SPARSE, P.get(), &plan, &dev, n_sm);
+  const vkv_status stt = attn_setup(a, false, split != 0, P.get(), &plan, &dev, n_sm);
   if (stt != VKV_OK) return stt;
   out->n_ctas = plan->n_ctas;
   out->n_units = (int32_t)plan->units.size();
@@ -605,7 +623,7 @@ extern "C" vkv_status vkv_debug_schedule(const vkv_attn_args* a, int32_t n_sm, i
 
 extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream) {
   if (!a) return VKV_ERR_NULL;
-  const bool want_split = a->workspace != nullptr && a->mode != VKV_MODE_BLOCK_SPARSE;
+  const bool want_split = a->workspace != nullptr;
   auto P = std::make_unique<AttnParams>();
   std::shared_ptr<Plan> plan;
   int dev = 0;
@@ -615,7 +633,7 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   const int mode = a->mode, B = a->B, H = a->H, Lq = a->Lq, Lkv = a->Lkv, d = a->d;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (plan->n_slots > 0) {
-    const int nbr = mode == VKV_MODE_RAGGED ? 1 : a->n_branches;
+    const int nbr = mode == VKV_MODE_SEGMENTS ? a->n_branches : 1;
     const WsLayout w = ws_layout(plan->n_slots, nbr, d);
     if (a->workspace_bytes < w.bytes) return VKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(a->workspace) & 255) return VKV_ERR_ALIGN;

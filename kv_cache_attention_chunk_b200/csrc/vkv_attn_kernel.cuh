@@ -191,11 +191,13 @@ __device__ __forceinline__ PieceInfo piece_info(const AttnParams& p, int k) {
 }
 
 // Steps of this unit entry: all `full` steps of the unit's stream, or the part
-// [j0, j1) of a piece.  RAGGED lengths are read on the device and may differ
-// from the host copy the pieces were cut from: the range is clamped to `full`,
-// and the unit's last piece runs to `full`, so the pieces always cover the
-// device's key range.  Advances the CTA's piece cursor; every role walks the
-// same unit list.
+// [j0, j1) of a piece (pi.j0 is set to the entry's first step).  RAGGED
+// lengths are read on the device and may differ from the host copy the pieces
+// were cut from: the range is clamped to `full`, and the unit's last piece
+// runs to `full`, so the pieces always cover the device's key range.  A
+// BLOCK_SPARSE unit's step count is known only on the device: its pieces were
+// cut from the host's estimate sp_est[ntiles - 1] and are scaled to `full`.
+// Advances the CTA's piece cursor; every role walks the same unit list.
 __device__ __forceinline__ int entry_steps(const AttnParams& p, const UnitInfo& u, int full, int& piece_k,
                                            PieceInfo& pi) {
   if (!u.piece) {
@@ -204,7 +206,14 @@ __device__ __forceinline__ int entry_steps(const AttnParams& p, const UnitInfo& 
     return full;
   }
   pi = piece_info(p, piece_k++);
-  const int j1 = (pi.idx == pi.n - 1) ? full : min(pi.j1, full);
+  const bool last = pi.idx == pi.n - 1;
+  if (p.mode == VKV_MODE_BLOCK_SPARSE) {
+    const int est = max(1, p.sp_est[u.ntiles - 1]);
+    pi.j0 = (int)(((long long)pi.j0 * full) / est);
+    pi.j1 = last ? full : (int)(((long long)pi.j1 * full) / est);
+    return max(0, min(pi.j1, full) - pi.j0);
+  }
+  const int j1 = last ? full : min(pi.j1, full);
   return max(0, j1 - pi.j0);
 }
 
@@ -442,12 +451,16 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float&
 
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Output branches of a launch: SEGMENTS has n_branches, the other modes one.
+__device__ __forceinline__ int out_branches(const AttnParams& p) {
+  return p.mode == VKV_MODE_SEGMENTS ? p.n_branches : 1;
+}
+
 // Key-axis pieces.  A piece of a split unit leaves, per branch it reached, O / l
 // (fp32) and its LSE (log2 units) in its workspace slot; the last piece of the
 // unit to arrive combines them (the LSE merge, the same as between branches).
 __device__ __forceinline__ size_t piece_row(const AttnParams& p, int slot, int t, int br, int r) {
-  const int nbr = p.mode == VKV_MODE_RAGGED ? 1 : p.n_branches;
-  return ((size_t)(slot * 2 + t) * nbr + br) * 128 + r;
+  return ((size_t)(slot * 2 + t) * out_branches(p) + br) * 128 + r;
 }
 
 // One branch of this piece: O from TMEM divided by l, and m + log2 l.  All
@@ -482,8 +495,7 @@ __device__ __forceinline__ void piece_store(const AttnParams& p, const PieceInfo
 template <int D>
 __device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
                                               int r, int qrow) {
-  const bool ragged = p.mode == VKV_MODE_RAGGED;
-  const int nbr = ragged ? 1 : p.n_branches;
+  const int nbr = out_branches(p);
   const bool do_merge = p.om != nullptr && nbr == 2;
   float w[2][kMaxPiecesPerUnit];
   float L[2] = {-INFINITY, -INFINITY};
@@ -1106,7 +1118,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       if (u.piece && active && ok) {
         // this piece's rows are in the workspace (LSE -inf for branches it did not
         // reach); the last piece of the unit to arrive combines every piece
-        const int nbr = ragged ? 1 : p.n_branches;
+        const int nbr = out_branches(p);
         if (row_ok)
           for (int br = 0; br < nbr; ++br)
             if (!((touched >> br) & 1u)) p.ws_l[piece_row(p, pi.slot0 + pi.idx, t, br, r)] = -INFINITY;

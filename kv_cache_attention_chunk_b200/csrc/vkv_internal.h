@@ -60,6 +60,7 @@ struct AttnParams {
   // key-axis pieces: per workspace slot, the partial outputs (O / l, fp32)
   // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (log2 units)
   // [slot][tile][branch][row]; one arrival counter per (unit, tile, row quarter)
+  int sp_est[2];  // BLOCK_SPARSE: key steps the schedule assumed for a 1- / 2-tile unit
   float* ws_o;
   float* ws_l;
   int* ws_cnt;  // [slot][8], zeroed before the launch; a unit uses its first slot's

@@ -382,11 +382,12 @@ def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, st
 
 
 def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_blk, scale=None,
-                            err=None, stream=None, out=None, qblk_order=None):
+                            err=None, stream=None, out=None, qblk_order=None, split=True, workspace=None):
     """Persistent blocks + selected window blocks (device int32 index tensors).
 
     qblk_order (optional device int32 [B*H, nQblk]): query-block permutation that
     groups blocks with similar selections into the same units (from block_select).
+    split / workspace: key-axis pieces, as in chunk_attn_segments.
     """
     d = q.shape[3]
     a = _base_args(MODE_BLOCK_SPARSE, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
@@ -404,7 +405,9 @@ def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_bl
     o, l = out if out is not None else _new_out(q)
     a.o[0] = tensor_desc(o)
     a.lse[0] = l.data_ptr()
-    _check(vkv_chunk_attn(a, _stream(stream)), "vkv_chunk_attn")
+    sh = _stream(stream)
+    ws = _attn_workspace(a, q, sh, split, workspace)  # noqa: F841 (alive until the launch)
+    _check(vkv_chunk_attn(a, sh), "vkv_chunk_attn")
     return o, l
 
 

@@ -171,3 +171,47 @@ def test_workspace_too_small_is_refused():
     with pytest.raises(v.VkvError) as e:
         v.chunk_attn_segments(c.q.to(DEV), c.k.to(DEV), c.v.to(DEV), c.branches, scale=c.scale, workspace=small)
     assert e.value.status == 7  # VKV_ERR_WORKSPACE
+
+
+def _sparse_schedule(c, topk, grouped):
+    v = vk()
+    a = v.vkv_attn_args()
+    a.mode = v.MODE_BLOCK_SPARSE
+    a.B, a.H, a.Lq, a.Lkv, a.d = c.B, c.H, c.q.shape[1], c.k.shape[1], c.d
+    a.scale = c.scale
+    a.block = 64
+    a.n_persist = c.persist_idx.shape[1]
+    a.topk = topk
+    a.window_blk0, a.n_win_blk = c.window_blk0, c.n_win_blk
+    a.qblk_order = 1 if grouped else None  # only NULL or not matters to the schedule
+    return v.attn_schedule(a, n_sm(), True)
+
+
+@pytest.mark.parametrize("topk,grouped", [(16, False), (6, True), (40, False)])
+def test_split_block_sparse_matches_oracle(topk, grouped):
+    """Block-sparse units learn their key count on the device; their pieces are cut
+    as fractions of it.  Long persistent lists make every unit long enough to cut."""
+    v = vk()
+    c = W.make_block_sparse("sp", seed=90 + topk, H=2, d=128, frame_tokens=256, block=64, hist_frames=40,
+                            win_frames=12, q_frames=1, n_persist=120)
+    assert len(_sparse_schedule(c, topk, grouped)["pieces"]) > 0, "the schedule was expected to split"
+    q, k, vv = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    order = None
+    if grouped:
+        idx, _, order = v.block_select(q, k, c.window_blk0, c.n_win_blk, topk, order=True)
+        sel = idx.cpu().numpy()
+    else:
+        sel = W.random_selection(7 + topk, c.B * c.H, c.n_qblk, c.n_win_blk, topk)
+        idx = torch.from_numpy(sel).to(DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, l = v.chunk_attn_block_sparse(q, k, vv, torch.from_numpy(c.persist_idx).to(DEV), idx, c.window_blk0,
+                                     c.n_win_blk, scale=c.scale, err=err, qblk_order=order)
+    o2, l2 = v.chunk_attn_block_sparse(q, k, vv, torch.from_numpy(c.persist_idx).to(DEV), idx, c.window_blk0,
+                                       c.n_win_blk, scale=c.scale, err=err, qblk_order=order, split=False)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel, c.window_blk0, c.block, c.scale)
+    assert_bf16_close(o, ro, "split sparse O")
+    assert_lse_close(l, rl, "split sparse LSE")
+    assert (o.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (l - l2).abs().max().item() <= 1e-4

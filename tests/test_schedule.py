@@ -77,20 +77,21 @@ def _check_cover(sch, n_seq, T, steps, n_sm):
             tiles = (tile0, tile0 + 1) if two else (tile0,)
             assert tile0 + len(tiles) <= T and s < n_seq
             rate = 1.0 if two else C1
+            S = steps(s, two) if callable(steps) else steps[s]
             if code & PIECE:
                 x, y = (int(v) for v in pieces[k])
                 k += 1
                 j0, j1 = x & 0xFFFF, x >> 16
                 slot0, idx, n = y & 0xFFFF, (y >> 16) & 0xFF, y >> 24
-                assert 2 <= n <= 8 and idx < n and 0 <= j0 < j1 <= steps[s]
+                assert 2 <= n <= 8 and idx < n and 0 <= j0 < j1 <= S
                 assert slot0 + idx < sch["n_slots"] and (slot0 + idx) not in slots
                 slots.add(slot0 + idx)
-                seen.setdefault((s, tiles), []).append((j0, j1, slot0, idx, n))
+                seen.setdefault((s, tiles), []).append((j0, j1, slot0, idx, n, S))
                 load[c] += rate * (j1 - j0 + 4.0)
             else:
                 assert (s, tiles) not in seen
                 seen[(s, tiles)] = "whole"
-                load[c] += rate * (steps[s] + 2.0)
+                load[c] += rate * (S + 2.0)
         assert k == cp[c + 1]
     # every query tile of every sequence exactly once
     covered = {}
@@ -102,7 +103,7 @@ def _check_cover(sch, n_seq, T, steps, n_sm):
             v = sorted(v)
             assert len({p[2] for p in v}) == 1 and sorted(p[3] for p in v) == list(range(v[0][4]))
             assert len(v) == v[0][4]
-            assert v[0][0] == 0 and v[-1][1] == steps[s]
+            assert v[0][0] == 0 and v[-1][1] == v[0][5]
             for a, b in zip(v, v[1:]):
                 assert a[1] == b[0]
     assert len(covered) == n_seq * T
@@ -172,3 +173,40 @@ def test_workspace_size_needs_no_device_but_a_device_count():
     import torch
     if not torch.cuda.is_available():
         assert vkv.vkv_chunk_attn_workspace_size(a) == 0
+
+
+@pytest.mark.parametrize("topk,grouped", [(72, True), (144, True), (48, False)])
+def test_block_sparse_split_schedule_covers_and_balances(topk, grouped):
+    """Block-sparse pieces are cut in the schedule's estimated key steps of a unit
+    (persistent blocks plus the expected union of its query blocks' selections,
+    two blocks per step) and scaled on the device to the real count."""
+    a = vkv.vkv_attn_args()
+    a.mode = vkv.MODE_BLOCK_SPARSE
+    a.B, a.H, a.Lq, a.Lkv, a.d = 1, 12, 4608, 36 * 1536, 128
+    a.scale, a.block, a.n_persist, a.topk = 0.088, 64, 32, topk
+    a.window_blk0, a.n_win_blk = 30 * 1536 // 64, 144
+    a.qblk_order = 1 if grouped else None  # only NULL or not matters to the schedule
+    u4 = min(144, (1.5 if grouped else 4.0) * topk)
+    u2 = min(144, (1.25 if grouped else 2.0) * topk)
+    S2, S1 = int(np.ceil((32 + u4) / 2)), int(np.ceil((32 + u2) / 2))
+    steps = lambda s, two: S2 if two else S1  # noqa: E731
+    whole = vkv.attn_schedule(a, 148, False)
+    lw = _check_cover(whole, 12, 36, steps, 148)
+    sp = vkv.attn_schedule(a, 148, True)
+    assert len(sp["pieces"]) > 0
+    ls = _check_cover(sp, 12, 36, steps, 148)
+    ideal = 216 * (S2 + 2.0) / 148
+    assert ls.max() <= 0.97 * lw.max() and ls.max() <= 1.15 * ideal
+
+
+@pytest.mark.parametrize("topk", [9, 18, 36])
+def test_short_block_sparse_units_are_not_split(topk):
+    """Units of fewer than 48 estimated key steps stay whole (their real key counts
+    vary with the selections, and a piece's fixed cost weighs too much on them)."""
+    a = vkv.vkv_attn_args()
+    a.mode = vkv.MODE_BLOCK_SPARSE
+    a.B, a.H, a.Lq, a.Lkv, a.d = 1, 12, 4608, 36 * 1536, 128
+    a.scale, a.block, a.n_persist, a.topk = 0.088, 64, 32, topk
+    a.window_blk0, a.n_win_blk = 30 * 1536 // 64, 144
+    a.qblk_order = 1
+    assert len(vkv.attn_schedule(a, 148, True)["pieces"]) == 0
