@@ -7,8 +7,9 @@ units over long caches, so the schedule is forced to split (checked through
 the host-side schedule for this device's SM count), and cover: pieces that
 start inside a branch and pieces that span the branch boundary, single-tile
 units and a ragged last query tile, d = 64 and 128, ragged caches, a device
-length table that differs from the host copy the pieces were cut from, and
-equality with the unsplit schedule up to rounding.
+length table that differs from the host copy the pieces were cut from,
+block-sparse units (whose pieces are fractions of a key count known only on
+the device), and equality with the unsplit schedule up to rounding.
 """
 import ctypes
 
