@@ -566,6 +566,8 @@ def run_ours(args):
                      "frac": achieved / peak, "traffic": recorded_traffic(),
                      "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": "chunk_attn_kernel<128>",
                      "launch_ms_median": statistics.median(launch_ms),
+                     "launch_ms_p10": float(np.percentile(launch_ms, 10)),
+                     "launch_ms_p90": float(np.percentile(launch_ms, 90)),
                      # the timed steps run back to back for about a second under the power cap,
                      # the regime of the sustained GEMM figure; reported beside the burst fraction
                      "peak_sustained": peak_sus, "frac_of_sustained": achieved / peak_sus if peak_sus else None},
