@@ -466,9 +466,9 @@ __device__ __forceinline__ size_t piece_row(const AttnParams& p, int slot, int t
 // One branch of this piece: O from TMEM divided by l, and m + log2 l.  All
 // lanes of the warp take part (tcgen05.ld); rows past Lq store nothing.
 template <int D>
-__device__ __forceinline__ void piece_store(const AttnParams& p, const PieceInfo& pi, int t, int br, int r,
-                                            bool row_ok, uint32_t tO, float m, float l) {
-  const size_t row = piece_row(p, pi.slot0 + pi.idx, t, br, r);
+__device__ __forceinline__ void piece_store(const AttnParams& p, int slot, int t, int br, int r, bool row_ok,
+                                            uint32_t tO, float m, float l) {
+  const size_t row = piece_row(p, slot, t, br, r);
   const bool has = l > 0.f;
   const float inv = has ? 1.f / l : 0.f;
   float* dst = p.ws_o + row * D;
@@ -487,6 +487,26 @@ __device__ __forceinline__ void piece_store(const AttnParams& p, const PieceInfo
     }
   }
   if (row_ok) p.ws_l[row] = has ? m + lg2_approx(l) : -INFINITY;
+}
+
+// Workspace slot of piece entry k.
+__device__ __forceinline__ int piece_slot(const AttnParams& p, int k) {
+  const uint32_t y = p.pieces[k].y;
+  return (int)(y & 0xFFFFu) + (int)((y >> 16) & 0xFFu);
+}
+
+// Branches that key steps [j0, j0 + n) of a unit's stream reach (bit b = branch b).
+__device__ __forceinline__ uint32_t branches_reached(const AttnParams& p, int j0, int n) {
+  if (n <= 0) return 0u;
+  if (p.mode != VKV_MODE_SEGMENTS) return 1u;
+  uint32_t m = 0u;
+  int b0 = 0;
+  for (int br = 0; br < p.n_branches; ++br) {
+    const int b1 = b0 + p.branch_steps[br];
+    if (b1 > b0 && j0 < b1 && j0 + n > b0) m |= 1u << br;
+    b0 = b1;
+  }
+  return m;
 }
 
 // Row r of tile t of a split unit from all of its pieces: per branch
@@ -874,8 +894,16 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       } else if (ragged) {
         ragged_range(p, u.s, rs, rl, false);
       }
-      PieceInfo pi;
-      const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
+      // the piece entry's index (its details are re-read from the parameters where
+      // needed, so that the step loop keeps no more state live than a whole unit)
+      const int pk = u.piece ? piece_k : -1;
+      int j0;
+      int nsteps;
+      {
+        PieceInfo pi;
+        nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
+        j0 = pi.j0;
+      }
       const bool active = t < u.ntiles;
       int qrow = (u.tile0 + t) * 128 + r;
       if (sparse) {
@@ -887,11 +915,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       float m = -INFINITY, l = 0.f;            // running state of the current branch
       float m_prev = -INFINITY, l_prev = 0.f;  // state of the branch closed before it
       int cur_branch = -1, prev_branch = -1;
-      uint32_t touched = 0;  // branches this unit entry reached
       if (active && nsteps > 0) {
         TileIter it;
         it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
-        if (u.piece) it.seek(pi.j0);
+        if (u.piece) it.seek(j0);
         for (int j = 0; j < nsteps; ++j) {
           const TileDesc td = it.next();
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
@@ -918,7 +945,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               l_prev = l;
             }
             cur_branch = td.branch;
-            touched |= 1u << td.branch;
             m = -INFINITY;
             l = 0.f;
           }
@@ -1001,7 +1027,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           const bool need_o = pending_epi || __any_sync(0xFFFFFFFFu, rescale);
           VKV_STAMP(tr < 0 ? -1 : tr + 4);
           if (pending_epi && u.piece) {
-            piece_store<D>(p, pi, t, prev_branch, r, row_ok, tO, m_prev, l_prev);
+            piece_store<D>(p, piece_slot(p, pk), t, prev_branch, r, row_ok, tO, m_prev, l_prev);
           } else if (pending_epi) {
             // close the previous branch: O / l and LSE
             const bool has = l_prev > 0.f;
@@ -1054,7 +1080,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
         if (ok && u.piece) {
           tc_fence_after();
-          piece_store<D>(p, pi, t, cur_branch, r, row_ok, tO, m, l);
+          piece_store<D>(p, piece_slot(p, pk), t, cur_branch, r, row_ok, tO, m, l);
         } else if (ok) {
           tc_fence_after();
           // close the last branch, and merge with the one before it when asked
@@ -1118,7 +1144,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       if (u.piece && active && ok) {
         // this piece's rows are in the workspace (LSE -inf for branches it did not
         // reach); the last piece of the unit to arrive combines every piece
+        const PieceInfo pi = piece_info(p, pk);
         const int nbr = out_branches(p);
+        const uint32_t touched = branches_reached(p, j0, nsteps);
         if (row_ok)
           for (int br = 0; br < nbr; ++br)
             if (!((touched >> br) & 1u)) p.ws_l[piece_row(p, pi.slot0 + pi.idx, t, br, r)] = -INFINITY;
