@@ -94,6 +94,7 @@ constexpr double kUnitOverhead = 2.0;
 constexpr double kPieceOverhead = 4.0;
 constexpr int kMinPieceSteps = 16;
 constexpr int kMinPieceStepsSparse = 24;
+constexpr double kSplitGain = 0.88;  // a split schedule is used below this makespan ratio
 
 // Schedule with key-axis pieces: longest-first onto the least loaded CTA, as for
 // whole units, but against a capacity T = slack * (total cost / CTAs).  A unit
@@ -238,7 +239,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
 // pair_cost[s] / single_cost[s]: estimated cost of a 2-tile / 1-tile unit of sequence s.
 // steps / steps1 (empty: unknown) give the key steps of sequence s's 2-tile /
 // 1-tile units; with them the schedule may split units along the key axis,
-// into pieces of at least min_steps, when that shortens it by 3 % or more.
+// into pieces of at least min_steps, when that shortens it by 12 % or more.
 bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
                Plan* plan) {
@@ -292,8 +293,11 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std
     Plan sp;
     double mk_split = 1e300;
     // the whole-unit makespan in the same cost terms (a split plan always uses n_sm CTAs)
+    // the instantiation with piece support runs the step loop ~10 % slower (its
+    // cold piece paths change the loop's register allocation), so a split schedule
+    // must model a larger gain than that
     if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, &sp, &mk_split) &&
-        mk_split < 0.97 * best) {
+        mk_split < kSplitGain * best) {
       *plan = std::move(sp);
       return true;
     }
@@ -324,28 +328,38 @@ std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const s
   return plan;
 }
 
-bool set_smem_attr(int dev, int D, bool sparse) {
+template <int D, bool SP, bool PC>
+bool set_smem_attr_t(int dev) {
   static std::mutex mu;
-  static unsigned long long done[4] = {0, 0, 0, 0};
+  static unsigned long long done = 0;
   std::lock_guard<std::mutex> lk(mu);
-  const int k = ((D == 128) ? 0 : 1) + (sparse ? 2 : 0);
-  if (done[k] & (1ull << dev)) return true;
-  const void* fn =
-      (D == 128) ? (sparse ? reinterpret_cast<const void*>(chunk_attn_kernel<128, true>)
-                           : reinterpret_cast<const void*>(chunk_attn_kernel<128, false>))
-                 : (sparse ? reinterpret_cast<const void*>(chunk_attn_kernel<64, true>)
-                           : reinterpret_cast<const void*>(chunk_attn_kernel<64, false>));
-  const int smem = (D == 128) ? AttnCfg<128>::SMEM_BYTES : AttnCfg<64>::SMEM_BYTES;
+  if (done & (1ull << dev)) return true;
+  const void* fn = reinterpret_cast<const void*>(chunk_attn_kernel<D, SP, PC>);
   cudaFuncAttributes fa;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM_BYTES) !=
+          cudaSuccess ||
       cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
   // the warpgroup register split needs every register the launch provides
   if (fa.numRegs < kRegsLaunchNeeded) return false;
-  done[k] |= 1ull << dev;
+  done |= 1ull << dev;
   return true;
+}
+
+// Sets the shared-memory size of the instantiation and launches it.
+template <int D, bool SP, bool PC>
+vkv_status launch_attn_t(int dev, const AttnParams& P, cudaStream_t st) {
+  if (!set_smem_attr_t<D, SP, PC>(dev)) return VKV_ERR_CUDA;
+  chunk_attn_kernel<D, SP, PC><<<P.n_ctas, 384, AttnCfg<D>::SMEM_BYTES, st>>>(P);
+  return cudaGetLastError() == cudaSuccess ? VKV_OK : VKV_ERR_CUDA;
+}
+
+template <int D>
+vkv_status launch_attn_d(int dev, bool sp, bool pc, const AttnParams& P, cudaStream_t st) {
+  if (sp) return pc ? launch_attn_t<D, true, true>(dev, P, st) : launch_attn_t<D, true, false>(dev, P, st);
+  return pc ? launch_attn_t<D, false, true>(dev, P, st) : launch_attn_t<D, false, false>(dev, P, st);
 }
 
 bool dims_ok_for_tma(const vkv_tensor& t, int B, int L, int H, int d) {
@@ -654,20 +668,8 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
       return VKV_ERR_CUDA;
   }
   const bool sp = mode == VKV_MODE_BLOCK_SPARSE;
-  if (!set_smem_attr(dev, d, sp)) return VKV_ERR_CUDA;
-  if (d == 128) {
-    if (sp)
-      chunk_attn_kernel<128, true><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
-    else
-      chunk_attn_kernel<128, false><<<P->n_ctas, 384, AttnCfg<128>::SMEM_BYTES, st>>>(*P);
-  } else {
-    if (sp)
-      chunk_attn_kernel<64, true><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
-    else
-      chunk_attn_kernel<64, false><<<P->n_ctas, 384, AttnCfg<64>::SMEM_BYTES, st>>>(*P);
-  }
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
-  return VKV_OK;
+  const bool pc = plan->n_slots > 0;
+  return d == 128 ? launch_attn_d<128>(dev, sp, pc, *P, st) : launch_attn_d<64>(dev, sp, pc, *P, st);
 }
 
 #ifdef VKV_TRACE

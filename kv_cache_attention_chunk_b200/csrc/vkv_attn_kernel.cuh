@@ -228,6 +228,15 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, uint32_t co
   return u;
 }
 
+// A unit entry as the kernel instantiation sees it: without piece support (PC
+// false) no entry is a piece, and every piece path folds away at compile time.
+template <bool PC>
+__device__ __forceinline__ UnitInfo decode_entry(const AttnParams& p, uint32_t code) {
+  UnitInfo u = decode_unit(p, code);
+  if (!PC) u.piece = false;
+  return u;
+}
+
 __device__ __forceinline__ void set_err(const AttnParams& p, int code) {
   if (p.err) atomicCAS(p.err, 0, code);
 }
@@ -463,32 +472,6 @@ __device__ __forceinline__ size_t piece_row(const AttnParams& p, int slot, int t
   return ((size_t)(slot * 2 + t) * out_branches(p) + br) * 128 + r;
 }
 
-// One branch of this piece: O from TMEM divided by l, and m + log2 l.  All
-// lanes of the warp take part (tcgen05.ld); rows past Lq store nothing.
-template <int D>
-__device__ __forceinline__ void piece_store(const AttnParams& p, int slot, int t, int br, int r, bool row_ok,
-                                            uint32_t tO, float m, float l) {
-  const size_t row = piece_row(p, slot, t, br, r);
-  const bool has = l > 0.f;
-  const float inv = has ? 1.f / l : 0.f;
-  float* dst = p.ws_o + row * D;
-#pragma unroll
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    uint32_t v[32];
-    tmem_ld32(tO + c0, v);
-    tmem_ld_wait();
-    reg_fence<32>(v);
-    if (row_ok) {
-      float4* d4 = reinterpret_cast<float4*>(dst + c0);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        d4[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
-                            __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
-    }
-  }
-  if (row_ok) p.ws_l[row] = has ? m + lg2_approx(l) : -INFINITY;
-}
-
 // Workspace slot of piece entry k.
 __device__ __forceinline__ int piece_slot(const AttnParams& p, int k) {
   const uint32_t y = p.pieces[k].y;
@@ -509,12 +492,32 @@ __device__ __forceinline__ uint32_t branches_reached(const AttnParams& p, int j0
   return m;
 }
 
+// A piece's slot row holds a branch's exact fp32 partial O / l split in two:
+// the high 16 bits of each value in its first D bf16, the low 16 bits in the
+// next D (the same split the two-branch merge uses), and its LSE (natural log)
+// at ws_l.  Reads go through L2 (the rows were written by other SMs).
+__device__ __forceinline__ void load_split32_l2(const __nv_bfloat16* hi, const __nv_bfloat16* lo, float* v) {
+  const uint4* h4 = reinterpret_cast<const uint4*>(hi);
+  const uint4* l4 = reinterpret_cast<const uint4*>(lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 H = __ldcg(h4 + q), L = __ldcg(l4 + q);
+    const uint32_t hw[4] = {H.x, H.y, H.z, H.w}, lw[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * q + 2 * e] = __uint_as_float((hw[e] << 16) | (lw[e] & 0xFFFFu));
+      v[8 * q + 2 * e + 1] = __uint_as_float((hw[e] & 0xFFFF0000u) | (lw[e] >> 16));
+    }
+  }
+}
+
 // Row r of tile t of a split unit from all of its pieces: per branch
 // L = log2 sum_i 2^L_i and O = sum_i 2^(L_i - L) O_i, then the outputs exactly
 // as an unsplit unit writes them (branch rows, LSEs, and the merge of two branches).
 template <int D>
 __device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
                                               int r, int qrow) {
+  constexpr float kLog2e = 1.4426950408889634f;
   const int nbr = out_branches(p);
   const bool do_merge = p.om != nullptr && nbr == 2;
   float w[2][kMaxPiecesPerUnit];
@@ -525,7 +528,7 @@ __device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInf
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-      Li[i] = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) : -INFINITY;
+      Li[i] = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) * kLog2e : -INFINITY;
       mx = fmaxf(mx, Li[i]);
     }
     float den = 0.f;
@@ -557,19 +560,19 @@ __device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInf
       float f[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) f[e] = 0.f;
+#pragma unroll 1
+      for (int i = 0; i < pi.n; ++i) {
+        float wi = 0.f;
 #pragma unroll
-      for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-        if (w[br][i] > 0.f) {
-          const float4* src =
-              reinterpret_cast<const float4*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D + c0);
+        for (int ii = 0; ii < kMaxPiecesPerUnit; ++ii)
+          if (ii == i) wi = w[br][ii];
+        if (wi > 0.f) {
+          const __nv_bfloat16* hi =
+              reinterpret_cast<const __nv_bfloat16*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D);
+          float x[32];
+          load_split32_l2(hi + c0, hi + D + c0, x);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 x = __ldcg(src + q);
-            f[4 * q] = fmaf(w[br][i], x.x, f[4 * q]);
-            f[4 * q + 1] = fmaf(w[br][i], x.y, f[4 * q + 1]);
-            f[4 * q + 2] = fmaf(w[br][i], x.z, f[4 * q + 2]);
-            f[4 * q + 3] = fmaf(w[br][i], x.w, f[4 * q + 3]);
-          }
+          for (int e = 0; e < 32; ++e) f[e] = fmaf(wi, x[e], f[e]);
         }
       }
       __nv_bfloat16* orow = p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
@@ -583,6 +586,58 @@ __device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInf
     p.lse[br][(size_t)u.s * p.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
   if (do_merge)
     p.lsem[(size_t)u.s * p.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
+}
+
+// A piece closes a branch into its workspace slot row: the exact fp32 partial
+// O / l (high halves in the row's first half, low halves in its second), and
+// the LSE beside it.  Out of line, like piece_finish.
+template <int D>
+__device__ __noinline__ void piece_close_branch(const AttnParams& p, int slot, int t, int br, int r, bool row_ok,
+                                                uint32_t tO, float m, float l) {
+  const size_t wrow = piece_row(p, slot, t, br, r);
+  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(p.ws_o + wrow * D);
+  const bool has = l > 0.f;
+  const float inv = has ? 1.f / l : 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tO + c0, v);
+    tmem_ld_wait();
+    reg_fence<32>(v);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
+    if (row_ok) store_split32(hi + c0, hi + D + c0, v);
+  }
+  if (row_ok) p.ws_l[wrow] = has ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
+}
+
+// End of a piece, for the 32 rows of one softmax warp (kept out of line so that
+// the step loop's register allocation is that of a whole unit): the partial of
+// the branch still open (cur_branch >= 0; O read from TMEM), LSE -inf for the
+// branches the piece did not reach, then the arrival; the warp that arrives
+// last for its (unit, tile, row quarter) combines every piece of the unit.
+template <int D>
+__device__ __noinline__ void piece_finish(const AttnParams& p, const UnitInfo& u, int k, int t, int quarter, int r,
+                                          bool row_ok, int qrow, uint32_t tO, int cur_branch, float m, float l,
+                                          int full) {
+  PieceInfo pi;
+  int kk = k;
+  const int nsteps = entry_steps(p, u, full, kk, pi);  // pi.j0: the entry's first step
+  const int slot = pi.slot0 + pi.idx;
+  if (cur_branch >= 0) piece_close_branch<D>(p, slot, t, cur_branch, r, row_ok, tO, m, l);
+  const uint32_t reached = branches_reached(p, pi.j0, nsteps);
+  if (row_ok)
+    for (int br = 0; br < out_branches(p); ++br)
+      if (!((reached >> br) & 1u)) p.ws_l[piece_row(p, slot, t, br, r)] = -INFINITY;
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane_id() == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8 + t * 4 + quarter, 1) == pi.n - 1) ? 1 : 0;
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (last) {
+    __threadfence();
+    if (row_ok) piece_combine<D>(p, u, pi, t, r, qrow);
+  }
 }
 
 // Register split between the producer/MMA warpgroup and the two softmax
@@ -600,7 +655,10 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xFFFFFFFFu
 // SP: the block-sparse instantiation.  It keeps two block lists, so the next
 // unit's list and its first copies are ready before the current unit ends; the
 // second list lives in the last K/V slot, which its ring then leaves out.
-template <int D, bool SP>
+// PC: the schedule has key-axis pieces.  Kept apart because the piece paths,
+// though cold, change the register allocation of the softmax step loop (measured
+// ~10 % more cycles per step on whole units with them compiled in).
+template <int D, bool SP, bool PC>
 __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constant__ AttnParams p) {
   using C = AttnCfg<D>;
   constexpr uint32_t NS = SP ? (uint32_t)C::NSLOT - 1u : (uint32_t)C::NSLOT;  // ring slots
@@ -675,7 +733,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       int piece_k = p.cta_piece0[blockIdx.x];
       bool ok = true;
       for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
-        const UnitInfo u = decode_unit(p, p.units[ui]);
+        const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
         int rs = 0, rl = 0;
         const int lb = SP ? (int)(ucnt & 1u) : 0;
         if (sparse) {
@@ -786,7 +844,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           mma_commit(b_sfull0 + 8 * t);
         };
         for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
-          const UnitInfo u = decode_unit(p, p.units[ui]);
+          const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
           int rs = 0, rl = 0;
           const int lb = SP ? (int)(ucnt & 1u) : 0;
           const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);  // this buffer's use parity
@@ -815,7 +873,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           if (nsteps == 1) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
             // a piece may start inside a branch: its first step starts the accumulator too
-            const bool first = (sparse || ragged) ? (j == 0) : (it.next().first || j == 0);
+            const bool first = (sparse || ragged) ? (j == 0) : (it.next().first || (PC && j == 0));
             const uint32_t vit = item + 2 * j + 1;
             const uint32_t knext = item + 2 * j + 2;
             const bool has_next = j + 1 < nsteps;
@@ -884,7 +942,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     int piece_k = p.cta_piece0[blockIdx.x];
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
-      const UnitInfo u = decode_unit(p, p.units[ui]);
+      const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
       int rs = 0, rl = 0;
       const int lb = SP ? (int)(ucnt & 1u) : 0;
       if (sparse) {
@@ -894,16 +952,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       } else if (ragged) {
         ragged_range(p, u.s, rs, rl, false);
       }
-      // the piece entry's index (its details are re-read from the parameters where
-      // needed, so that the step loop keeps no more state live than a whole unit)
-      const int pk = u.piece ? piece_k : -1;
-      int j0;
-      int nsteps;
-      {
-        PieceInfo pi;
-        nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
-        j0 = pi.j0;
-      }
+      // a piece's details are re-read from the parameters where needed (its entry
+      // is piece_k - 1), so that the step loop keeps no more state live than a
+      // whole unit does
+      PieceInfo pi0;
+      const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi0);
       const bool active = t < u.ntiles;
       int qrow = (u.tile0 + t) * 128 + r;
       if (sparse) {
@@ -918,7 +971,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       if (active && nsteps > 0) {
         TileIter it;
         it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
-        if (u.piece) it.seek(j0);
+        if (u.piece) it.seek(pi0.j0);
         for (int j = 0; j < nsteps; ++j) {
           const TileDesc td = it.next();
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
@@ -937,7 +990,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           reg_fence<128>(sr);
           VKV_STAMP(tr < 0 ? -1 : tr + 2);
           bool pending_epi = false;
-          if (td.first || j == 0) {
+          if (td.first || (PC && j == 0)) {
             if (cur_branch >= 0) {
               pending_epi = true;
               prev_branch = cur_branch;
@@ -1026,8 +1079,8 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           // O_t += P_t(j-1) V_{j-1}, and a commit covers all earlier MMAs.
           const bool need_o = pending_epi || __any_sync(0xFFFFFFFFu, rescale);
           VKV_STAMP(tr < 0 ? -1 : tr + 4);
-          if (pending_epi && u.piece) {
-            piece_store<D>(p, piece_slot(p, pk), t, prev_branch, r, row_ok, tO, m_prev, l_prev);
+          if (PC && pending_epi && u.piece) {
+            piece_close_branch<D>(p, piece_slot(p, piece_k - 1), t, prev_branch, r, row_ok, tO, m_prev, l_prev);
           } else if (pending_epi) {
             // close the previous branch: O / l and LSE
             const bool has = l_prev > 0.f;
@@ -1078,10 +1131,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ++np;
         }
         if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
-        if (ok && u.piece) {
-          tc_fence_after();
-          piece_store<D>(p, piece_slot(p, pk), t, cur_branch, r, row_ok, tO, m, l);
-        } else if (ok) {
+        if (ok && !u.piece) {
           tc_fence_after();
           // close the last branch, and merge with the one before it when asked
           const int lb = cur_branch;
@@ -1142,23 +1192,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         }
       }
       if (u.piece && active && ok) {
-        // this piece's rows are in the workspace (LSE -inf for branches it did not
-        // reach); the last piece of the unit to arrive combines every piece
-        const PieceInfo pi = piece_info(p, pk);
-        const int nbr = out_branches(p);
-        const uint32_t touched = branches_reached(p, j0, nsteps);
-        if (row_ok)
-          for (int br = 0; br < nbr; ++br)
-            if (!((touched >> br) & 1u)) p.ws_l[piece_row(p, pi.slot0 + pi.idx, t, br, r)] = -INFINITY;
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8 + t * 4 + quarter, 1) == pi.n - 1) ? 1 : 0;
-        last = __shfl_sync(0xFFFFFFFFu, last, 0);
-        if (last) {
-          __threadfence();
-          if (row_ok) piece_combine<D>(p, u, pi, t, r, qrow);
-        }
+        tc_fence_after();
+        piece_finish<D>(p, u, piece_k - 1, t, quarter, r, row_ok, qrow, tO, nsteps > 0 ? cur_branch : -1, m, l,
+                        unit_steps(p, ctl->list_count[lb], rl));
       }
       if (ok && active && row_ok && !u.piece) {
         // branches without any key tile: O = 0, LSE = -inf

@@ -116,8 +116,11 @@ WAN13B = (1, 12, 4680, 37440, [[(0, 1560), (32760, 4680)], [(1560, 31200)]])
 PYRAMID = [21840] * 4 + [53040, 39000, 31200, 26520] + [15600] * 4
 
 
-@pytest.mark.parametrize("shape", [WAN14B, WAN13B], ids=["wan14b", "wan13b"])
-def test_dense_split_schedule_covers_and_balances(shape):
+@pytest.mark.parametrize("shape,splits", [(WAN14B, False), (WAN13B, True)], ids=["wan14b", "wan13b"])
+def test_dense_split_schedule_covers_and_balances(shape, splits):
+    """A split schedule is taken only when it models at least 12 % less makespan (the
+    piece-enabled kernel runs its step loop ~10 % slower): Wan-1.3B (whole units
+    leave one pair and one lone tile per SM) is split, Wan-14B (a modelled 11 %) is not."""
     B, H, Lq, Lkv, br = shape
     a, steps = _seg_args(B, H, Lq, Lkv, br)
     T = (Lq + 127) // 128
@@ -125,11 +128,14 @@ def test_dense_split_schedule_covers_and_balances(shape):
     assert len(whole["pieces"]) == 0 and whole["n_slots"] == 0
     lw = _check_cover(whole, B * H, T, steps, 148)
     sp = vkv.attn_schedule(a, 148, True)
-    assert sp["n_slots"] > 0
     ls = _check_cover(sp, B * H, T, steps, 148)
-    ideal = (B * H) * ((T // 2) + C1 * (T & 1)) * (steps[0] + 2.0) / 148
-    assert ls.max() <= 1.05 * ideal
-    assert ls.max() <= 0.92 * lw.max()
+    assert (sp["n_slots"] > 0) == splits
+    if splits:
+        ideal = (B * H) * ((T // 2) + C1 * (T & 1)) * (steps[0] + 2.0) / 148
+        assert ls.max() <= 1.05 * ideal
+        assert ls.max() <= 0.88 * lw.max()
+    else:
+        assert np.array_equal(sp["units"], whole["units"])
 
 
 def test_ragged_split_schedule_covers_and_balances():
@@ -175,7 +181,7 @@ def test_workspace_size_needs_no_device_but_a_device_count():
         assert vkv.vkv_chunk_attn_workspace_size(a) == 0
 
 
-@pytest.mark.parametrize("topk,grouped", [(72, True), (144, True), (48, False)])
+@pytest.mark.parametrize("topk,grouped", [(72, True), (144, True), (144, False)])
 def test_block_sparse_split_schedule_covers_and_balances(topk, grouped):
     """Block-sparse pieces are cut in the schedule's estimated key steps of a unit
     (persistent blocks plus the expected union of its query blocks' selections,
@@ -196,7 +202,7 @@ def test_block_sparse_split_schedule_covers_and_balances(topk, grouped):
     assert len(sp["pieces"]) > 0
     ls = _check_cover(sp, 12, 36, steps, 148)
     ideal = 216 * (S2 + 2.0) / 148
-    assert ls.max() <= 0.97 * lw.max() and ls.max() <= 1.15 * ideal
+    assert ls.max() <= 0.88 * lw.max() and ls.max() <= 1.15 * ideal
 
 
 @pytest.mark.parametrize("topk", [9, 18, 36])
