@@ -468,8 +468,8 @@ int32_t vkv_version(void);
 
 /* sizeof() of the ABI structs, for bindings to check their layout:
  * 0 vkv_attn_args, 1 vkv_select_args, 2 vkv_tensor, 3 vkv_segment,
- * 4 vkv_compact_args, 5 vkv_head_rule, 6 vkv_persist_args, 7 vkv_latent_args;
- * -1 otherwise. */
+ * 4 vkv_compact_args, 5 vkv_head_rule, 6 vkv_persist_args, 7 vkv_latent_args,
+ * 8 vkv_schedule; -1 otherwise. */
 int32_t vkv_abi_sizeof(int32_t which);
 
 #ifdef __cplusplus

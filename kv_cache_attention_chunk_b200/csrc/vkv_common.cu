@@ -109,7 +109,7 @@ extern "C" const char* vkv_status_string(vkv_status s) {
   return "unknown status";
 }
 
-extern "C" int32_t vkv_version(void) { return 200; }
+extern "C" int32_t vkv_version(void) { return 300; }
 
 extern "C" int32_t vkv_abi_sizeof(int32_t which) {
   switch (which) {
@@ -121,6 +121,7 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
     case 5: return (int32_t)sizeof(vkv_head_rule);
     case 6: return (int32_t)sizeof(vkv_persist_args);
     case 7: return (int32_t)sizeof(vkv_latent_args);
+    case 8: return (int32_t)sizeof(vkv_schedule);
   }
   return -1;
 }

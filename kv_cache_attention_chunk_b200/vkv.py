@@ -174,7 +174,7 @@ def lib() -> ctypes.CDLL:
     L.vkv_debug_withhold_copy.argtypes = [c_int32]
     L.vkv_debug_withhold_copy.restype = c_int32
     for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
-                            vkv_head_rule, vkv_persist_args, vkv_latent_args)):
+                            vkv_head_rule, vkv_persist_args, vkv_latent_args, vkv_schedule)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
             raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
                                f"binding {ctypes.sizeof(st)} B")
