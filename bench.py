@@ -111,6 +111,13 @@ def load_peaks():
 ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx.cuh")
 
 
+def headline_kernel_name(vkv, q, k, v, case) -> str:
+    """The attention instantiation the headline call runs: with piece support when
+    its schedule cuts units along the key axis (a non-zero workspace)."""
+    pc = vkv.vkv_chunk_attn_workspace_size(vkv.segments_args(q, k, v, case.branches, case.scale)) > 0
+    return f"chunk_attn_kernel<128, 0, {int(pc)}>"
+
+
 def kernel_source_hash() -> str:
     """Hash of the attention kernel's code (ties recorded ncu counters to a kernel version).
 
@@ -564,7 +571,7 @@ def run_ours(args):
                    "flops_per_chunk": fl},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(),
-                     "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": "chunk_attn_kernel<128>",
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": headline_kernel_name(vkv, q, k, v, case),
                      "launch_ms_median": statistics.median(launch_ms),
                      "launch_ms_p10": float(np.percentile(launch_ms, 10)),
                      "launch_ms_p90": float(np.percentile(launch_ms, 90)),

@@ -342,6 +342,22 @@ def _new_out(q):
             torch.empty((B, H, Lq), dtype=torch.float32, device=q.device))
 
 
+def segments_args(q, k, v, branches, scale=None, err=None) -> vkv_attn_args:
+    """vkv_attn_args of a SEGMENTS call, inputs filled in, outputs left empty (the
+    segment arrays are kept alive by the returned struct)."""
+    d = q.shape[3]
+    a = _base_args(MODE_SEGMENTS, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
+    a.n_branches = len(branches)
+    keep = []
+    for i, br in enumerate(branches):
+        arr = (vkv_segment * max(1, len(br)))(*[vkv_segment(int(s), int(n)) for s, n in br])
+        keep.append(arr)
+        a.segs[i] = ctypes.cast(arr, POINTER(vkv_segment))
+        a.n_segs[i] = len(br)
+    a._keep_segs = keep
+    return a
+
+
 def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, stream=None, out=None,
                         split=True, workspace=None):
     """Dual-branch (or single-branch) chunk attention over token segments.
@@ -352,15 +368,7 @@ def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, st
     Returns dict(o=[...], lse=[...], o_merged, lse_merged).
     """
     nb = len(branches)
-    d = q.shape[3]
-    a = _base_args(MODE_SEGMENTS, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
-    a.n_branches = nb
-    keep = []
-    for i, br in enumerate(branches):
-        arr = (vkv_segment * max(1, len(br)))(*[vkv_segment(int(s), int(n)) for s, n in br])
-        keep.append(arr)
-        a.segs[i] = ctypes.cast(arr, POINTER(vkv_segment))
-        a.n_segs[i] = len(br)
+    a = segments_args(q, k, v, branches, scale, err)
     res = out if out is not None else {}
     if out is None:
         res["o"], res["lse"] = [], []
