@@ -655,7 +655,10 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     P->ws_cnt = reinterpret_cast<int*>(ws + w.cnt_off);
     P->ws_l = reinterpret_cast<float*>(ws + w.l_off);
     P->ws_o = reinterpret_cast<float*>(ws + w.o_off);
-    if (cudaMemsetAsync(P->ws_cnt, 0, (size_t)plan->n_slots * 8 * sizeof(int), st) != cudaSuccess)
+    // arrival counters to zero; partial LSEs to NaN, which marks a branch a piece
+    // did not reach
+    if (cudaMemsetAsync(P->ws_cnt, 0, (size_t)plan->n_slots * 8 * sizeof(int), st) != cudaSuccess ||
+        cudaMemsetAsync(P->ws_l, 0xFF, (size_t)plan->n_slots * 2 * nbr * 128 * sizeof(float), st) != cudaSuccess)
       return VKV_ERR_CUDA;
   }
 

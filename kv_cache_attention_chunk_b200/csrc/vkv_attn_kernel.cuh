@@ -70,6 +70,7 @@ struct Ctl {
   uint32_t tmem_base;
   int abort_flag;
   int list_count[2];
+  int piece_arrived[8];  // per softmax warp (tile * 4 + quarter): pieces whose partials it has stored
   uint32_t bitmap[4][32];
   uint32_t list[kMaxListEntries];  // block-list buffer 0 (buffer 1: the ring's last K/V slot)
 };
@@ -478,119 +479,14 @@ __device__ __forceinline__ int piece_slot(const AttnParams& p, int k) {
   return (int)(y & 0xFFFFu) + (int)((y >> 16) & 0xFFu);
 }
 
-// Branches that key steps [j0, j0 + n) of a unit's stream reach (bit b = branch b).
-__device__ __forceinline__ uint32_t branches_reached(const AttnParams& p, int j0, int n) {
-  if (n <= 0) return 0u;
-  if (p.mode != VKV_MODE_SEGMENTS) return 1u;
-  uint32_t m = 0u;
-  int b0 = 0;
-  for (int br = 0; br < p.n_branches; ++br) {
-    const int b1 = b0 + p.branch_steps[br];
-    if (b1 > b0 && j0 < b1 && j0 + n > b0) m |= 1u << br;
-    b0 = b1;
-  }
-  return m;
-}
-
 // A piece's slot row holds a branch's exact fp32 partial O / l split in two:
 // the high 16 bits of each value in its first D bf16, the low 16 bits in the
-// next D (the same split the two-branch merge uses), and its LSE (natural log)
-// at ws_l.  Reads go through L2 (the rows were written by other SMs).
-__device__ __forceinline__ void load_split32_l2(const __nv_bfloat16* hi, const __nv_bfloat16* lo, float* v) {
-  const uint4* h4 = reinterpret_cast<const uint4*>(hi);
-  const uint4* l4 = reinterpret_cast<const uint4*>(lo);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 H = __ldcg(h4 + q), L = __ldcg(l4 + q);
-    const uint32_t hw[4] = {H.x, H.y, H.z, H.w}, lw[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[8 * q + 2 * e] = __uint_as_float((hw[e] << 16) | (lw[e] & 0xFFFFu));
-      v[8 * q + 2 * e + 1] = __uint_as_float((hw[e] & 0xFFFF0000u) | (lw[e] >> 16));
-    }
-  }
-}
+// next D (the split the fused two-branch merge uses), and its LSE (natural
+// log) at ws_l.  The host fills ws_l with NaN before the launch, so a branch
+// a piece did not reach reads as absent.
 
-// Row r of tile t of a split unit from all of its pieces: per branch
-// L = log2 sum_i 2^L_i and O = sum_i 2^(L_i - L) O_i, then the outputs exactly
-// as an unsplit unit writes them (branch rows, LSEs, and the merge of two branches).
-template <int D>
-__device__ __forceinline__ void piece_combine(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
-                                              int r, int qrow) {
-  constexpr float kLog2e = 1.4426950408889634f;
-  const int nbr = out_branches(p);
-  const bool do_merge = p.om != nullptr && nbr == 2;
-  float w[2][kMaxPiecesPerUnit];
-  float L[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int br = 0; br < 2; ++br) {
-    float Li[kMaxPiecesPerUnit];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-      Li[i] = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) * kLog2e : -INFINITY;
-      mx = fmaxf(mx, Li[i]);
-    }
-    float den = 0.f;
-#pragma unroll
-    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-      w[br][i] = (Li[i] == -INFINITY) ? 0.f : ex2_approx(Li[i] - mx);
-      den += w[br][i];
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-    for (int i = 0; i < kMaxPiecesPerUnit; ++i) w[br][i] *= inv;
-    L[br] = den > 0.f ? mx + lg2_approx(den) : -INFINITY;
-  }
-  const float M = fmaxf(L[0], L[1]);
-  const float Ms = (M == -INFINITY) ? 0.f : M;
-  const float e0 = (L[0] == -INFINITY) ? 0.f : ex2_approx(L[0] - Ms);
-  const float e1 = (L[1] == -INFINITY) ? 0.f : ex2_approx(L[1] - Ms);
-  const float den = e0 + e1;
-  const float cb[2] = {den > 0.f ? e0 / den : 0.f, den > 0.f ? e1 / den : 0.f};
-  __nv_bfloat16* mrow = do_merge ? p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh : nullptr;
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    float g[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) g[e] = 0.f;
-#pragma unroll
-    for (int br = 0; br < 2; ++br) {
-      if (br >= nbr) continue;
-      float f[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) f[e] = 0.f;
-#pragma unroll 1
-      for (int i = 0; i < pi.n; ++i) {
-        float wi = 0.f;
-#pragma unroll
-        for (int ii = 0; ii < kMaxPiecesPerUnit; ++ii)
-          if (ii == i) wi = w[br][ii];
-        if (wi > 0.f) {
-          const __nv_bfloat16* hi =
-              reinterpret_cast<const __nv_bfloat16*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D);
-          float x[32];
-          load_split32_l2(hi + c0, hi + D + c0, x);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) f[e] = fmaf(wi, x[e], f[e]);
-        }
-      }
-      __nv_bfloat16* orow = p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
-      store_row32(orow + c0, f);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) g[e] = fmaf(cb[br], f[e], g[e]);
-    }
-    if (do_merge) store_row32(mrow + c0, g);
-  }
-  for (int br = 0; br < nbr; ++br)
-    p.lse[br][(size_t)u.s * p.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
-  if (do_merge)
-    p.lsem[(size_t)u.s * p.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
-}
-
-// A piece closes a branch into its workspace slot row: the exact fp32 partial
-// O / l (high halves in the row's first half, low halves in its second), and
-// the LSE beside it.  Out of line, like piece_finish.
+// A piece closes a branch into its workspace slot row (out of line, so that
+// the softmax step loop keeps the register allocation of a whole unit).
 template <int D>
 __device__ __noinline__ void piece_close_branch(const AttnParams& p, int slot, int t, int br, int r, bool row_ok,
                                                 uint32_t tO, float m, float l) {
@@ -611,33 +507,132 @@ __device__ __noinline__ void piece_close_branch(const AttnParams& p, int slot, i
   if (row_ok) p.ws_l[wrow] = has ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
 }
 
-// End of a piece, for the 32 rows of one softmax warp (kept out of line so that
-// the step loop's register allocation is that of a whole unit): the partial of
-// the branch still open (cur_branch >= 0; O read from TMEM), LSE -inf for the
-// branches the piece did not reach, then the arrival; the warp that arrives
-// last for its (unit, tile, row quarter) combines every piece of the unit.
-template <int D>
-__device__ __noinline__ void piece_finish(const AttnParams& p, const UnitInfo& u, int k, int t, int quarter, int r,
-                                          bool row_ok, int qrow, uint32_t tO, int cur_branch, float m, float l,
-                                          int full) {
-  PieceInfo pi;
-  int kk = k;
-  const int nsteps = entry_steps(p, u, full, kk, pi);  // pi.j0: the entry's first step
-  const int slot = pi.slot0 + pi.idx;
-  if (cur_branch >= 0) piece_close_branch<D>(p, slot, t, cur_branch, r, row_ok, tO, m, l);
-  const uint32_t reached = branches_reached(p, pi.j0, nsteps);
-  if (row_ok)
-    for (int br = 0; br < out_branches(p); ++br)
-      if (!((reached >> br) & 1u)) p.ws_l[piece_row(p, slot, t, br, r)] = -INFINITY;
-  __threadfence();
-  __syncwarp();
-  int last = 0;
-  if (lane_id() == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8 + t * 4 + quarter, 1) == pi.n - 1) ? 1 : 0;
-  last = __shfl_sync(0xFFFFFFFFu, last, 0);
-  if (last) {
-    __threadfence();
-    if (row_ok) piece_combine<D>(p, u, pi, t, r, qrow);
+// Bounded wait until the shared counter reaches `target` (raised by other warps).
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, volatile int* abort_flag, int* err) {
+  const volatile int* c = cnt;
+  if (*c >= target) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t n = 0;
+  while (*c < target) {
+    __nanosleep(128);
+    if (((++n) & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        if (err) atomicCAS(err, 0, VKV_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
   }
+  return true;
+}
+
+// One query row of a split unit from all of its pieces (row r of tile t): per
+// branch L = log2 sum_i 2^L_i and O = sum_i 2^(L_i - L) O_i, then the outputs
+// exactly as an unsplit unit writes them (branch rows, LSEs, and the merge of
+// two branches).  Eight columns at a time: it runs in the producer warpgroup's
+// register budget.
+template <int D>
+__device__ __forceinline__ void piece_combine_row(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
+                                                  int r, int qrow) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int nbr = out_branches(p);
+  const bool do_merge = p.om != nullptr && nbr == 2;
+  float w[2][kMaxPiecesPerUnit];
+  float L[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+      float x = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) : -INFINITY;
+      x = (x == x) ? x * kLog2e : -INFINITY;  // NaN: a branch this piece did not reach
+      w[br][i] = x;
+      mx = fmaxf(mx, x);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+      w[br][i] = (w[br][i] == -INFINITY) ? 0.f : ex2_approx(w[br][i] - mx);
+      den += w[br][i];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) w[br][i] *= inv;
+    L[br] = den > 0.f ? mx + lg2_approx(den) : -INFINITY;
+  }
+  const float M = fmaxf(L[0], L[1]);
+  const float Ms = (M == -INFINITY) ? 0.f : M;
+  const float e0 = (L[0] == -INFINITY) ? 0.f : ex2_approx(L[0] - Ms);
+  const float e1 = (L[1] == -INFINITY) ? 0.f : ex2_approx(L[1] - Ms);
+  const float den = e0 + e1;
+  const float cb[2] = {den > 0.f ? e0 / den : 0.f, den > 0.f ? e1 / den : 0.f};
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 8) {
+    float g[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g[e] = 0.f;
+#pragma unroll
+    for (int br = 0; br < 2; ++br) {
+      if (br >= nbr) continue;
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0.f;
+#pragma unroll 1
+      for (int i = 0; i < pi.n; ++i) {
+        float wi = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < kMaxPiecesPerUnit; ++ii)
+          if (ii == i) wi = w[br][ii];
+        if (wi > 0.f) {
+          const __nv_bfloat16* hi =
+              reinterpret_cast<const __nv_bfloat16*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D);
+          const uint4 H = __ldcg(reinterpret_cast<const uint4*>(hi + c0));
+          const uint4 Lo = __ldcg(reinterpret_cast<const uint4*>(hi + D + c0));
+          const uint32_t hw[4] = {H.x, H.y, H.z, H.w}, lw[4] = {Lo.x, Lo.y, Lo.z, Lo.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            f[2 * e] = fmaf(wi, __uint_as_float((hw[e] << 16) | (lw[e] & 0xFFFFu)), f[2 * e]);
+            f[2 * e + 1] = fmaf(wi, __uint_as_float((hw[e] & 0xFFFF0000u) | (lw[e] >> 16)), f[2 * e + 1]);
+          }
+        }
+      }
+      __nv_bfloat16* orow = p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
+      *reinterpret_cast<uint4*>(orow + c0) =
+          make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                     pack_bf16x2(f[6], f[7]));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = fmaf(cb[br], f[e], g[e]);
+    }
+    if (do_merge) {
+      __nv_bfloat16* mrow = p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh;
+      *reinterpret_cast<uint4*>(mrow + c0) =
+          make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
+                     pack_bf16x2(g[6], g[7]));
+    }
+  }
+  for (int br = 0; br < nbr; ++br)
+    p.lse[br][(size_t)u.s * p.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
+  if (do_merge)
+    p.lsem[(size_t)u.s * p.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
+}
+
+// Every row of a split unit, by one warp (32 lanes, rows r = lane, lane + 32, ...).
+// Inlined: it runs in the producer warpgroup after setmaxnreg lowered its
+// registers, and only inlined code is allocated within that budget.
+template <int D>
+__device__ __forceinline__ void piece_combine_unit(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi,
+                                                int lane) {
+  const bool sparse = p.mode == VKV_MODE_BLOCK_SPARSE;
+  for (int t = 0; t < u.ntiles; ++t)
+    for (int r = lane; r < 128; r += 32) {
+      int qrow = (u.tile0 + t) * 128 + r;
+      if (sparse) {
+        const int qbr = unit_qblk(p, u.s, 2 * (u.tile0 + t) + (r >> 6), false);
+        qrow = qbr >= 0 ? qbr * 64 + (r & 63) : p.Lq;
+      }
+      if (qrow < p.Lq) piece_combine_row<D>(p, u, pi, t, r, qrow);
+    }
 }
 
 // Register split between the producer/MMA warpgroup and the two softmax
@@ -703,6 +698,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     ctl->abort_flag = 0;
     ctl->list_count[0] = 0;
     ctl->list_count[1] = 0;
+    for (int i = 0; i < 8; ++i) ctl->piece_arrived[i] = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -923,6 +919,36 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         // every MMA issued so far completes before TMEM is released
         mma_commit(b_drain);
         mbar_wait_drain(b_drain, 0);
+      }
+      __syncwarp();
+    } else if (PC && warp == 2) {
+      // ------------------------------------------------------------ pieces
+      // For each piece of this CTA's list: wait until the unit's softmax warps have
+      // stored their partials, count the piece in at its unit's arrival counter, and
+      // when it is the unit's last piece to arrive, combine every piece of the unit.
+      // Each softmax warp counts its own arrivals, so a count of k means that warp has
+      // stored the k-th piece it took part in (a single-tile piece has no tile-1 warps).
+      int piece_k = p.cta_piece0[blockIdx.x];
+      int expected[2] = {0, 0};
+      bool ok = true;
+      for (int ui = u_begin; ui < u_end && ok; ++ui) {
+        const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
+        if (!u.piece) continue;
+        const PieceInfo pi = piece_info(p, piece_k++);
+        for (int t = 0; t < u.ntiles && ok; ++t) {
+          ++expected[t];
+          for (int q = 0; q < 4 && ok; ++q)
+            ok = wait_count(&ctl->piece_arrived[t * 4 + q], expected[t], abort_flag, p.err);
+        }
+        if (!ok) break;
+        __threadfence();
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8, 1) == pi.n - 1) ? 1 : 0;
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (last) {
+          __threadfence();
+          piece_combine_unit<D>(p, u, pi, (int)lane);
+        }
       }
       __syncwarp();
     }
@@ -1192,9 +1218,12 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         }
       }
       if (u.piece && active && ok) {
+        // close the branch still open, then report to the piece warp (warp 2)
         tc_fence_after();
-        piece_finish<D>(p, u, piece_k - 1, t, quarter, r, row_ok, qrow, tO, nsteps > 0 ? cur_branch : -1, m, l,
-                        unit_steps(p, ctl->list_count[lb], rl));
+        if (nsteps > 0) piece_close_branch<D>(p, piece_slot(p, piece_k - 1), t, cur_branch, r, row_ok, tO, m, l);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(&ctl->piece_arrived[t * 4 + quarter], 1);
       }
       if (ok && active && row_ok && !u.piece) {
         // branches without any key tile: O = 0, LSE = -inf
