@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <deque>
 #include <functional>
 #include <map>
 #include <memory>
@@ -28,6 +29,8 @@ struct Plan {
   std::vector<int> cta_piece0;
   std::vector<uint2> pieces;
   int n_slots = 0;
+  // the split units, for the combine kernel: unit code, first slot | piece count << 16
+  std::vector<uint32_t> split_code, split_slots;
 };
 
 struct Cand {
@@ -76,6 +79,8 @@ double lpt(std::vector<Cand>& units, int g, Plan* out) {
     out->cta_piece0.assign(g + 1, 0);
     out->pieces.clear();
     out->n_slots = 0;
+    out->split_code.clear();
+    out->split_slots.clear();
   }
   return mk;
 }
@@ -94,17 +99,31 @@ constexpr double kUnitOverhead = 2.0;
 constexpr double kPieceOverhead = 4.0;
 constexpr int kMinPieceSteps = 16;
 constexpr int kMinPieceStepsSparse = 24;
-constexpr double kSplitGain = 0.88;  // a split schedule is used below this makespan ratio
+#ifndef VKV_HEAD_MAJOR
+#define VKV_HEAD_MAJOR 1
+#endif
+#ifndef VKV_SPLIT_GAIN
+#define VKV_SPLIT_GAIN 0.97
+#endif
+constexpr double kSplitGain = VKV_SPLIT_GAIN;  // a split schedule is used below this makespan ratio
 
-// Schedule with key-axis pieces: longest-first onto the least loaded CTA, as for
-// whole units, but against a capacity T = slack * (total cost / CTAs).  A unit
-// that does not fit the least loaded CTA is cut: the piece that fills that CTA
-// up to T stays there, and the rest of its key steps goes back into the queue
-// as an item of its own (cut again if needed, at most kMaxPiecesPerUnit pieces).
-// The best of a few slacks is kept.  steps[s] is the key-step count of sequence s.
+// Schedule with key-axis pieces: each unit onto the least loaded CTA against a
+// capacity T = slack * (total cost / CTAs).  A unit that does not fit the least
+// loaded CTA is cut: the piece that fills that CTA up to T stays there, and the
+// rest of its key steps is placed next (cut again if needed, at most
+// kMaxPiecesPerUnit pieces).  The best of a few slacks is kept.  steps[s] is the
+// key-step count of sequence s.
+//
+// Order of placement.  head_major: units in sequence order, each sequence's
+// tiles in order, and the rest of a cut unit right after its piece.  With equal
+// unit costs this deals the units out in waves, so the CTAs working on one
+// head's query tiles (its odd last tile included) run at the same time and its
+// K/V is read from DRAM about once; only the last wave is cut into pieces.
+// Otherwise longest first (for unequal costs: ragged caches), the rest of a cut
+// unit going back into the queue by its cost.
 bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
-                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm, Plan* out,
-                double* mk_out) {
+                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
+                bool head_major, Plan* out, double* mk_out) {
   struct Item {
     double cost;
     uint32_t code;
@@ -145,15 +164,23 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
   for (double x : {1.15, 1.2, 1.3, 1.4}) slacks.push_back(x);
   for (double slack : slacks) {
     const double cap = lb * slack;
-    std::priority_queue<Item, std::vector<Item>, decltype(cmp)> q(cmp, base);
+    std::priority_queue<Item, std::vector<Item>, decltype(cmp)> q(cmp, head_major ? std::vector<Item>() : base);
+    std::deque<Item> fifo;
+    if (head_major) fifo.assign(base.begin(), base.end());
     std::priority_queue<E, std::vector<E>, std::greater<E>> heap;
     for (int c = 0; c < g; ++c) heap.push({0.0, c});
     // per CTA: (unit index, j0, j1) in placement order; j1 < 0 marks a whole unit
     std::vector<std::vector<std::pair<int, std::pair<int, int>>>> lists(g);
     std::vector<int> n_cut(base.size(), 0);
-    while (!q.empty()) {
-      Item it = q.top();
-      q.pop();
+    while (head_major ? !fifo.empty() : !q.empty()) {
+      Item it;
+      if (head_major) {
+        it = fifo.front();
+        fifo.pop_front();
+      } else {
+        it = q.top();
+        q.pop();
+      }
       E e = heap.top();
       heap.pop();
       const bool whole_unit = it.k == 0;
@@ -177,7 +204,10 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
         rest.j0 = it.j0 + n;
         rest.k = it.k + 1;
         rest.cost = it.rate * (rest.j1 - rest.j0 + kPieceOverhead);
-        q.push(rest);
+        if (head_major)
+          fifo.push_front(rest);
+        else
+          q.push(rest);
       }
       heap.push(e);
     }
@@ -196,7 +226,9 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
         n_pieces += n_cut[i];
       }
     for (int c = 0; c < g; ++c) n_units += (int)lists[c].size();
-    if (n_pieces > kMaxPieces || n_units > kMaxUnits || n_slots > 0xFFFF) continue;
+    int n_split = 0;
+    for (size_t i = 0; i < base.size(); ++i) n_split += n_cut[i] > 0 ? 1 : 0;
+    if (n_pieces > kMaxPieces || n_units > kMaxUnits || n_slots > 0xFFFF || n_split > kMaxSplitUnits) continue;
     if (!(mk < best)) continue;
     best = mk;
     // piece index of a cut = its rank among the unit's cuts by j0
@@ -230,6 +262,13 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
     out->cta_begin[g] = (int)out->units.size();
     out->cta_piece0[g] = (int)out->pieces.size();
     out->n_slots = n_slots;
+    out->split_code.clear();
+    out->split_slots.clear();
+    for (size_t i = 0; i < base.size(); ++i)
+      if (n_cut[i] > 0) {
+        out->split_code.push_back(base[i].code);
+        out->split_slots.push_back((uint32_t)slot0[i] | ((uint32_t)n_cut[i] << 16));
+      }
   }
   if (best >= 1e299) return false;
   *mk_out = best;
@@ -242,7 +281,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
 // into pieces of at least min_steps, when that shortens it by 12 % or more.
 bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
-               Plan* plan) {
+               bool head_major, Plan* plan) {
   // sequences by decreasing pair cost: their pairs are split first
   std::vector<int> order(n_seq);
   for (int s = 0; s < n_seq; ++s) order[s] = s;
@@ -292,11 +331,11 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std
   if (!steps.empty()) {
     Plan sp;
     double mk_split = 1e300;
-    // the whole-unit makespan in the same cost terms (a split plan always uses n_sm CTAs)
-    // the instantiation with piece support runs the step loop ~10 % slower (its
-    // cold piece paths change the loop's register allocation), so a split schedule
-    // must model a larger gain than that
-    if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, &sp, &mk_split) &&
+    // compared with the whole-unit makespan in the same cost terms (a split plan
+    // always uses n_sm CTAs); pieces add a workspace fill, partial stores and the
+    // combine launch, so a split must model a few per cent of gain (measured on
+    // B200: the Wan-14B shape, modelled 11 % shorter, ran 5-8 % faster split)
+    if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, head_major, &sp, &mk_split) &&
         mk_split < kSplitGain * best) {
       *plan = std::move(sp);
       return true;
@@ -314,14 +353,14 @@ std::map<std::string, std::shared_ptr<Plan>> g_plans;
 
 std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const std::vector<double>& pc,
                                const std::vector<double>& oc, const std::vector<int>& steps,
-                               const std::vector<int>& steps1, int min_steps, int n_sm) {
+                               const std::vector<int>& steps1, int min_steps, int n_sm, bool head_major) {
   {
     std::lock_guard<std::mutex> lk(g_plan_mu);
     auto it = g_plans.find(key);
     if (it != g_plans.end()) return it->second;
   }
   auto plan = std::make_shared<Plan>();
-  if (!make_plan(n_seq, T, pc, oc, steps, steps1, min_steps, n_sm, plan.get())) return nullptr;
+  if (!make_plan(n_seq, T, pc, oc, steps, steps1, min_steps, n_sm, head_major, plan.get())) return nullptr;
   std::lock_guard<std::mutex> lk(g_plan_mu);
   if (g_plans.size() > 256) g_plans.clear();
   g_plans[key] = plan;
@@ -391,6 +430,50 @@ bool out_ok(const vkv_tensor& t) {
   return t.ptr != nullptr && tensor_aligned(t);
 }
 
+// The piece combine kernel behind the attention grid (programmatic dependent
+// launch: its blocks wait for the whole attention grid with griddepcontrol.wait).
+vkv_status launch_combine(const AttnParams& P, const Plan& plan, int d, cudaStream_t st) {
+  auto c = std::make_unique<CombineParams>();
+  std::memset(c.get(), 0, sizeof(CombineParams));
+  c->mode = P.mode;
+  c->H = P.H;
+  c->Lq = P.Lq;
+  c->n_qblk = P.n_qblk;
+  c->nbr = P.mode == VKV_MODE_SEGMENTS ? P.n_branches : 1;
+  c->qblk_order = P.qblk_order;
+  c->ws_o = P.ws_o;
+  c->ws_l = P.ws_l;
+  for (int br = 0; br < VKV_MAX_BRANCHES; ++br) {
+    c->o[br] = P.o[br];
+    c->o_sb[br] = P.o_sb[br];
+    c->o_st[br] = P.o_st[br];
+    c->o_sh[br] = P.o_sh[br];
+    c->lse[br] = P.lse[br];
+  }
+  c->om = P.om;
+  c->om_sb = P.om_sb;
+  c->om_st = P.om_st;
+  c->om_sh = P.om_sh;
+  c->lsem = P.lsem;
+  c->n_units = (int)plan.split_code.size();
+  std::copy(plan.split_code.begin(), plan.split_code.end(), c->code);
+  std::copy(plan.split_slots.begin(), plan.split_slots.end(), c->slots);
+  const int rows_per_block = 256 / (d / 8);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(c->n_units * 2 * (128 / rows_per_block)));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = d == 128 ? cudaLaunchKernelEx(&cfg, piece_combine_kernel<128>, *c)
+                                 : cudaLaunchKernelEx(&cfg, piece_combine_kernel<64>, *c);
+  return e == cudaSuccess ? VKV_OK : VKV_ERR_CUDA;
+}
+
 }  // namespace
 
 }  // namespace vkv
@@ -398,17 +481,16 @@ bool out_ok(const vkv_tensor& t) {
 namespace vkv {
 namespace {
 
-// Bytes of the piece workspace: counters, LSEs, partial outputs (all 256-aligned).
+// Bytes of the piece workspace: partial LSEs, then partial outputs (256-aligned).
 struct WsLayout {
-  size_t cnt_off, l_off, o_off, bytes;
+  size_t l_off, o_off, bytes;
 };
 
 WsLayout ws_layout(int n_slots, int nbr, int d) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   WsLayout w;
-  w.cnt_off = 0;
-  w.l_off = al((size_t)n_slots * 8 * sizeof(int));
-  w.o_off = w.l_off + al((size_t)n_slots * 2 * nbr * 128 * sizeof(float));
+  w.l_off = 0;
+  w.o_off = al((size_t)n_slots * 2 * nbr * 128 * sizeof(float));
   w.bytes = n_slots > 0 ? w.o_off + (size_t)n_slots * 2 * nbr * 128 * d * sizeof(float) : 0;
   return w;
 }
@@ -585,7 +667,9 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
   key += "@" + std::to_string(g_max) + ":" + std::to_string(c1) + (steps.empty() ? "" : "/split");
   if (mode == VKV_MODE_BLOCK_SPARSE) min_steps = kMinPieceStepsSparse;
   if (steps1.empty()) steps1 = steps;
-  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, steps1, min_steps, g_max);
+  // equal unit costs (every mode but ragged): units dealt out head by head
+  const bool head_major = VKV_HEAD_MAJOR && mode != VKV_MODE_RAGGED;
+  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, steps1, min_steps, g_max, head_major);
   if (!plan) return VKV_ERR_UNSUPPORTED;
   P->n_ctas = plan->n_ctas;
   std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);
@@ -652,13 +736,10 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
     if (a->workspace_bytes < w.bytes) return VKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(a->workspace) & 255) return VKV_ERR_ALIGN;
     uint8_t* ws = reinterpret_cast<uint8_t*>(a->workspace);
-    P->ws_cnt = reinterpret_cast<int*>(ws + w.cnt_off);
     P->ws_l = reinterpret_cast<float*>(ws + w.l_off);
     P->ws_o = reinterpret_cast<float*>(ws + w.o_off);
-    // arrival counters to zero; partial LSEs to NaN, which marks a branch a piece
-    // did not reach
-    if (cudaMemsetAsync(P->ws_cnt, 0, (size_t)plan->n_slots * 8 * sizeof(int), st) != cudaSuccess ||
-        cudaMemsetAsync(P->ws_l, 0xFF, (size_t)plan->n_slots * 2 * nbr * 128 * sizeof(float), st) != cudaSuccess)
+    // partial LSEs to NaN (all bits set), which marks a branch a piece did not reach
+    if (cudaMemsetAsync(P->ws_l, 0xFF, (size_t)plan->n_slots * 2 * nbr * 128 * sizeof(float), st) != cudaSuccess)
       return VKV_ERR_CUDA;
   }
 
@@ -672,7 +753,9 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   }
   const bool sp = mode == VKV_MODE_BLOCK_SPARSE;
   const bool pc = plan->n_slots > 0;
-  return d == 128 ? launch_attn_d<128>(dev, sp, pc, *P, st) : launch_attn_d<64>(dev, sp, pc, *P, st);
+  const vkv_status ls = d == 128 ? launch_attn_d<128>(dev, sp, pc, *P, st) : launch_attn_d<64>(dev, sp, pc, *P, st);
+  if (ls != VKV_OK || !pc) return ls;
+  return launch_combine(*P, *plan, d, st);
 }
 
 #ifdef VKV_TRACE

@@ -22,6 +22,8 @@
 //   warp 1       MMA issuer: S_t = Q_t K^T and O_t += P_t V with tcgen05.mma,
 //                accumulators in tensor memory (TMEM); owns the TMEM allocation.
 //   warps 2-3    idle.
+// With key-axis pieces (PC), a piece leaves fp32 partials in a workspace and
+// piece_combine_kernel, launched behind this grid, merges them.
 //   warps 4-7    softmax + epilogue for query tile 0 (one thread per row).
 //   warps 8-11   softmax + epilogue for query tile 1.
 //
@@ -70,7 +72,6 @@ struct Ctl {
   uint32_t tmem_base;
   int abort_flag;
   int list_count[2];
-  int piece_arrived[8];  // per softmax warp (tile * 4 + quarter): pieces whose partials it has stored
   uint32_t bitmap[4][32];
   uint32_t list[kMaxListEntries];  // block-list buffer 0 (buffer 1: the ring's last K/V slot)
 };
@@ -467,10 +468,14 @@ __device__ __forceinline__ int out_branches(const AttnParams& p) {
 }
 
 // Key-axis pieces.  A piece of a split unit leaves, per branch it reached, O / l
-// (fp32) and its LSE (log2 units) in its workspace slot; the last piece of the
-// unit to arrive combines them (the LSE merge, the same as between branches).
+// (fp32) and its LSE (natural log) in its workspace slot; the combine kernel,
+// launched behind the attention grid, merges a unit's pieces (the LSE merge,
+// the same as between branches).  Slot rows: [slot][tile 2][branch nbr][row 128].
+__device__ __forceinline__ size_t piece_row_n(int nbr, int slot, int t, int br, int r) {
+  return ((size_t)(slot * 2 + t) * nbr + br) * 128 + r;
+}
 __device__ __forceinline__ size_t piece_row(const AttnParams& p, int slot, int t, int br, int r) {
-  return ((size_t)(slot * 2 + t) * out_branches(p) + br) * 128 + r;
+  return piece_row_n(out_branches(p), slot, t, br, r);
 }
 
 // Workspace slot of piece entry k.
@@ -479,11 +484,9 @@ __device__ __forceinline__ int piece_slot(const AttnParams& p, int k) {
   return (int)(y & 0xFFFFu) + (int)((y >> 16) & 0xFFu);
 }
 
-// A piece's slot row holds a branch's exact fp32 partial O / l split in two:
-// the high 16 bits of each value in its first D bf16, the low 16 bits in the
-// next D (the split the fused two-branch merge uses), and its LSE (natural
-// log) at ws_l.  The host fills ws_l with NaN before the launch, so a branch
-// a piece did not reach reads as absent.
+// A piece's slot row holds a branch's exact fp32 partial O / l (D floats at
+// ws_o) and its LSE (natural log, at ws_l).  The host fills ws_l with NaN before
+// the launch, so a branch a piece did not reach reads as absent.
 
 // A piece closes a branch into its workspace slot row (out of line, so that
 // the softmax step loop keeps the register allocation of a whole unit).
@@ -491,7 +494,7 @@ template <int D>
 __device__ __noinline__ void piece_close_branch(const AttnParams& p, int slot, int t, int br, int r, bool row_ok,
                                                 uint32_t tO, float m, float l) {
   const size_t wrow = piece_row(p, slot, t, br, r);
-  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(p.ws_o + wrow * D);
+  float* dst = p.ws_o + wrow * D;
   const bool has = l > 0.f;
   const float inv = has ? 1.f / l : 0.f;
 #pragma unroll
@@ -500,139 +503,119 @@ __device__ __noinline__ void piece_close_branch(const AttnParams& p, int slot, i
     tmem_ld32(tO + c0, v);
     tmem_ld_wait();
     reg_fence<32>(v);
+    if (row_ok) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
-    if (row_ok) store_split32(hi + c0, hi + D + c0, v);
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst + c0)[q] =
+            make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
+                        __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
+    }
   }
   if (row_ok) p.ws_l[wrow] = has ? (m + lg2_approx(l)) * kLn2 : -INFINITY;
 }
 
-// Bounded wait until the shared counter reaches `target` (raised by other warps).
-__device__ __forceinline__ bool wait_count(const int* cnt, int target, volatile int* abort_flag, int* err) {
-  const volatile int* c = cnt;
-  if (*c >= target) return true;
-  const uint64_t t0 = globaltimer();
-  uint32_t n = 0;
-  while (*c < target) {
-    __nanosleep(128);
-    if (((++n) & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        if (err) atomicCAS(err, 0, VKV_DEVERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-  return true;
-}
-
-// One query row of a split unit from all of its pieces (row r of tile t): per
-// branch L = log2 sum_i 2^L_i and O = sum_i 2^(L_i - L) O_i, then the outputs
-// exactly as an unsplit unit writes them (branch rows, LSEs, and the merge of
-// two branches).  Eight columns at a time: it runs in the producer warpgroup's
-// register budget.
+// Merges the pieces of the split units of one launch (one thread per 8 columns of
+// a query row), after the attention grid before it on the stream has completed:
+// per branch L = log sum_i e^L_i and O = sum_i e^(L_i - L) O_i, then the outputs as
+// an unsplit unit writes them (branch rows, LSEs, and the merge of two branches).
+// Launched as a programmatic dependent, so its blocks are placed while the
+// attention grid drains.
 template <int D>
-__device__ __forceinline__ void piece_combine_row(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi, int t,
-                                                  int r, int qrow) {
+__global__ void __launch_bounds__(256) piece_combine_kernel(const __grid_constant__ CombineParams c) {
+  constexpr int TPR = D / 8;       // threads per row
+  constexpr int RPB = 256 / TPR;   // rows per block
+  constexpr int BPT = 128 / RPB;   // blocks per 128-row query tile
   constexpr float kLog2e = 1.4426950408889634f;
-  const int nbr = out_branches(p);
-  const bool do_merge = p.om != nullptr && nbr == 2;
-  float w[2][kMaxPiecesPerUnit];
+  griddep_wait();
+  const int ui = blockIdx.x / (2 * BPT);
+  const int t = (blockIdx.x / BPT) & 1;
+  const int r = (blockIdx.x % BPT) * RPB + (int)threadIdx.x / TPR;
+  const int c0 = ((int)threadIdx.x % TPR) * 8;
+  if (ui >= c.n_units) return;
+  const uint32_t code = c.code[ui];
+  const int tile0 = (int)(code & 0xFFFu);
+  const int ntiles = ((code >> 13) & 1u) ? 2 : 1;
+  const int s = (int)(code >> 14);
+  if (t >= ntiles) return;
+  const int b = s / c.H, h = s - b * c.H;
+  int qrow = (tile0 + t) * 128 + r;
+  if (c.mode == VKV_MODE_BLOCK_SPARSE) {
+    // the unit's query blocks follow qblk_order (the attention kernel reports a bad entry)
+    const int pos = 2 * (tile0 + t) + (r >> 6);
+    int qb = pos < c.n_qblk ? pos : -1;
+    if (qb >= 0 && c.qblk_order) {
+      const int q = __ldg(c.qblk_order + (size_t)s * c.n_qblk + pos);
+      if (q >= 0 && q < c.n_qblk) qb = q;
+    }
+    qrow = qb >= 0 ? qb * 64 + (r & 63) : c.Lq;
+  }
+  if (qrow >= c.Lq) return;
+  const int slot0 = (int)(c.slots[ui] & 0xFFFFu);
+  const int n = (int)(c.slots[ui] >> 16);
+  const bool do_merge = c.om != nullptr && c.nbr == 2;
   float L[2] = {-INFINITY, -INFINITY};
+  float f[2][8];
 #pragma unroll
   for (int br = 0; br < 2; ++br) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[br][e] = 0.f;
+    if (br >= c.nbr) continue;
+    float w[kMaxPiecesPerUnit];
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-      float x = (br < nbr && i < pi.n) ? __ldcg(p.ws_l + piece_row(p, pi.slot0 + i, t, br, r)) : -INFINITY;
-      x = (x == x) ? x * kLog2e : -INFINITY;  // NaN: a branch this piece did not reach
-      w[br][i] = x;
+      float x = -INFINITY;
+      if (i < n) {
+        x = __ldcg(c.ws_l + piece_row_n(c.nbr, slot0 + i, t, br, r));
+        x = (x == x) ? x * kLog2e : -INFINITY;  // NaN: a branch this piece did not reach
+      }
+      w[i] = x;
       mx = fmaxf(mx, x);
     }
     float den = 0.f;
 #pragma unroll
     for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
-      w[br][i] = (w[br][i] == -INFINITY) ? 0.f : ex2_approx(w[br][i] - mx);
-      den += w[br][i];
+      w[i] = (w[i] == -INFINITY) ? 0.f : ex2_approx(w[i] - mx);
+      den += w[i];
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-    for (int i = 0; i < kMaxPiecesPerUnit; ++i) w[br][i] *= inv;
     L[br] = den > 0.f ? mx + lg2_approx(den) : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxPiecesPerUnit; ++i) {
+      if (w[i] > 0.f) {
+        const float wi = w[i] * inv;
+        const float4* src = reinterpret_cast<const float4*>(c.ws_o + piece_row_n(c.nbr, slot0 + i, t, br, r) * D + c0);
+        const float4 A = __ldcg(src), B2 = __ldcg(src + 1);
+        f[br][0] = fmaf(wi, A.x, f[br][0]);
+        f[br][1] = fmaf(wi, A.y, f[br][1]);
+        f[br][2] = fmaf(wi, A.z, f[br][2]);
+        f[br][3] = fmaf(wi, A.w, f[br][3]);
+        f[br][4] = fmaf(wi, B2.x, f[br][4]);
+        f[br][5] = fmaf(wi, B2.y, f[br][5]);
+        f[br][6] = fmaf(wi, B2.z, f[br][6]);
+        f[br][7] = fmaf(wi, B2.w, f[br][7]);
+      }
+    }
+    __nv_bfloat16* orow = c.o[br] + b * c.o_sb[br] + (long long)qrow * c.o_st[br] + h * c.o_sh[br] + c0;
+    *reinterpret_cast<uint4*>(orow) = make_uint4(pack_bf16x2(f[br][0], f[br][1]), pack_bf16x2(f[br][2], f[br][3]),
+                                                 pack_bf16x2(f[br][4], f[br][5]), pack_bf16x2(f[br][6], f[br][7]));
+    if (c0 == 0) c.lse[br][(size_t)s * c.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
   }
-  const float M = fmaxf(L[0], L[1]);
-  const float Ms = (M == -INFINITY) ? 0.f : M;
-  const float e0 = (L[0] == -INFINITY) ? 0.f : ex2_approx(L[0] - Ms);
-  const float e1 = (L[1] == -INFINITY) ? 0.f : ex2_approx(L[1] - Ms);
-  const float den = e0 + e1;
-  const float cb[2] = {den > 0.f ? e0 / den : 0.f, den > 0.f ? e1 / den : 0.f};
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 8) {
+  if (do_merge) {
+    const float M = fmaxf(L[0], L[1]);
+    const float Ms = (M == -INFINITY) ? 0.f : M;
+    const float e0 = (L[0] == -INFINITY) ? 0.f : ex2_approx(L[0] - Ms);
+    const float e1 = (L[1] == -INFINITY) ? 0.f : ex2_approx(L[1] - Ms);
+    const float den = e0 + e1;
+    const float a0 = den > 0.f ? e0 / den : 0.f, a1 = den > 0.f ? e1 / den : 0.f;
     float g[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) g[e] = 0.f;
-#pragma unroll
-    for (int br = 0; br < 2; ++br) {
-      if (br >= nbr) continue;
-      float f[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0.f;
-#pragma unroll 1
-      for (int i = 0; i < pi.n; ++i) {
-        float wi = 0.f;
-#pragma unroll
-        for (int ii = 0; ii < kMaxPiecesPerUnit; ++ii)
-          if (ii == i) wi = w[br][ii];
-        if (wi > 0.f) {
-          const __nv_bfloat16* hi =
-              reinterpret_cast<const __nv_bfloat16*>(p.ws_o + piece_row(p, pi.slot0 + i, t, br, r) * D);
-          const uint4 H = __ldcg(reinterpret_cast<const uint4*>(hi + c0));
-          const uint4 Lo = __ldcg(reinterpret_cast<const uint4*>(hi + D + c0));
-          const uint32_t hw[4] = {H.x, H.y, H.z, H.w}, lw[4] = {Lo.x, Lo.y, Lo.z, Lo.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            f[2 * e] = fmaf(wi, __uint_as_float((hw[e] << 16) | (lw[e] & 0xFFFFu)), f[2 * e]);
-            f[2 * e + 1] = fmaf(wi, __uint_as_float((hw[e] & 0xFFFF0000u) | (lw[e] >> 16)), f[2 * e + 1]);
-          }
-        }
-      }
-      __nv_bfloat16* orow = p.o[br] + u.b * p.o_sb[br] + (long long)qrow * p.o_st[br] + u.h * p.o_sh[br];
-      *reinterpret_cast<uint4*>(orow + c0) =
-          make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                     pack_bf16x2(f[6], f[7]));
-#pragma unroll
-      for (int e = 0; e < 8; ++e) g[e] = fmaf(cb[br], f[e], g[e]);
-    }
-    if (do_merge) {
-      __nv_bfloat16* mrow = p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh;
-      *reinterpret_cast<uint4*>(mrow + c0) =
-          make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
-                     pack_bf16x2(g[6], g[7]));
-    }
+    for (int e = 0; e < 8; ++e) g[e] = fmaf(a0, f[0][e], a1 * f[1][e]);
+    __nv_bfloat16* mrow = c.om + b * c.om_sb + (long long)qrow * c.om_st + h * c.om_sh + c0;
+    *reinterpret_cast<uint4*>(mrow) = make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]),
+                                                 pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
+    if (c0 == 0) c.lsem[(size_t)s * c.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
   }
-  for (int br = 0; br < nbr; ++br)
-    p.lse[br][(size_t)u.s * p.Lq + qrow] = (L[br] == -INFINITY) ? -INFINITY : L[br] * kLn2;
-  if (do_merge)
-    p.lsem[(size_t)u.s * p.Lq + qrow] = (M == -INFINITY) ? -INFINITY : (Ms + lg2_approx(den)) * kLn2;
-}
-
-// Every row of a split unit, by one warp (32 lanes, rows r = lane, lane + 32, ...).
-// Inlined: it runs in the producer warpgroup after setmaxnreg lowered its
-// registers, and only inlined code is allocated within that budget.
-template <int D>
-__device__ __forceinline__ void piece_combine_unit(const AttnParams& p, const UnitInfo& u, const PieceInfo& pi,
-                                                int lane) {
-  const bool sparse = p.mode == VKV_MODE_BLOCK_SPARSE;
-  for (int t = 0; t < u.ntiles; ++t)
-    for (int r = lane; r < 128; r += 32) {
-      int qrow = (u.tile0 + t) * 128 + r;
-      if (sparse) {
-        const int qbr = unit_qblk(p, u.s, 2 * (u.tile0 + t) + (r >> 6), false);
-        qrow = qbr >= 0 ? qbr * 64 + (r & 63) : p.Lq;
-      }
-      if (qrow < p.Lq) piece_combine_row<D>(p, u, pi, t, r, qrow);
-    }
 }
 
 // Register split between the producer/MMA warpgroup and the two softmax
@@ -698,7 +681,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     ctl->abort_flag = 0;
     ctl->list_count[0] = 0;
     ctl->list_count[1] = 0;
-    for (int i = 0; i < 8; ++i) ctl->piece_arrived[i] = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -713,6 +695,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the piece combine kernel behind this grid may be placed as SMs free up; it waits
+  // for this whole grid before it reads a partial
+  if (PC) griddep_launch_dependents();
   const uint32_t tmem = ctl->tmem_base;
   const int u_begin = p.cta_begin[blockIdx.x];
   const int u_end = p.cta_begin[blockIdx.x + 1];
@@ -919,36 +904,6 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         // every MMA issued so far completes before TMEM is released
         mma_commit(b_drain);
         mbar_wait_drain(b_drain, 0);
-      }
-      __syncwarp();
-    } else if (PC && warp == 2) {
-      // ------------------------------------------------------------ pieces
-      // For each piece of this CTA's list: wait until the unit's softmax warps have
-      // stored their partials, count the piece in at its unit's arrival counter, and
-      // when it is the unit's last piece to arrive, combine every piece of the unit.
-      // Each softmax warp counts its own arrivals, so a count of k means that warp has
-      // stored the k-th piece it took part in (a single-tile piece has no tile-1 warps).
-      int piece_k = p.cta_piece0[blockIdx.x];
-      int expected[2] = {0, 0};
-      bool ok = true;
-      for (int ui = u_begin; ui < u_end && ok; ++ui) {
-        const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
-        if (!u.piece) continue;
-        const PieceInfo pi = piece_info(p, piece_k++);
-        for (int t = 0; t < u.ntiles && ok; ++t) {
-          ++expected[t];
-          for (int q = 0; q < 4 && ok; ++q)
-            ok = wait_count(&ctl->piece_arrived[t * 4 + q], expected[t], abort_flag, p.err);
-        }
-        if (!ok) break;
-        __threadfence();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(p.ws_cnt + pi.slot0 * 8, 1) == pi.n - 1) ? 1 : 0;
-        last = __shfl_sync(0xFFFFFFFFu, last, 0);
-        if (last) {
-          __threadfence();
-          piece_combine_unit<D>(p, u, pi, (int)lane);
-        }
       }
       __syncwarp();
     }
@@ -1217,13 +1172,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           }
         }
       }
-      if (u.piece && active && ok) {
-        // close the branch still open, then report to the piece warp (warp 2)
+      if (u.piece && active && ok && nsteps > 0) {
+        // close the branch still open; the combine kernel that follows this grid on
+        // the stream merges the unit's pieces
         tc_fence_after();
-        if (nsteps > 0) piece_close_branch<D>(p, piece_slot(p, piece_k - 1), t, cur_branch, r, row_ok, tO, m, l);
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(&ctl->piece_arrived[t * 4 + quarter], 1);
+        piece_close_branch<D>(p, piece_slot(p, piece_k - 1), t, cur_branch, r, row_ok, tO, m, l);
       }
       if (ok && active && row_ok && !u.piece) {
         // branches without any key tile: O = 0, LSE = -inf

@@ -17,6 +17,7 @@ constexpr int kCtlBytes = 2048;        // control block in shared memory
 constexpr int kMaxFlatSegs = VKV_MAX_BRANCHES * VKV_MAX_SEGMENTS;
 constexpr int kMaxPieces = 384;        // key-axis pieces per launch (kernel parameter space)
 constexpr int kMaxPiecesPerUnit = 8;   // pieces one split unit may be cut into
+constexpr int kMaxSplitUnits = kMaxPieces / 2;  // split units per launch (each has >= 2 pieces)
 
 // Kernel parameters of the attention kernel, passed as __grid_constant__.
 // Unit code: bits [0,12) first query tile, bit 12 piece (the unit covers only the
@@ -58,18 +59,36 @@ struct AttnParams {
   int* err;
   int withhold_first_copy;  // test aid: the producer skips its first K/V copy (see vkv_debug_withhold_copy)
   // key-axis pieces: per workspace slot, the partial outputs (O / l, fp32)
-  // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (log2 units)
-  // [slot][tile][branch][row]; one arrival counter per (unit, tile, row quarter)
+  // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (natural log)
+  // [slot][tile][branch][row]
   int sp_est[2];  // BLOCK_SPARSE: key steps the schedule assumed for a 1- / 2-tile unit
   float* ws_o;
   float* ws_l;
-  int* ws_cnt;  // [slot][8], zeroed before the launch; a unit uses its first slot's
   // schedule: CTA c runs units[cta_begin[c] .. cta_begin[c+1])
   int n_ctas;
   int cta_begin[kMaxCtas + 1];
   int cta_piece0[kMaxCtas + 1];
   uint2 pieces[kMaxPieces];
   uint32_t units[kMaxUnits];
+};
+
+// Parameters of the piece combine kernel: the split units of one attention launch
+// (code = the unit code without the piece bit; slots = first workspace slot |
+// piece count << 16) and where their outputs go.
+struct CombineParams {
+  int mode, H, Lq, n_qblk, nbr;
+  const int* qblk_order;
+  const float* ws_o;
+  const float* ws_l;
+  __nv_bfloat16* o[VKV_MAX_BRANCHES];
+  long long o_sb[VKV_MAX_BRANCHES], o_st[VKV_MAX_BRANCHES], o_sh[VKV_MAX_BRANCHES];
+  float* lse[VKV_MAX_BRANCHES];
+  __nv_bfloat16* om;
+  long long om_sb, om_st, om_sh;
+  float* lsem;
+  int n_units;
+  uint32_t code[kMaxSplitUnits];
+  uint32_t slots[kMaxSplitUnits];
 };
 
 // Host helpers (vkv_common.cu).
