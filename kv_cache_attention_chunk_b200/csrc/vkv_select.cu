@@ -3,22 +3,21 @@
 // representative token per block for coarse scoring; component 3 "PBSA":
 // top-K blocks of the local window, per query block).
 //
-// Two kernels on the caller's stream:
-//   pool_kernel     mean of every 64-row block of Q and of the window part of K,
-//                   in fp32, written to the caller's workspace.  One CTA of 256
-//                   threads per (block, batch, group of 512/d heads): the group's
-//                   contiguous slice of each row is read with 16-byte loads,
-//                   16 rows per thread in flight; row groups are combined in
-//                   shared memory.  HBM-bound.
-//   select_kernel   one CTA per (batch*head, 8 query blocks): the pooled keys
-//                   are copied to shared memory 160 blocks at a time (cp.async),
-//                   each thread scores one window block against the CTA's eight
-//                   pooled queries, then one warp per query block runs an exact
-//                   top-K: radix selection of the K-th largest score on
-//                   order-preserving keys, ties at the threshold to the lower
-//                   block index; kept blocks are written in ascending order.
-//                   Launched as a programmatic dependent of the pooling kernel,
-//                   so its launch overlaps the pooling kernel's last CTAs.
+// Kernels on the caller's stream:
+//   pool_kernel     (unless the caller passes cached window block means) the
+//                   fp32 mean of every 64-row window block of K, written to the
+//                   caller's workspace.  One CTA of 256 threads per (block,
+//                   batch, group of 512/d heads): the group's contiguous slice of
+//                   each row is read with 16-byte loads, 16 rows per thread in
+//                   flight; row groups are combined in shared memory.  HBM-bound.
+//   select_kernel   one CTA per (batch*head, 4 query blocks): pools its query
+//                   blocks from Q into shared memory, scores them against the
+//                   window block means and keeps the exact top-K by counting
+//                   (below).  Launched as a programmatic dependent of the
+//                   pooling kernel, so its query pooling overlaps the window
+//                   pooling; it reads the window means only after the wait.
+//   order_kernel    (optional) the query-block order that groups similar
+//                   selections.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -29,176 +28,148 @@
 
 namespace vkv {
 
-// Development timeline (compiled only with -DVKV_TRACE): clock stamps of the
-// phases of select CTA (0, 0), read back with vkv_debug_sel_trace().
-#ifdef VKV_TRACE
-__device__ unsigned long long g_vkv_sel_trace[64];
-#define VKV_SEL_STAMP(i)                                                              \
-  do {                                                                                \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && (threadIdx.x & 31) == 0)               \
-      g_vkv_sel_trace[(threadIdx.x >> 5) * 8 + (i)] = clock64();                     \
-  } while (0)
-#else
-#define VKV_SEL_STAMP(i) \
-  do {                   \
-  } while (0)
-#endif
-
 namespace {
 
 struct SelParams {
-  const float* qbar;
-  const float* kbar;
-  int BH, n_qblk, n_win, topk;
+  const __nv_bfloat16* q;
+  long long q_sb, q_st, q_sh;
+  const float* kbar;  // [B*H][n_win][D] window block means
+  int H, Lq, n_qblk, n_win, topk;
   int* out_idx;
   float* out_scores;
 };
 
-constexpr int kSelWarps = 8;     // query blocks per CTA (one warp each for the top-K)
-constexpr int kSelChunk = 160;   // window blocks staged in shared memory at a time
+constexpr int kSelQ = 4;  // query blocks per CTA
 
 template <int D>
-__host__ __device__ constexpr int sel_row_stride() { return D + 4; }  // floats; keeps rows 16-byte aligned
-
-template <int D>
-constexpr size_t sel_smem_bytes(int n_win) {
-  return ((size_t)kSelWarps * D + (size_t)kSelChunk * sel_row_stride<D>() + (size_t)kSelWarps * n_win) *
-         sizeof(float);
+constexpr size_t sel_smem_bytes() {
+  // pooled queries + (row-group partial sums | 64-bit ranking keys) + kept bitmaps
+  constexpr size_t part = (size_t)(256 / (D / 8)) * kSelQ * D * sizeof(float);
+  constexpr size_t keys = (size_t)kSelQ * 1024 * sizeof(unsigned long long);
+  return (size_t)kSelQ * D * sizeof(float) + (part > keys ? part : keys) + (size_t)kSelQ * 32 * sizeof(uint32_t);
 }
-constexpr int kSelMaxSmem = (int)sel_smem_bytes<128>(1024);
 
-// grid: x = ceil(n_qblk / kSelWarps), y = b*H + h; 32 * kSelWarps threads.
-// Shared memory: the CTA's pooled queries [kSelWarps][D], a chunk of pooled
-// keys [kSelChunk][D + 4] and the scores [kSelWarps][n_win].  Pooled vectors
-// are copied with cp.async (every copy of a chunk in flight at once).  Thread i
-// scores window block w0 + i against all of the CTA's pooled queries: its key
-// row is read from shared memory once (float4 reads; with the 4-float pad the
-// eight rows of a quarter warp fall in distinct banks), the query rows are
-// broadcast.  Then warp q selects the top-K of query block j0 + q.
-template <int D, int kMaxPerLane>
-__global__ void __launch_bounds__(32 * kSelWarps) select_kernel(const SelParams p) {
-  extern __shared__ __align__(16) float sm[];
-  constexpr int RS = sel_row_stride<D>();
-  constexpr int D4 = D / 4;
-  float* qs = sm;                              // kSelWarps * D
-  float* ks = qs + kSelWarps * D;              // kSelChunk * RS
-  float* scs = ks + kSelChunk * RS;            // kSelWarps * n_win
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+// grid: x = ceil(n_qblk / kSelQ), y = b*H + h; 256 threads.
+//  1. Pool the CTA's kSelQ query blocks from q: thread (g, c) sums 16-byte column
+//     chunk c of rows g, g + G, ... of every block (all loads in flight at
+//     once), the row groups are added in shared memory, then divided by the
+//     block's row count.  This reads only q, so it runs before the wait for the
+//     window pooling kernel (a programmatic dependent launch overlaps the two).
+//  2. Thread w scores window block w against the kSelQ pooled queries, its
+//     block mean read once from global memory (L2).  NaN scores rank last and
+//     -0 counts as +0, so equal scores tie on the block index.
+//  3. Exact top-K by counting: each score becomes a unique 64-bit key (the
+//     order-preserving integer image of the score, then 1023 - w, so that of
+//     equal scores the lower block id ranks higher); a block is kept when fewer
+//     than topk keys of its query block exceed its own.  Kept blocks are marked
+//     in a bitmap and written in ascending order (their rank among kept ids).
+template <int D>
+__global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
+  constexpr int CPR = D / 8;     // 16-byte chunks per row
+  constexpr int G = 256 / CPR;   // row groups
+  constexpr int RPT = 64 / G;    // rows per thread and block
+  extern __shared__ __align__(16) uint8_t sel_sm[];
+  float* qs = reinterpret_cast<float*>(sel_sm);                                   // [kSelQ][D]
+  float* part = qs + kSelQ * D;                                                   // [G][kSelQ * D]
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part);        // [kSelQ][n_win] (after part)
+  constexpr size_t kUnion = sel_smem_bytes<D>() - (size_t)kSelQ * D * sizeof(float) - kSelQ * 32 * sizeof(uint32_t);
+  uint32_t* kept = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(part) + kUnion);  // [kSelQ][32]
   const int s = blockIdx.y;
-  const int j0 = blockIdx.x * kSelWarps;
-  const int nq = min(kSelWarps, p.n_qblk - j0);
-  const int j = j0 + warp;
-  const bool active = warp < nq;
-  VKV_SEL_STAMP(0);
-  griddep_launch_dependents();  // the (small) order kernel may be scheduled alongside
-  griddep_wait();  // the pooling kernel before this one on the stream has completed
-  VKV_SEL_STAMP(1);
-  const float* qsrc = p.qbar + ((size_t)s * p.n_qblk + j0) * D;
-  for (int x = threadIdx.x; x < kSelWarps * D4; x += blockDim.x) {
-    if (x < nq * D4)
-      cp_async16(qs + 4 * x, qsrc + 4 * x);
-    else
-      reinterpret_cast<float4*>(qs)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  const float* kb = p.kbar + (size_t)s * p.n_win * D;
-  for (int w0 = 0; w0 < p.n_win; w0 += kSelChunk) {
-    const int nw = min(kSelChunk, p.n_win - w0);
-    __syncthreads();  // the previous chunk is fully consumed
-    for (int x = threadIdx.x; x < nw * D4; x += blockDim.x) {
-      const int r = x / D4, c4 = x - (x / D4) * D4;
-      cp_async16(ks + r * RS + 4 * c4, kb + (size_t)(w0 + r) * D + 4 * c4);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    VKV_SEL_STAMP(2);
-    for (int r = threadIdx.x; r < nw; r += blockDim.x) {
-      const float4* kr = reinterpret_cast<const float4*>(ks + r * RS);
-      float acc[kSelWarps][4];
+  const int b = s / p.H, h = s - (s / p.H) * p.H;
+  const int j0 = blockIdx.x * kSelQ;
+  const int nq = min(kSelQ, p.n_qblk - j0);
+  const int tid = threadIdx.x;
+  {
+    const int c = tid % CPR, g = tid / CPR;
+    const __nv_bfloat16* base = p.q + b * p.q_sb + h * p.q_sh;
+    uint4 v[kSelQ][RPT];
 #pragma unroll
-      for (int q = 0; q < kSelWarps; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-#pragma unroll 4
-      for (int c = 0; c < D4; ++c) {
-        const float4 kv = kr[c];
+    for (int q = 0; q < kSelQ; ++q)
 #pragma unroll
-        for (int q = 0; q < kSelWarps; ++q) {
-          const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[c];
-          acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
-          acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
-          acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
-          acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+      for (int i = 0; i < RPT; ++i) {
+        const int row = (j0 + q) * 64 + g + G * i;
+        v[q][i] = (q < nq && row < p.Lq)
+                      ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * p.q_st) + c)
+                      : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+    for (int q = 0; q < kSelQ; ++q) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const uint32_t w[4] = {v[q][i].x, v[q][i].y, v[q][i].z, v[q][i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += __uint_as_float(w[e] << 16);
+          acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
         }
       }
+      float4* dst = reinterpret_cast<float4*>(part + (size_t)g * kSelQ * D + q * D + c * 8);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+  if (tid < kSelQ * 32) kept[tid] = 0u;
+  __syncthreads();
+  for (int x = tid; x < kSelQ * D; x += 256) {
+    const int q = x / D;
+    float sum = 0.f;
 #pragma unroll
-      for (int q = 0; q < kSelWarps; ++q) {
-        const float v = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
-        // NaN ranks last; -0 becomes +0 so that equal scores tie on the block index
-        scs[q * p.n_win + w0 + r] = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+    for (int g = 0; g < G; ++g) sum += part[(size_t)g * kSelQ * D + x];
+    const int nrows = q < nq ? min(64, p.Lq - (j0 + q) * 64) : 1;
+    qs[x] = sum * (1.f / (float)nrows);
+  }
+  __syncthreads();  // part is dead from here on: its space holds the keys
+  griddep_wait();   // the window pooling kernel before this one (if any) has completed
+  for (int w = tid; w < p.n_win; w += 256) {
+    const float4* kr = reinterpret_cast<const float4*>(p.kbar + ((size_t)s * p.n_win + w) * D);
+    float acc[kSelQ][4];
+#pragma unroll
+    for (int q = 0; q < kSelQ; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+      const float4 kv = __ldg(kr + c4);
+#pragma unroll
+      for (int q = 0; q < kSelQ; ++q) {
+        const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[c4];
+        acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
+        acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
+        acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
+        acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
       }
+    }
+#pragma unroll
+    for (int q = 0; q < kSelQ; ++q) {
+      float sc = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
+      sc = (sc != sc) ? -INFINITY : (sc == 0.f ? 0.f : sc);
+      if (q < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + q) * p.n_win + w] = sc;
+      const uint32_t u = __float_as_uint(sc);
+      const uint32_t ok = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);  // larger score -> larger key
+      keys[q * p.n_win + w] = ((unsigned long long)ok << 10) | (unsigned long long)(1023 - w);
     }
   }
   __syncthreads();
-  VKV_SEL_STAMP(3);
-  const float* sc = scs + warp * p.n_win;
-  if (!active) return;
-  if (p.out_scores) {
-    float* so = p.out_scores + ((size_t)s * p.n_qblk + j) * p.n_win;
-    for (int w = lane; w < p.n_win; w += 32) so[w] = sc[w];
+  const int npairs = nq * p.n_win;
+  for (int x = tid; x < npairs; x += 256) {
+    const int q = x / p.n_win, w = x - q * p.n_win;
+    const unsigned long long* kq = keys + q * p.n_win;
+    const unsigned long long kw = kq[w];
+    int above = 0;
+    for (int v = 0; v < p.n_win; ++v) above += kq[v] > kw ? 1 : 0;
+    if (above < p.topk) atomicOr(&kept[q * 32 + (w >> 5)], 1u << (w & 31));
   }
-  // exact top-K by radix selection of the topk-th largest score on
-  // order-preserving integer keys (32 rounds); every block above that
-  // score is kept, and of the blocks equal to it the lowest indices are kept.
-  // Each lane owns blocks w = lane + 32m.
-  const int per = (p.n_win + 31) >> 5;  // <= kMaxPerLane
-  uint32_t key[kMaxPerLane];
-#pragma unroll
-  for (int m = 0; m < kMaxPerLane; ++m) {
-    const int w = lane + 32 * m;
-    if (m < per && w < p.n_win) {
-      const uint32_t u = __float_as_uint(sc[w]);
-      key[m] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);  // larger score -> larger key
-    } else {
-      key[m] = 0u;  // absent: below every real score (whose keys are >= 0x007FFFFF)
-    }
+  __syncthreads();
+  for (int x = tid; x < npairs; x += 256) {
+    const int q = x / p.n_win, w = x - q * p.n_win;
+    const uint32_t* kb = kept + q * 32;
+    const uint32_t word = kb[w >> 5];
+    if (!((word >> (w & 31)) & 1u)) continue;
+    int pos = __popc(word & ((1u << (w & 31)) - 1u));
+    for (int i = 0; i < (w >> 5); ++i) pos += __popc(kb[i]);
+    p.out_idx[((size_t)s * p.n_qblk + j0 + q) * p.topk + pos] = w;
   }
-  uint32_t prefix = 0u, mask = 0u;
-  int need = p.topk;  // rank, among the not-yet-excluded keys, of the threshold
-  // one bit per round, most significant first (one warp sum per round: warp
-  // collectives are the cost here, so the fewest of them wins)
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t want = prefix | (1u << bit), mk = mask | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int m = 0; m < kMaxPerLane; ++m)
-      if (m < per) cnt += ((key[m] & mk) == want) ? 1 : 0;
-    cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-    if (cnt >= need) {
-      prefix = want;
-    } else {
-      need -= cnt;
-    }
-    mask = mk;
-  }
-  VKV_SEL_STAMP(4);
-  // prefix = key of the topk-th largest score; `need` of its equals are kept
-  int* oi = p.out_idx + ((size_t)s * p.n_qblk + j) * p.topk;
-  int written = 0, eq_seen = 0;
-#pragma unroll
-  for (int m = 0; m < kMaxPerLane; ++m) {
-    if (m < per) {
-      const int w = lane + 32 * m;
-      const bool valid = w < p.n_win;
-      const bool eq = valid && key[m] == prefix;
-      const uint32_t beq = __ballot_sync(0xFFFFFFFFu, eq);
-      const int eq_rank = eq_seen + __popc(beq & ((1u << lane) - 1u));
-      const bool keep = valid && (key[m] > prefix || (eq && eq_rank < need));
-      eq_seen += __popc(beq);
-      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-      if (keep) oi[written + __popc(bal & ((1u << lane) - 1u))] = w;
-      written += __popc(bal);
-    }
-  }
-  VKV_SEL_STAMP(5);
 }
 
 // Query-block order that groups blocks with similar selections (a work-grouping
@@ -261,42 +232,25 @@ bool launch_order(const int* sel, int* order, int BH, int n_qblk, int topk, cuda
   return cudaLaunchKernelEx(&cfg, order_kernel, op) == cudaSuccess;
 }
 
-// Instantiation by head dimension and by window size (candidates per lane).
-template <int D, int PER>
-bool launch_select_t(dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(select_kernel<D, PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxSmem) !=
-        cudaSuccess)
-      return false;
-    attr_set[dev] = true;
-  }
-  // programmatic dependent launch: set-up overlaps the tail of the pooling kernel
+// The selection kernel, as a programmatic dependent of the window pooling kernel
+// when one runs just before it (`after_pool`), else as an ordinary launch.
+template <int D>
+bool launch_select_t(dim3 g, bool after_pool, cudaStream_t st, const SelParams& sp) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = g;
-  cfg.blockDim = dim3(32 * kSelWarps);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = sel_smem_bytes<D>();
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel<D, PER>, sp) == cudaSuccess;
+  cfg.numAttrs = after_pool ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, select_kernel<D>, sp) == cudaSuccess;
 }
 
-template <int D>
-bool launch_select_d(int n_win, dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
-  if (n_win <= 160) return launch_select_t<D, 5>(g, smem, st, sp);
-  if (n_win <= 256) return launch_select_t<D, 8>(g, smem, st, sp);
-  if (n_win <= 512) return launch_select_t<D, 16>(g, smem, st, sp);
-  return launch_select_t<D, 32>(g, smem, st, sp);
-}
-
-bool launch_select(int d, int n_win, dim3 g, size_t smem, cudaStream_t st, const SelParams& sp) {
-  return d == 128 ? launch_select_d<128>(n_win, g, smem, st, sp) : launch_select_d<64>(n_win, g, smem, st, sp);
+bool launch_select(int d, dim3 g, bool after_pool, cudaStream_t st, const SelParams& sp) {
+  return d == 128 ? launch_select_t<128>(g, after_pool, st, sp) : launch_select_t<64>(g, after_pool, st, sp);
 }
 
 }  // namespace
@@ -304,20 +258,11 @@ bool launch_select(int d, int n_win, dim3 g, size_t smem, cudaStream_t st, const
 
 using namespace vkv;
 
-#ifdef VKV_TRACE
-// Development only (not in the public header): copy select CTA (0, 0)'s stamps.
-extern "C" int vkv_debug_sel_trace(void* dst, size_t bytes) {
-  cudaDeviceSynchronize();
-  return (int)cudaMemcpyFromSymbol(dst, vkv::g_vkv_sel_trace,
-                                   bytes < sizeof(vkv::g_vkv_sel_trace) ? bytes : sizeof(vkv::g_vkv_sel_trace));
-}
-#endif
-
 extern "C" size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,
                                                   int32_t block, int32_t d) {
   if (B <= 0 || H <= 0 || Lq <= 0 || n_win_blk <= 0 || block <= 0 || d <= 0) return 0;
-  const size_t n_qblk = (size_t)(Lq + block - 1) / block;
-  const size_t bytes = (size_t)B * H * (n_qblk + (size_t)n_win_blk) * d * sizeof(float);
+  // the window block means; the query blocks are pooled in shared memory
+  const size_t bytes = (size_t)B * H * (size_t)n_win_blk * d * sizeof(float);
   return (bytes + 255) & ~(size_t)255;
 }
 
@@ -340,46 +285,47 @@ vkv_status check_select_args(const vkv_select_args* a) {
   return VKV_OK;
 }
 
-// Pooling (query blocks, and the window blocks unless cached), scoring and
-// top-K, and the optional query-block order, on `st`; `scratch` holds the
-// pooled vectors.
-vkv_status run_select(const vkv_select_args* a, float* scratch, cudaStream_t st) {
+// Window pooling (unless the caller passes cached block means), then scoring
+// and top-K (the query blocks are pooled inside the selection kernel), and the
+// optional query-block order, on `st`; `kbar_scratch` receives the window
+// block means.
+vkv_status run_select(const vkv_select_args* a, float* kbar_scratch, cudaStream_t st) {
   const int BH = a->B * a->H;
   const int n_qblk = (a->Lq + 63) / 64;
-  PoolParams pp;
-  pp.q = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
-  pp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
-  pp.q_sb = a->q.sb; pp.q_st = a->q.st; pp.q_sh = a->q.sh;
-  pp.k_sb = a->k.sb; pp.k_st = a->k.st; pp.k_sh = a->k.sh;
-  pp.B = a->B;
-  pp.H = a->H;
-  pp.d = a->d;
-  pp.Lq = a->Lq;
-  pp.n_qblk = n_qblk;
-  pp.n_win = a->n_win_blk;
-  pp.win_row0 = a->window_blk0 * a->block;
-  pp.qbar = scratch;
-  pp.kbar = pp.qbar + (size_t)BH * n_qblk * a->d;
-  const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
-  // with cached window representatives only the query blocks are pooled
-  const dim3 pg(n_qblk + (a->kbar ? 0 : a->n_win_blk), a->B * ((a->H + ph - 1) / ph));
-  if (a->d == 128)
-    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
-  else
-    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  const bool pool_win = a->kbar == nullptr;
+  if (pool_win) {
+    PoolParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
+    pp.k_sb = a->k.sb; pp.k_st = a->k.st; pp.k_sh = a->k.sh;
+    pp.B = a->B;
+    pp.H = a->H;
+    pp.d = a->d;
+    pp.n_qblk = 0;
+    pp.n_win = a->n_win_blk;
+    pp.win_row0 = a->window_blk0 * a->block;
+    pp.kbar = kbar_scratch;
+    const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
+    const dim3 pg(a->n_win_blk, a->B * ((a->H + ph - 1) / ph));
+    if (a->d == 128)
+      pool_kernel<128><<<pg, 256, 0, st>>>(pp);
+    else
+      pool_kernel<64><<<pg, 256, 0, st>>>(pp);
+    if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
+  }
   SelParams sp;
-  sp.qbar = pp.qbar;
-  sp.kbar = a->kbar ? a->kbar : pp.kbar;
-  sp.BH = BH;
+  sp.q = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
+  sp.q_sb = a->q.sb; sp.q_st = a->q.st; sp.q_sh = a->q.sh;
+  sp.kbar = pool_win ? kbar_scratch : a->kbar;
+  sp.H = a->H;
+  sp.Lq = a->Lq;
   sp.n_qblk = n_qblk;
   sp.n_win = a->n_win_blk;
   sp.topk = a->topk;
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
-  const dim3 sg((n_qblk + kSelWarps - 1) / kSelWarps, BH);
-  const size_t smem = a->d == 128 ? sel_smem_bytes<128>(a->n_win_blk) : sel_smem_bytes<64>(a->n_win_blk);
-  if (!launch_select(a->d, a->n_win_blk, sg, smem, st, sp)) return VKV_ERR_CUDA;
+  const dim3 sg((n_qblk + kSelQ - 1) / kSelQ, BH);
+  if (!launch_select(a->d, sg, pool_win, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
   if (a->out_order && !launch_order(a->out_idx, a->out_order, BH, n_qblk, a->topk, st)) return VKV_ERR_CUDA;
   return VKV_OK;
@@ -391,9 +337,12 @@ vkv_status run_select(const vkv_select_args* a, float* scratch, cudaStream_t st)
 extern "C" vkv_status vkv_block_select(const vkv_select_args* a, vkv_stream_t stream) {
   const vkv_status chk = check_select_args(a);
   if (chk != VKV_OK) return chk;
-  const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
-  if (!a->workspace || a->workspace_bytes < need) return VKV_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
+  // the workspace holds the window block means, so it is needed only when they are pooled here
+  if (!a->kbar) {
+    const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
+    if (!a->workspace || a->workspace_bytes < need) return VKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
+  }
   int dev = 0;
   if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
   return run_select(a, reinterpret_cast<float*>(a->workspace), reinterpret_cast<cudaStream_t>(stream));
@@ -440,17 +389,20 @@ extern "C" vkv_status vkv_block_pool(vkv_tensor x, int32_t B, int32_t L, int32_t
 // loop whose device memory was fully planned at start-up and that hands the
 // library no allocator, or a host program that drives the library only
 // through this C interface and has no way to size, own and free a workspace.
-// For them the pooled block vectors live in one file-scope device array of
-// fixed size, kNoallocScratchBytes, which every GPU that loads the library
-// holds until the process exits.
+// For them the pooled window block vectors live in one file-scope device
+// array of fixed size, kNoallocScratchBytes, which every GPU that loads the
+// library holds until the process exits (calls that pass cached window means
+// in `kbar` do not use it).
 //
 // In host code `g_select_scratch` is only a host-side stand-in for the array;
 // its device address is looked up once per device (cudaGetSymbolAddress, with
-// that device current) on the first call made on it, and cached.  Every call
-// on a device shares the array and leaves the last call's contents behind;
-// nothing needs clearing, because every element the select kernel reads is
-// written by the pool kernel of the same call.  Calls that overlap on the GPU
-// (for example on two streams at once) race on the array.
+// that device current) on the first call made on it, and cached.  The cached
+// address belongs to the device's context at that time: after a
+// cudaDeviceReset the entry point must not be called again in the process.
+// Every call on a device shares the array and leaves the last call's contents
+// behind; nothing needs clearing, because every element the select kernel
+// reads is written by the pool kernel of the same call.  Calls that overlap on
+// the GPU (for example on two streams at once) race on the array.
 // ---------------------------------------------------------------------------
 namespace vkv {
 namespace {
@@ -482,7 +434,9 @@ void* noalloc_scratch(int dev) {
 extern "C" vkv_status vkv_block_select_noalloc(const vkv_select_args* a, vkv_stream_t stream) {
   const vkv_status chk = check_select_args(a);
   if (chk != VKV_OK) return chk;
-  const size_t need = vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
+  // the scratch holds the window block means, which cached representatives (kbar) replace
+  const size_t need =
+      a->kbar ? 0 : vkv_block_select_workspace_size(a->B, a->H, a->Lq, a->n_win_blk, a->block, a->d);
   if (need > kNoallocScratchBytes) return VKV_ERR_WORKSPACE;  // larger than the fixed scratch array
   int dev = 0;
   if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
