@@ -38,6 +38,11 @@ def _bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(BF16)
 
 
+def _bf16_values(a: np.ndarray) -> np.ndarray:
+    """float64 copy of the bf16 values (round to nearest even) of a float32 array."""
+    return _bf16(a).to(torch.float64).numpy()
+
+
 # ---------------------------------------------------------------------------
 # Mode 1: dual-branch chunk over a segmented cache (configs 1, 2 and 5)
 # ---------------------------------------------------------------------------
@@ -138,10 +143,14 @@ class SparseCase:
         return -(-self.Lq // self.block)
 
 
+MIN_TOPK_GAP = 0.05  # fp64 score gap at every ranking boundary the selection tests use
+
+
 def make_block_sparse(name: str = "sparse", seed: int = 2, H: int = 12, d: int = 128,
                       frame_tokens: int = 32 * 48, block: int = 64, hist_frames: int = 30,
                       win_frames: int = 6, q_frames: int = 3, n_persist: int = 32,
-                      B: int = 1, planted: bool = True) -> SparseCase:
+                      B: int = 1, planted: bool = True, noise: str = "antithetic",
+                      gap_fn=None, max_tries: int = 64) -> SparseCase:
     """Cache of ``hist_frames`` history frames followed by a ``win_frames`` local window.
 
     The query chunk is the window's last ``q_frames`` frames (its keys sit in
@@ -153,15 +162,25 @@ def make_block_sparse(name: str = "sparse", seed: int = 2, H: int = 12, d: int =
     * window block b carries the offset a_{h,b} = 0.25 * (r_{h,b} - (n_win-1)/2)
       along u_h, r_{h,b} a random permutation of 0..n_win-1, added to every
       key of the block;
-    * the key noise of every window block is drawn as antithetic pairs
-      (z, -z), randomly placed inside the block, so that it sums to zero over
-      the block;
     * query block j carries beta_{h,j} = +/-(1 + U[0,1)) along u_h, added to
       every query of the block.
 
-    The block ranking of query block j is then the order of beta_{h,j} * a_{h,b}
-    up to bf16 rounding, with neighbouring ranks at least about
-    0.25 * |beta| apart: the selection is unambiguous by construction.
+    Key noise of the window blocks (``noise``):
+
+    * ``"antithetic"``: drawn as pairs (z, -z), randomly placed inside the
+      block, so that it sums to zero over the block.  The block ranking of
+      query block j is then the order of beta_{h,j} * a_{h,b} up to bf16
+      rounding, neighbouring ranks at least about 0.25 * |beta| apart: the
+      selection is unambiguous by construction, with no scoring needed here.
+    * ``"iid"``: plain N(0, 1), as every other key.  The ranking margin then
+      has to be checked: ``gap_fn(q_h, k_win_h)`` (supplied by the caller; this
+      module computes no scores) receives one head's query rows [Lq, d] and
+      window key rows [n_win * block, d] as float64 copies of the bf16 values
+      and returns, per query block, the smallest score gap at the ranking
+      boundaries the caller cares about.  Every query block whose gap is below
+      MIN_TOPK_GAP gets a new beta and new query noise, drawn from the sub-seed
+      (seed, b, h, j, try), until all pass (at most ``max_tries`` rounds).
+
     Persistent blocks carry no offset.
     """
     assert frame_tokens % block == 0
@@ -178,6 +197,8 @@ def make_block_sparse(name: str = "sparse", seed: int = 2, H: int = 12, d: int =
     persist = np.zeros((B * H, n_persist), dtype=np.int32)
     meta = dict(seed=seed, hist_frames=hist_frames, win_frames=win_frames, q_frames=q_frames,
                 frame_tokens=frame_tokens, planted=planted)
+    if noise not in ("antithetic", "iid"):
+        raise ValueError(noise)
     if planted:
         u = rng.standard_normal((B, H, d))
         u /= np.linalg.norm(u, axis=-1, keepdims=True)
@@ -190,13 +211,42 @@ def make_block_sparse(name: str = "sparse", seed: int = 2, H: int = 12, d: int =
         for b in range(B):
             for h in range(H):
                 for wb in range(n_win_blk):
-                    z = rng.standard_normal((half, d), dtype=np.float32)
-                    rows = np.concatenate([z, -z], axis=0)[rng.permutation(block)]
                     s = w0 + wb * block
+                    if noise == "antithetic":
+                        z = rng.standard_normal((half, d), dtype=np.float32)
+                        rows = np.concatenate([z, -z], axis=0)[rng.permutation(block)]
+                    else:
+                        rows = k[b, s:s + block, h, :]
                     k[b, s:s + block, h, :] = rows + (a[b, h, wb] * u[b, h]).astype(np.float32)
                 for j in range(n_qblk):
                     q[b, j * block:(j + 1) * block, h, :] += (beta[b, h, j] * u[b, h]).astype(np.float32)
-        meta.update(a=a, beta=beta, u=u)
+        meta.update(a=a, beta=beta, u=u, noise=noise)
+        if noise == "iid":
+            if gap_fn is None:
+                raise ValueError("noise='iid' needs gap_fn to check the ranking margin")
+            min_gap = np.inf
+            tries = 0
+            for b in range(B):
+                for h in range(H):
+                    kw = _bf16_values(k[b, w0:w0 + n_win_blk * block, h, :])
+                    for t in range(max_tries + 1):
+                        gaps = np.asarray(gap_fn(_bf16_values(q[b, :, h, :]), kw), dtype=np.float64)
+                        bad = np.nonzero(gaps < MIN_TOPK_GAP)[0]
+                        if len(bad) == 0:
+                            min_gap = min(min_gap, float(gaps.min()))
+                            tries = max(tries, t)
+                            break
+                        if t == max_tries:
+                            raise RuntimeError(f"query blocks {bad.tolist()} of (b={b}, h={h}) still have a "
+                                               f"top-K gap below {MIN_TOPK_GAP} after {max_tries} redraws")
+                        for j in bad:
+                            sub = np.random.default_rng([seed, b, h, int(j), t + 1])
+                            bj = sub.choice(np.array([-1.0, 1.0])) * (1.0 + sub.random())
+                            lo, hi = j * block, min(Lq, (j + 1) * block)
+                            q[b, lo:hi, h, :] = (sub.standard_normal((hi - lo, d), dtype=np.float32) +
+                                                 (bj * u[b, h]).astype(np.float32))
+                            beta[b, h, j] = bj
+            meta.update(min_topk_gap=min_gap, redraw_rounds=tries)
     for bh in range(B * H):
         persist[bh] = np.sort(rng.choice(n_hist_blk, size=n_persist, replace=False)).astype(np.int32)
     return SparseCase(name, B, H, d, block, _bf16(q), _bf16(k), _bf16(v), persist,

@@ -39,3 +39,28 @@ def assert_lse_close(gpu, ref, what=""):
         assert d.max() <= LSE_ABS, f"{what}: LSE max-abs {d.max():.3e} > {LSE_ABS}"
         return float(d.max())
     return 0.0
+
+
+def config3_gap_fn(topks, block=64):
+    """Margin check for the i.i.d. config-3 generator (test infrastructure).
+
+    Returns gap_fn(q_h, k_win_h) -> per query block, the smallest fp64 score gap
+    between the K-th and (K+1)-th window block over K in `topks`, with the
+    scores taken from the oracle (mean-pooled blocks, inner product).
+    """
+    import oracle
+
+    def fn(qh, kwin):
+        n_win = kwin.shape[0] // block
+        s = oracle.block_scores(qh[None, :, None, :], kwin[None, :, None, :], 0, n_win, block)[0]
+        return np.min([oracle.topk_gap(s, K) for K in topks], axis=0)
+
+    return fn
+
+
+def sparse_iid_case(**kw):
+    """Config 3 with i.i.d. N(0,1) window-key noise, redrawn until every query block
+    has an fp64 top-K gap >= 0.05 at K = 9, 18, 36 (6.25 / 12.5 / 25 % of 144)."""
+    from kv_cache_attention_chunk_b200 import workloads as W
+    topks = kw.pop("topks", (9, 18, 36))
+    return W.make_block_sparse(noise="iid", gap_fn=config3_gap_fn(topks), **kw)

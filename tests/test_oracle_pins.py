@@ -403,3 +403,41 @@ def test_planted_mistakes_are_caught(monkeypatch, mutant, target, pins):
         except AssertionError:
             caught = True
     assert caught, f"mutant {mutant.__name__} slipped past {pins}"
+
+
+@pytest.mark.slow
+def test_iid_sparse_config_margin_and_noise():
+    """Config 3 with i.i.d. key noise: the redraw loop leaves every (head, query block)
+    with a margin >= 0.05 at K = 9, 18, 36, recomputed here on the final tensors, and
+    the window keys' noise does not cancel inside a block (it is not antithetic)."""
+    from parity_util import sparse_iid_case
+    c = sparse_iid_case(name="iid")
+    s = oracle.block_scores(c.q, c.k, c.window_blk0, c.n_win_blk, c.block)
+    for K in (9, 18, 36):
+        assert oracle.topk_gap(s, K).min() >= W.MIN_TOPK_GAP
+    assert c.meta["min_topk_gap"] >= W.MIN_TOPK_GAP
+    k = oracle.to64(c.k)[0]
+    u = c.meta["u"][0]
+    w0 = c.window_blk0 * c.block
+    for h in (0, 5, 11):
+        kw = k[w0:w0 + c.n_win_blk * c.block, h, :].reshape(c.n_win_blk, c.block, -1)
+        planted = (c.meta["a"][0, h][:, None] * u[h][None, :])
+        resid = kw.mean(axis=1) - planted  # block mean of the noise alone
+        # N(0, 1) noise: each coordinate of a 64-row mean has std 1/8
+        assert 0.09 < resid.std() < 0.16
+
+
+def test_iid_sparse_reduced_margin():
+    from parity_util import sparse_iid_case
+    c = sparse_iid_case(name="iid-mid", seed=5, H=2, d=128, frame_tokens=1536, block=64, hist_frames=2,
+                        win_frames=6, q_frames=3, n_persist=4)
+    s = oracle.block_scores(c.q, c.k, c.window_blk0, c.n_win_blk, c.block)
+    for K in (9, 18, 36):
+        assert oracle.topk_gap(s, K).min() >= 0.05
+    assert c.meta["redraw_rounds"] >= 1  # the i.i.d. recipe does need redraws
+
+
+def test_iid_generator_refuses_without_margin_check():
+    with pytest.raises(ValueError):
+        W.make_block_sparse("x", seed=1, H=1, d=16, frame_tokens=64, block=16, hist_frames=1, win_frames=2,
+                            q_frames=1, n_persist=1, noise="iid")
