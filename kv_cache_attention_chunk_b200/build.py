@@ -5,6 +5,8 @@
 Each .cu under csrc/ is compiled to an object in <repo>/_build/ (in parallel),
 then linked into kv_cache_attention_chunk_b200/libvkv.so with the CUDA runtime
 linked statically, so the library loads on machines without a GPU driver.
+The same sources built with VKV_TEST_AIDS defined give libvkv_test.so, the
+test build that also exports the test aids of include/vkv_test.h.
 """
 from __future__ import annotations
 
@@ -22,6 +24,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvkv.so")
+LIB_TEST = os.path.join(PKG, "libvkv_test.so")
+TEST_DEFINES = ("VKV_TEST_AIDS",)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-Xptxas", "-v",
@@ -41,13 +45,13 @@ def _sources():
 
 def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
-        [os.path.join(INCLUDE, "vkv.h"), os.path.abspath(__file__)]
+        glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(target: str = LIB) -> bool:
+    if not os.path.exists(target):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(target)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -64,15 +68,23 @@ def _compile(src: str, verbose: bool, defines=(), tag: str = "") -> tuple[str, s
 
 
 def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
-    """Compile every CUDA source for sm_100a and link libvkv.so; returns its path.
+    """Compile every CUDA source for sm_100a and link libvkv.so and its test build
+    libvkv_test.so; returns the path of libvkv.so.
 
-    `out` / `defines` build a variant library (extra -D macros) at another path.
+    `out` / `defines` build one variant library (extra -D macros) at another path.
     """
-    target = out or LIB
-    if not force and out is None and not defines and up_to_date():
+    if out is None and not defines:
+        _build_one(LIB, (), force, verbose)
+        _build_one(LIB_TEST, TEST_DEFINES, force, verbose)
         return LIB
+    return _build_one(out or LIB, tuple(defines), True, verbose)
+
+
+def _build_one(target: str, defines, force: bool, verbose: bool) -> str:
+    if not force and up_to_date(target):
+        return target
     os.makedirs(BUILD, exist_ok=True)
-    tag = "" if out is None else os.path.basename(out).replace(".so", "") + "_"
+    tag = "" if target == LIB else os.path.basename(target).replace(".so", "") + "_"
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         results = list(ex.map(lambda s: _compile(s, verbose, defines, tag), _sources()))
     objs = [o for o, _ in results]

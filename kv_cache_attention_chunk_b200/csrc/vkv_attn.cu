@@ -98,7 +98,10 @@ inline uint32_t unit_code(int s, int tile0, bool two) {
 constexpr double kUnitOverhead = 2.0;
 constexpr double kPieceOverhead = 4.0;
 constexpr int kMinPieceSteps = 16;
-constexpr int kMinPieceStepsSparse = 24;
+#ifndef VKV_MIN_PIECE_SPARSE
+#define VKV_MIN_PIECE_SPARSE 24
+#endif
+constexpr int kMinPieceStepsSparse = VKV_MIN_PIECE_SPARSE;
 #ifndef VKV_HEAD_MAJOR
 #define VKV_HEAD_MAJOR 1
 #endif
@@ -727,7 +730,9 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   int dev = 0;
   const vkv_status stt = attn_setup(a, true, want_split, P.get(), &plan, &dev);
   if (stt != VKV_OK) return stt;
+#ifdef VKV_TEST_AIDS
   P->withhold_first_copy = take_withhold_request() ? 1 : 0;
+#endif
   const int mode = a->mode, B = a->B, H = a->H, Lq = a->Lq, Lkv = a->Lkv, d = a->d;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (plan->n_slots > 0) {
@@ -757,6 +762,33 @@ extern "C" vkv_status vkv_chunk_attn(const vkv_attn_args* a, vkv_stream_t stream
   if (ls != VKV_OK || !pc) return ls;
   return launch_combine(*P, *plan, d, st);
 }
+
+#ifdef VKV_TEST_AIDS
+namespace vkv {
+namespace {
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float e0, e1;
+  exp2_poly2(x0, x1, e0, e1);
+  y[i] = e0;
+  if (i + 1 < n) y[i + 1] = e1;
+}
+}  // namespace
+}  // namespace vkv
+
+// Test build only (vkv_test.h): the attention softmax's FMA-pipe exp2 on n DEVICE floats.
+extern "C" vkv_status vkv_debug_exp2_poly(const float* x, float* y, int32_t n, vkv_stream_t stream) {
+  if (!x || !y) return VKV_ERR_NULL;
+  if (n <= 0) return VKV_ERR_SHAPE;
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
+  const int pairs = (n + 1) / 2;
+  vkv::exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? VKV_OK : VKV_ERR_CUDA;
+}
+#endif
 
 #ifdef VKV_TRACE
 // Development only (not in the public header): copy CTA 0's pipeline timeline.

@@ -413,18 +413,25 @@ __device__ __forceinline__ void load_split32(const __nv_bfloat16* hi, const __nv
   }
 }
 
-// Optional exp2 on the FMA pipe for part of the columns, to unload the MUFU
-// pipe (one exponential per score; MUFU and the tensor pipe are co-critical).
-// Measured on B200 with this kernel it does not pay (the per-row softmax is
-// latency-bound rather than MUFU-bound), so it is compiled out by default.  2^x = 2^r * q(f) with r = round(x) taken by the 1.5*2^23 rounding
-// trick and f = x - r in [-1/2, 1/2]; q is a cubic fitted here to 2^f by
-// relative-error minimax (max relative error 7.5e-5, far below the 2^-9
-// rounding of P to bf16); 2^r is added into the exponent field as an integer.
-// Arguments below -125 give exactly 0 (masked scores are -inf).
+// exp2 on the FMA pipe for kExpEmu16 of every 16 score columns, which takes that
+// share of the exponentials off the MUFU pipe (one exponential per score).
+// 2^x = 2^r * q(f): r = round(x) by the 1.5 * 2^23 rounding trick, f = x - r in
+// [-1/2, 1/2], q the cubic that minimises the maximum relative error of q(f) / 2^f
+// on that interval (Lawson's iteratively reweighted least squares, fp32
+// coefficients; fit_exp2_poly.py beside this file reproduces them): max relative
+// error 7.5e-5, far below the 2^-9 rounding of P to bf16.  2^r is added into the
+// exponent field as an integer.  Arguments are clamped to -126 first, so -inf
+// (a masked score) gives at most 2^-126, which no output can resolve.
 #ifndef VKV_EXP_EMU16
-#define VKV_EXP_EMU16 0
+#define VKV_EXP_EMU16 4
 #endif
 constexpr int kExpEmu16 = VKV_EXP_EMU16;
+
+// L2 prefetch of the earlier branch's split rows before the final epilogue (1 = on).
+#ifndef VKV_EPI_PREFETCH
+#define VKV_EPI_PREFETCH 1
+#endif
+
 
 // Development timeline (compiled only with -DVKV_TRACE): SM clock stamps of the
 // pipeline events of CTA 0, read back with vkv_debug_trace().
@@ -771,10 +778,12 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               const uint32_t slot = item % NS, use = item / NS;
               if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
               if (!ok) break;
+#ifdef VKV_TEST_AIDS
               if (item == 0 && p.withhold_first_copy) {
                 ++item;  // test aid: this copy never arrives, so the wait for it runs out
                 continue;
               }
+#endif
               VKV_STAMP(20480 + (int)item);
               mbar_arrive_expect_tx(b_full0 + 8 * slot, (uint32_t)C::KV_BYTES);
               const CUtensorMap* tm = kv ? &p.tm_v : &p.tm_k;
@@ -1110,6 +1119,20 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           VKV_STAMP(tr < 0 ? -1 : tr + 5);
           if (lane == 0) mbar_arrive(b_pfull);
           ++np;
+        }
+        if (VKV_EPI_PREFETCH && ok && !u.piece && p.om != nullptr && p.n_branches == 2 && !sparse && !ragged &&
+            prev_branch >= 0 && row_ok) {
+          // the earlier branch's fp32 partial (its two split rows, written at its close
+          // long before and likely out of L2) is read by the epilogue below: bring it
+          // into L2 while the last PV product completes
+          const __nv_bfloat16* mr = p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh;
+          const __nv_bfloat16* pr = p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
+                                    (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch];
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 64) {
+            prefetch_l2(mr + c0);
+            prefetch_l2(pr + c0);
+          }
         }
         if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
         if (ok && !u.piece) {

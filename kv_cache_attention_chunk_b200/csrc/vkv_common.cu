@@ -76,6 +76,7 @@ bool encode_tmap_bf16_4d_swizzle(CUtensorMap* tm, const void* ptr, const uint64_
   return r == CUDA_SUCCESS;
 }
 
+#ifdef VKV_TEST_AIDS
 namespace {
 std::atomic<int> g_withhold{0};
 }  // namespace
@@ -87,6 +88,7 @@ bool take_withhold_request() {
   }
   return false;
 }
+#endif
 
 bool tensor_aligned(const vkv_tensor& t) {
   return (reinterpret_cast<uintptr_t>(t.ptr) & 15u) == 0 && (t.sb % 8) == 0 && (t.st % 8) == 0 &&
@@ -126,8 +128,11 @@ extern "C" int32_t vkv_abi_sizeof(int32_t which) {
   return -1;
 }
 
+#ifdef VKV_TEST_AIDS
+// Test build only (vkv_test.h).
 extern "C" vkv_status vkv_debug_withhold_copy(int32_t n_calls) {
   if (n_calls < 0) return VKV_ERR_SHAPE;
   vkv::g_withhold.store(n_calls);
   return VKV_OK;
 }
+#endif

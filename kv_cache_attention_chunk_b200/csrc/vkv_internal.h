@@ -57,7 +57,7 @@ struct AttnParams {
   long long om_sb, om_st, om_sh;
   float* lsem;
   int* err;
-  int withhold_first_copy;  // test aid: the producer skips its first K/V copy (see vkv_debug_withhold_copy)
+  int withhold_first_copy;  // test build only: the producer skips its first K/V copy (vkv_debug_withhold_copy)
   // key-axis pieces: per workspace slot, the partial outputs (O / l, fp32)
   // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (natural log)
   // [slot][tile][branch][row]
@@ -96,8 +96,11 @@ int device_sm_count(int* dev_out);                // -1 when no usable sm_100 de
 bool encode_tmap_bf16_4d(CUtensorMap* tm, const void* ptr, const uint64_t dims[4],
                          const uint64_t strides_bytes[3], const uint32_t box[4]);
 bool tensor_aligned(const vkv_tensor& t);
-// Test aid (vkv_common.cu): true when the calling launch should withhold its first
-// cache-tile copy (consumes one of the calls armed by vkv_debug_withhold_copy).
+#ifdef VKV_TEST_AIDS
+// Test aid (vkv_common.cu, test build only): true when the calling launch should
+// withhold its first cache-tile copy (consumes one of the calls armed by
+// vkv_debug_withhold_copy).
 bool take_withhold_request();
+#endif
 
 }  // namespace vkv

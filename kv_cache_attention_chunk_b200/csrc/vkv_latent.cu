@@ -94,7 +94,7 @@ struct LatParams {
   long long o_sb, o_st, o_sh;
   float* lse;  // optional [B, H, Lq]
   int* err;
-  int withhold_first_copy;  // test aid (vkv_debug_withhold_copy)
+  int withhold_first_copy;  // test build only (vkv_debug_withhold_copy)
   int B, H, Lq, Lkv, n_qt, n_tiles;
   float scale_log2;
 };
@@ -252,10 +252,12 @@ __global__ void __launch_bounds__(256, 1) latent_attn_kernel(const __grid_consta
           const uint32_t slot = item % C::NSLOT, use = item / C::NSLOT;
           if (use > 0) ok = mbar_wait(b_empty0 + 8 * slot, (use - 1) & 1, abort_flag, p.err);
           if (!ok) break;
+#ifdef VKV_TEST_AIDS
           if (item == 0 && p.withhold_first_copy) {
             ++item;  // test aid: this copy never arrives, so the wait for it runs out
             continue;
           }
+#endif
           const uint32_t bar = b_full0 + 8 * slot;
           const uint32_t dst = sKV + slot * C::TILE;
           mbar_arrive_expect_tx(bar, (uint32_t)C::TILE);
@@ -583,7 +585,9 @@ extern "C" vkv_status vkv_latent_attn(const vkv_latent_args* a, vkv_stream_t str
   P.o_sh = a->o.sh;
   P.lse = a->lse;
   P.err = a->err_word;
+#ifdef VKV_TEST_AIDS
   P.withhold_first_copy = take_withhold_request() ? 1 : 0;
+#endif
   P.B = a->B;
   P.H = a->H;
   P.Lq = a->Lq;

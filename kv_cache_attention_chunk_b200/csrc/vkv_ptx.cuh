@@ -356,6 +356,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// Bring the 128-byte line holding `p` into L2 (no register is written).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Programmatic dependent launch: the kernel launched after this one on the
 // stream (with the programmatic-serialization attribute) may start once every
 // CTA of this grid has executed launch_dependents or exited; it must call

@@ -14,6 +14,7 @@ Convenience wrappers that allocate outputs with torch: ``chunk_attn_segments``,
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from ctypes import POINTER, c_float, c_int32, c_int64, c_size_t, c_void_p
@@ -22,6 +23,7 @@ import numpy as np
 import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvkv.so")
+LIB_TEST_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvkv_test.so")
 
 MODE_SEGMENTS, MODE_BLOCK_SPARSE, MODE_RAGGED = 0, 1, 2
 MAX_BRANCHES, MAX_SEGMENTS = 2, 8
@@ -126,17 +128,48 @@ class vkv_schedule(ctypes.Structure):
 
 
 _lib = None
+_test_lib = None
 
 
 def lib() -> ctypes.CDLL:
     """Load libvkv.so (built in-tree by kv_cache_attention_chunk_b200.build); raise if absent."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_attention_chunk_b200.build`"
+    if _lib is None:
+        _lib = _load(LIB_PATH)
+    return _lib
+
+
+def test_lib() -> ctypes.CDLL:
+    """Load the test build libvkv_test.so: the same library plus the test aids of
+    include/vkv_test.h (vkv_debug_withhold_copy)."""
+    global _test_lib
+    if _test_lib is None:
+        L = _load(LIB_TEST_PATH)
+        L.vkv_debug_withhold_copy.argtypes = [c_int32]
+        L.vkv_debug_withhold_copy.restype = c_int32
+        L.vkv_debug_exp2_poly.argtypes = [c_void_p, c_void_p, c_int32, c_void_p]
+        L.vkv_debug_exp2_poly.restype = c_int32
+        _test_lib = L
+    return _test_lib
+
+
+@contextlib.contextmanager
+def using_test_library():
+    """Route the calls of this module through the test build while the block runs."""
+    global _lib
+    saved = lib()
+    _lib = test_lib()
+    try:
+        yield _lib
+    finally:
+        _lib = saved
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m kv_cache_attention_chunk_b200.build`"
                            " (there is no fallback implementation)")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     L.vkv_chunk_attn.argtypes = [POINTER(vkv_attn_args), c_void_p]
     L.vkv_chunk_attn.restype = c_int32
     L.vkv_chunk_attn_workspace_size.argtypes = [POINTER(vkv_attn_args)]
@@ -171,14 +204,11 @@ def lib() -> ctypes.CDLL:
     L.vkv_persist_update.restype = c_int32
     L.vkv_latent_attn.argtypes = [POINTER(vkv_latent_args), c_void_p]
     L.vkv_latent_attn.restype = c_int32
-    L.vkv_debug_withhold_copy.argtypes = [c_int32]
-    L.vkv_debug_withhold_copy.restype = c_int32
     for i, st in enumerate((vkv_attn_args, vkv_select_args, vkv_tensor, vkv_segment, vkv_compact_args,
                             vkv_head_rule, vkv_persist_args, vkv_latent_args, vkv_schedule)):
         if L.vkv_abi_sizeof(i) != ctypes.sizeof(st):
             raise RuntimeError(f"ABI mismatch for {st.__name__}: C {L.vkv_abi_sizeof(i)} B, "
                                f"binding {ctypes.sizeof(st)} B")
-    _lib = L
     return L
 
 
@@ -242,8 +272,9 @@ def vkv_latent_attn(args: vkv_latent_args, stream: int | None) -> int:
 
 
 def vkv_debug_withhold_copy(n_calls: int) -> int:
-    """Test aid: the next n_calls attention launches withhold their first cache-tile copy."""
-    return int(lib().vkv_debug_withhold_copy(int(n_calls)))
+    """Test aid of the test build (include/vkv_test.h): the next n_calls attention
+    launches of libvkv_test.so withhold their first cache-tile copy."""
+    return int(test_lib().vkv_debug_withhold_copy(int(n_calls)))
 
 
 def vkv_compact_rows(args: vkv_compact_args) -> int:

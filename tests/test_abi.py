@@ -26,8 +26,8 @@ def _built():
     vkv.lib()
 
 
-def declared_functions():
-    src = open(os.path.join(ROOT, "include", "vkv.h")).read()
+def declared_functions(header="vkv.h"):
+    src = open(os.path.join(ROOT, "include", header)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(vkv_\w+)\s*\(", src)))
 
@@ -38,6 +38,21 @@ def test_exports_every_declared_function():
     L = vkv.lib()
     for n in names:
         assert hasattr(L, n), f"{n} declared in vkv.h but not exported"
+
+
+def test_test_aids_only_in_the_test_build():
+    """include/vkv_test.h is exported by libvkv_test.so (which also exports all of
+    vkv.h) and by no means by the production libvkv.so."""
+    aids = declared_functions("vkv_test.h")
+    assert aids == ["vkv_debug_exp2_poly", "vkv_debug_withhold_copy"]
+    T_ = vkv.test_lib()
+    for n in aids + declared_functions():
+        assert hasattr(T_, n), f"{n} not exported by the test build"
+    prod = ctypes.CDLL(vkv.LIB_PATH)
+    for n in aids:
+        assert not hasattr(prod, n), f"{n} is a test aid but the production library exports it"
+    headers = sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
+    assert headers == ["vkv.h", "vkv_test.h"]
 
 
 def test_struct_layouts_match_binding():

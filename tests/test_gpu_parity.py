@@ -161,14 +161,16 @@ def test_stalled_pipeline_reports_timeout_and_device_stays_usable():
     c = W.cfg_tiny()
     q, k, vv = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
     err = err_word()
-    assert v.vkv_debug_withhold_copy(1) == 0
-    try:
-        v.chunk_attn_segments(q, k, vv, c.branches, scale=c.scale, err=err)
-        torch.cuda.synchronize()
-    finally:
-        v.vkv_debug_withhold_copy(0)
-    assert int(err.item()) == v.DEVERR_TIMEOUT
-    check_segments_full(c, run_segments(c))
+    with v.using_test_library():  # the test aid exists only in the test build
+        assert v.vkv_debug_withhold_copy(1) == 0
+        try:
+            v.chunk_attn_segments(q, k, vv, c.branches, scale=c.scale, err=err)
+            torch.cuda.synchronize()
+        finally:
+            v.vkv_debug_withhold_copy(0)
+        assert int(err.item()) == v.DEVERR_TIMEOUT
+        check_segments_full(c, run_segments(c))
+    check_segments_full(c, run_segments(c))  # and the production library on the same context
 
 
 # ---------------------------------------------------------------------------
