@@ -237,8 +237,10 @@ vkv_status vkv_debug_schedule(const vkv_attn_args* args, int32_t n_sm, int32_t s
  * the lower block id first.  out_scores [B*H][ceil(Lq/block)][n_win_blk]
  * (optional, fp32) receives every score.
  * `workspace` is DEVICE scratch of at least vkv_block_select_workspace_size()
- * bytes, 256-byte aligned, owned by the caller; its contents need no
- * initialisation and are dead after the call.
+ * bytes (the window blocks' means: B*H*n_win_blk*d*4, rounded up to 256),
+ * 256-byte aligned, owned by the caller; its contents need no initialisation
+ * and are dead after the call.  It is not used, and may be NULL, when `kbar`
+ * supplies the window means (the query blocks are pooled on chip).
  */
 typedef struct {
   int32_t B, H, d, block; /* d in {64, 128}; block = 64                       */
@@ -292,16 +294,20 @@ vkv_status vkv_block_pool(vkv_tensor x, int32_t B, int32_t L, int32_t H, int32_t
  * through this C interface alone and cannot size and own a workspace).
  *
  * Same arguments, results and errors as vkv_block_select, except that
- * `workspace` / `workspace_bytes` are ignored: the pooled block vectors go to
- * a fixed scratch array inside the library, VKV_NOALLOC_SCRATCH_BYTES in size,
- * which every GPU that loads the library holds until the process exits.
+ * `workspace` / `workspace_bytes` are ignored: the pooled window block vectors
+ * go to a fixed scratch array inside the library, VKV_NOALLOC_SCRATCH_BYTES in
+ * size, which every GPU that loads the library holds until the process exits.
  * Requests whose vkv_block_select_workspace_size() exceeds that size return
- * VKV_ERR_WORKSPACE.  The call allocates nothing (no cudaMalloc / cudaFree).
- * The first call on a device looks up the array's device address on that
- * device (cudaGetSymbolAddress); make that first call before any stream
- * capture.  All calls on a device share the array and leave the last call's
- * contents in it; calls that overlap on the GPU (e.g. on two streams at once)
- * race on it.  Nothing in it needs clearing between calls.
+ * VKV_ERR_WORKSPACE; calls that pass cached window means in `kbar` use no
+ * scratch and are never refused for size.  The call allocates nothing (no
+ * cudaMalloc / cudaFree).  The first call on a device looks up the array's
+ * device address on that device (cudaGetSymbolAddress) and keeps it; make that
+ * first call before any stream capture, and do not call this entry point again
+ * after a cudaDeviceReset of that device in the same process (the kept address
+ * belongs to the context that was reset).  All calls on a device share the
+ * array and leave the last call's contents in it; calls that overlap on the
+ * GPU (e.g. on two streams at once) race on it.  Nothing in it needs clearing
+ * between calls.
  */
 #define VKV_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
 vkv_status vkv_block_select_noalloc(const vkv_select_args* args, vkv_stream_t stream);
@@ -448,17 +454,6 @@ typedef struct {
 } vkv_latent_args;
 
 vkv_status vkv_latent_attn(const vkv_latent_args* args, vkv_stream_t stream);
-
-/*
- * vkv_debug_withhold_copy -- test aid for the bounded pipeline waits.  The next
- * n_calls launches of vkv_chunk_attn or vkv_latent_attn (in any thread) run with
- * the first cache-tile copy of every CTA withheld: the wait for it runs out
- * after its time limit (1 s), the kernel stops its work, lets the copies it did
- * issue land, releases its resources and writes VKV_DEVERR_TIMEOUT to err_word;
- * the outputs of that launch are incomplete and the device stays usable.
- * n_calls = 0 disarms it.  Returns VKV_ERR_SHAPE for n_calls < 0.
- */
-vkv_status vkv_debug_withhold_copy(int32_t n_calls);
 
 /* Human-readable name of a status code (static storage). */
 const char* vkv_status_string(vkv_status s);

@@ -37,48 +37,92 @@ struct SelParams {
   int H, Lq, n_qblk, n_win, topk;
   int* out_idx;
   float* out_scores;
+  int* err;
+  int stage;  // the head's window means are copied to shared memory (they fit)
 };
 
-constexpr int kSelQ = 4;  // query blocks per CTA
+constexpr int kSelQ = 4;                    // query blocks per CTA (one warp each for the top-K)
+constexpr int kSelStageBytes = 96 * 1024;   // largest staged window (n_win * D * 4 bytes)
 
+// Shared memory of the selection kernel (bytes): the staged window means
+// [n_win][D] fp32 (when they fit in kSelStageBytes), the pooled queries
+// [kSelQ][D] fp32, the row-group partial sums [G][kSelQ * D] fp32 -- whose space
+// later holds the ranking keys [kSelQ][n_win] uint32 --, one 256-bin digit
+// histogram per query block, an mbarrier and an abort flag.
 template <int D>
-constexpr size_t sel_smem_bytes() {
-  // pooled queries + (row-group partial sums | 64-bit ranking keys) + kept bitmaps
-  constexpr size_t part = (size_t)(256 / (D / 8)) * kSelQ * D * sizeof(float);
-  constexpr size_t keys = (size_t)kSelQ * 1024 * sizeof(unsigned long long);
-  return (size_t)kSelQ * D * sizeof(float) + (part > keys ? part : keys) + (size_t)kSelQ * 32 * sizeof(uint32_t);
+constexpr size_t sel_part_bytes() { return (size_t)(256 / (D / 8)) * kSelQ * D * sizeof(float); }
+template <int D>
+constexpr int sel_row_stride() { return D + 4; }  // floats per staged row: conflict-free column reads
+template <int D>
+size_t sel_smem_bytes(int n_win, bool stage) {
+  return (stage ? (size_t)n_win * sel_row_stride<D>() * sizeof(float) : 0) + (size_t)kSelQ * D * sizeof(float) +
+         sel_part_bytes<D>() + (size_t)kSelQ * 256 * sizeof(int) + 16;
 }
 
 // grid: x = ceil(n_qblk / kSelQ), y = b*H + h; 256 threads.
+//  0. After the window pooling kernel before it (if any) has completed, warp 0
+//     starts one bulk copy per window block mean into shared memory (when they
+//     fit), into rows padded to d + 4 floats; they land while the query blocks
+//     are pooled.
 //  1. Pool the CTA's kSelQ query blocks from q: thread (g, c) sums 16-byte column
 //     chunk c of rows g, g + G, ... of every block (all loads in flight at
 //     once), the row groups are added in shared memory, then divided by the
-//     block's row count.  This reads only q, so it runs before the wait for the
-//     window pooling kernel (a programmatic dependent launch overlaps the two).
-//  2. Thread w scores window block w against the kSelQ pooled queries, its
-//     block mean read once from global memory (L2).  NaN scores rank last and
-//     -0 counts as +0, so equal scores tie on the block index.
-//  3. Exact top-K by counting: each score becomes a unique 64-bit key (the
-//     order-preserving integer image of the score, then 1023 - w, so that of
-//     equal scores the lower block id ranks higher); a block is kept when fewer
-//     than topk keys of its query block exceed its own.  Kept blocks are marked
-//     in a bitmap and written in ascending order (their rank among kept ids).
+//     block's row count.
+//  2. Thread w scores window block w against the kSelQ pooled queries from its
+//     staged row (the padding puts the rows of a quarter-warp in different
+//     banks; every row is summed in the same order, so equal block means give
+//     equal scores); without staging, a warp reads whole block means from
+//     global memory and adds the lanes' partial products by shuffles.  NaN
+//     scores rank last and -0 counts as +0, so equal scores tie on the block
+//     index.  A score becomes its order-preserving 32-bit integer image (larger
+//     score, larger key).
+//  3. Warp q selects the top-K of query block q on its own (warp barriers only):
+//     radix selection of the K-th largest key, 8 bits a pass (4 passes): the
+//     keys still in play (those sharing the threshold's digits found so far)
+//     are counted per digit in the warp's shared-memory histogram, one atomic
+//     per distinct digit and chunk of 32 keys; the lanes scan it from the top and
+//     fix the next digit (where the running count reaches the number still to
+//     take).  Then, in ascending block order, every key above the threshold is
+//     kept, and of the keys equal to it the lowest ids, as many as are still to
+//     take; a ballot gives each kept block its output position.
 template <int D>
 __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
-  constexpr int CPR = D / 8;     // 16-byte chunks per row
+  constexpr int CPR = D / 8;     // 16-byte chunks per row (bf16)
   constexpr int G = 256 / CPR;   // row groups
   constexpr int RPT = 64 / G;    // rows per thread and block
+  constexpr int CH = D / 4;      // 16-byte chunks per block mean (fp32)
   extern __shared__ __align__(16) uint8_t sel_sm[];
-  float* qs = reinterpret_cast<float*>(sel_sm);                                   // [kSelQ][D]
-  float* part = qs + kSelQ * D;                                                   // [G][kSelQ * D]
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part);        // [kSelQ][n_win] (after part)
-  constexpr size_t kUnion = sel_smem_bytes<D>() - (size_t)kSelQ * D * sizeof(float) - kSelQ * 32 * sizeof(uint32_t);
-  uint32_t* kept = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(part) + kUnion);  // [kSelQ][32]
+  constexpr int RS = sel_row_stride<D>();
+  const size_t stage_bytes = p.stage ? (size_t)p.n_win * RS * sizeof(float) : 0;
+  float* kbs = reinterpret_cast<float*>(sel_sm);                                      // [n_win][D + 4] (staged)
+  float* qs = reinterpret_cast<float*>(sel_sm + stage_bytes);                         // [kSelQ][D]
+  float* part = qs + kSelQ * D;                                                       // [G][kSelQ * D]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(part);                                 // [kSelQ][n_win] (after part)
+  int* hist = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(part) + sel_part_bytes<D>());  // [kSelQ][256]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hist + kSelQ * 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
   const int s = blockIdx.y;
   const int b = s / p.H, h = s - (s / p.H) * p.H;
   const int j0 = blockIdx.x * kSelQ;
   const int nq = min(kSelQ, p.n_qblk - j0);
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const uint32_t b_kb = smem_u32(bar);
+  const float* kb_head = p.kbar + (size_t)s * p.n_win * D;
+  if (tid == 0) {
+    mbar_init(b_kb, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the window pooling kernel before this one (if any) has completed
+  if (p.stage && warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(b_kb, (uint32_t)(p.n_win * D * sizeof(float)));
+    __syncwarp();
+    for (int w = lane; w < p.n_win; w += 32)
+      bulk_load(smem_u32(kbs + (size_t)w * RS), kb_head + (size_t)w * D, (uint32_t)(D * sizeof(float)), b_kb);
+  }
+  // 1. pooled query blocks
   {
     const int c = tid % CPR, g = tid / CPR;
     const __nv_bfloat16* base = p.q + b * p.q_sb + h * p.q_sh;
@@ -111,7 +155,6 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
   }
-  if (tid < kSelQ * 32) kept[tid] = 0u;
   __syncthreads();
   for (int x = tid; x < kSelQ * D; x += 256) {
     const int q = x / D;
@@ -122,53 +165,149 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
     qs[x] = sum * (1.f / (float)nrows);
   }
   __syncthreads();  // part is dead from here on: its space holds the keys
-  griddep_wait();   // the window pooling kernel before this one (if any) has completed
-  for (int w = tid; w < p.n_win; w += 256) {
-    const float4* kr = reinterpret_cast<const float4*>(p.kbar + ((size_t)s * p.n_win + w) * D);
-    float acc[kSelQ][4];
+  // 2. scores
+  if (p.stage) {
+    if (!mbar_wait(b_kb, 0, abort_flag, p.err)) {
+      // the copy did not arrive in time: let it land before the CTA exits
+      if (tid == 0) mbar_wait_drain(b_kb, 0);
+      return;
+    }
+    for (int w = tid; w < p.n_win; w += 256) {
+      const float4* kr = reinterpret_cast<const float4*>(kbs + (size_t)w * RS);
+      float acc[kSelQ][4];
 #pragma unroll
-    for (int q = 0; q < kSelQ; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+      for (int q = 0; q < kSelQ; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
 #pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const float4 kv = __ldg(kr + c4);
+      for (int cc = 0; cc < CH; ++cc) {
+        const float4 kv = kr[cc];
+#pragma unroll
+        for (int q = 0; q < kSelQ; ++q) {
+          const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[cc];
+          acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
+          acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
+          acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
+          acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+        }
+      }
 #pragma unroll
       for (int q = 0; q < kSelQ; ++q) {
-        const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[c4];
-        acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
-        acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
-        acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
-        acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+        float v = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
+        v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+        if (q < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + q) * p.n_win + w] = v;
+        const uint32_t u = __float_as_uint(v);
+        keys[q * p.n_win + w] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);
       }
     }
+  } else {
+    // a warp reads whole block means (lane l: 16-byte chunk l % CH of row w0 + l / CH),
+    // six rows of each lane in flight; the lanes' partial products are added by shuffles
+    constexpr int RPW = 32 / CH;
+    constexpr int kRows = 6;
+    const int c = lane % CH, rsub = lane / CH;
+    for (int w0 = warp * RPW; w0 < p.n_win; w0 += 8 * RPW * kRows) {
+      float4 kv[kRows];
 #pragma unroll
-    for (int q = 0; q < kSelQ; ++q) {
-      float sc = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
-      sc = (sc != sc) ? -INFINITY : (sc == 0.f ? 0.f : sc);
-      if (q < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + q) * p.n_win + w] = sc;
-      const uint32_t u = __float_as_uint(sc);
-      const uint32_t ok = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);  // larger score -> larger key
-      keys[q * p.n_win + w] = ((unsigned long long)ok << 10) | (unsigned long long)(1023 - w);
+      for (int i = 0; i < kRows; ++i) {
+        const int w = w0 + i * 8 * RPW + rsub;
+        kv[i] = w < p.n_win ? __ldg(reinterpret_cast<const float4*>(kb_head + (size_t)w * D) + c)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int w = w0 + i * 8 * RPW + rsub;
+        float sc[kSelQ];
+#pragma unroll
+        for (int q = 0; q < kSelQ; ++q) {
+          const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[c];
+          sc[q] = fmaf(qv.x, kv[i].x, fmaf(qv.y, kv[i].y, fmaf(qv.z, kv[i].z, qv.w * kv[i].w)));
+        }
+#pragma unroll
+        for (int o = CH / 2; o > 0; o >>= 1)
+#pragma unroll
+          for (int q = 0; q < kSelQ; ++q) sc[q] += __shfl_xor_sync(0xFFFFFFFFu, sc[q], o);
+        if (c < kSelQ && w < p.n_win) {
+          float v = sc[0];
+#pragma unroll
+          for (int q = 1; q < kSelQ; ++q) v = (c == q) ? sc[q] : v;
+          v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+          if (c < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + c) * p.n_win + w] = v;
+          const uint32_t u = __float_as_uint(v);
+          keys[c * p.n_win + w] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);
+        }
+      }
     }
   }
   __syncthreads();
-  const int npairs = nq * p.n_win;
-  for (int x = tid; x < npairs; x += 256) {
-    const int q = x / p.n_win, w = x - q * p.n_win;
-    const unsigned long long* kq = keys + q * p.n_win;
-    const unsigned long long kw = kq[w];
-    int above = 0;
-    for (int v = 0; v < p.n_win; ++v) above += kq[v] > kw ? 1 : 0;
-    if (above < p.topk) atomicOr(&kept[q * 32 + (w >> 5)], 1u << (w & 31));
+  // 3. warp q: top-K of query block q
+  if (warp >= nq) return;
+  const uint32_t* kq = keys + warp * p.n_win;
+  int* hq = hist + warp * 256;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t thr = 0u;
+  int need = p.topk;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hq[lane + 32 * i] = 0;
+    __syncwarp();
+    for (int w0 = 0; w0 < p.n_win; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t k = w < p.n_win ? kq[w] : 0u;
+      const bool in_play = w < p.n_win && (k & hi_mask) == thr;
+      const uint32_t digit = in_play ? ((k >> shift) & 255u) : 0xFFFFFFFFu;
+      const unsigned grp = __match_any_sync(0xFFFFFFFFu, digit);
+      if (in_play && (grp & lt) == 0u) atomicAdd(&hq[digit], __popc(grp));
+    }
+    __syncwarp();
+    // lane l holds digits 255 - 8l .. 248 - 8l (lane 0 the largest)
+    int cnt[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cnt[i] = hq[255 - (8 * lane + i)];
+      sum += cnt[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int above = incl - sum;  // keys in play with a digit above this lane's bins
+    const bool mine = above < need && need <= incl;
+    uint32_t digit = 0u;
+    int rest = 0;
+    if (mine) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (above + cnt[i] >= need) {
+          digit = (uint32_t)(255 - (8 * lane + i));
+          rest = need - above;
+          break;
+        }
+        above += cnt[i];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+    thr |= __shfl_sync(0xFFFFFFFFu, digit, src) << shift;
+    need = __shfl_sync(0xFFFFFFFFu, rest, src);
+    __syncwarp();  // the histogram is read before the next pass clears it
   }
-  __syncthreads();
-  for (int x = tid; x < npairs; x += 256) {
-    const int q = x / p.n_win, w = x - q * p.n_win;
-    const uint32_t* kb = kept + q * 32;
-    const uint32_t word = kb[w >> 5];
-    if (!((word >> (w & 31)) & 1u)) continue;
-    int pos = __popc(word & ((1u << (w & 31)) - 1u));
-    for (int i = 0; i < (w >> 5); ++i) pos += __popc(kb[i]);
-    p.out_idx[((size_t)s * p.n_qblk + j0 + q) * p.topk + pos] = w;
+  // keys above the threshold, then the lowest-id keys equal to it, in ascending order
+  int* oi = p.out_idx + ((size_t)s * p.n_qblk + j0 + warp) * p.topk;
+  int written = 0, eq_seen = 0;
+  for (int w0 = 0; w0 < p.n_win; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t k = w < p.n_win ? kq[w] : 0u;
+    const bool valid = w < p.n_win;
+    const bool eq = valid && k == thr;
+    const uint32_t beq = __ballot_sync(0xFFFFFFFFu, eq);
+    const bool keep = valid && (k > thr || (eq && eq_seen + __popc(beq & lt) < need));
+    eq_seen += __popc(beq);
+    const uint32_t bk = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) oi[written + __popc(bk & lt)] = w;
+    written += __popc(bk);
   }
 }
 
@@ -236,10 +375,23 @@ bool launch_order(const int* sel, int* order, int BH, int n_qblk, int topk, cuda
 // when one runs just before it (`after_pool`), else as an ordinary launch.
 template <int D>
 bool launch_select_t(dim3 g, bool after_pool, cudaStream_t st, const SelParams& sp) {
+  static std::mutex mu;
+  static unsigned long long attr_done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && !(attr_done & (1ull << dev))) {
+      if (cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)sel_smem_bytes<D>(kSelStageBytes / (D * 4), true)) != cudaSuccess)
+        return false;
+      attr_done |= 1ull << dev;
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = g;
   cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = sel_smem_bytes<D>();
+  cfg.dynamicSmemBytes = sel_smem_bytes<D>(sp.n_win, sp.stage != 0);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -324,6 +476,11 @@ vkv_status run_select(const vkv_select_args* a, float* kbar_scratch, cudaStream_
   sp.topk = a->topk;
   sp.out_idx = a->out_idx;
   sp.out_scores = a->out_scores;
+  sp.err = a->err_word;
+  // the head's window means are staged in shared memory when they fit (16-byte
+  // aligned source: every head's block holds n_win * d floats)
+  const size_t wbytes = (size_t)a->n_win_blk * (a->d + 4) * sizeof(float);
+  sp.stage = (wbytes <= (size_t)kSelStageBytes && (reinterpret_cast<uintptr_t>(sp.kbar) & 15u) == 0) ? 1 : 0;
   const dim3 sg((n_qblk + kSelQ - 1) / kSelQ, BH);
   if (!launch_select(a->d, sg, pool_win, st, sp)) return VKV_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;

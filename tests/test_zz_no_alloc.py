@@ -42,7 +42,7 @@ def _args(B, H, Lq, Lkv, window_blk0, n_win_blk, topk, q_ptr, k_ptr, q_strides, 
 
 
 def test_noalloc_refuses_requests_larger_than_its_scratch():
-    # 2 x 40 heads x (512 + 1024) blocks x 128 x 4 B = 62.9 MB > 4 MiB: refused before any device work
+    # 2 x 40 heads x 1024 window blocks x 128 x 4 B = 41.9 MB > 4 MiB: refused before any device work
     need = vkv.vkv_block_select_workspace_size(2, 40, 512 * 64, 1024, 64, 128)
     assert need > vkv.NOALLOC_SCRATCH_BYTES
     a = _args(2, 40, 512 * 64, 2048 * 64, 1024, 1024, 9, 0x10000, 0x10000,
@@ -50,24 +50,58 @@ def test_noalloc_refuses_requests_larger_than_its_scratch():
     assert vkv.vkv_block_select_noalloc(a, None) == 7  # VKV_ERR_WORKSPACE
 
 
+def _case(seed, H, win_frames):
+    return W.make_block_sparse("noalloc", seed=seed, H=H, d=128, frame_tokens=1536, block=64,
+                               hist_frames=4, win_frames=win_frames, q_frames=3, n_persist=4)
+
+
+def _noalloc_call(c, q, k, topk, kbar=None, order=False):
+    dev = q.device
+    idx = torch.full((c.B * c.H, c.n_qblk, topk), -1, dtype=torch.int32, device=dev)
+    sc = torch.full((c.B * c.H, c.n_qblk, c.n_win_blk), float("nan"), dtype=torch.float32, device=dev)
+    a = _args(c.B, c.H, c.Lq, c.k.shape[1], c.window_blk0, c.n_win_blk, topk, q.data_ptr(), k.data_ptr(),
+              (q.stride(0), q.stride(1), q.stride(2)), (k.stride(0), k.stride(1), k.stride(2)),
+              idx.data_ptr(), sc.data_ptr())
+    od = None
+    if kbar is not None:
+        a.kbar = kbar.data_ptr()
+    if order:
+        od = torch.full((c.B * c.H, c.n_qblk), -1, dtype=torch.int32, device=dev)
+        a.out_order = od.data_ptr()
+    assert vkv.vkv_block_select_noalloc(a, torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    return idx, sc, od
+
+
 @pytest.mark.gpu
-def test_noalloc_matches_workspace_entry_point_twice():
+def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
+    """Calls in a row share the scratch array: a large call, then a smaller one with the
+    same top-K on other inputs (if it read anything the first call left behind, its
+    sets would differ from the workspace entry point's), then the first again."""
     dev = "cuda:0"
-    outs = []
-    for seed, topk in ((2, 9), (5, 36)):  # two calls in a row with different inputs
-        c = W.make_block_sparse("noalloc", seed=seed, H=12, d=128, frame_tokens=1536, block=64,
-                                hist_frames=4, win_frames=6, q_frames=3, n_persist=4)
+    for seed, H, win in ((2, 12, 6), (5, 3, 4), (2, 12, 6)):
+        c = _case(seed, H, win)
         q, k = c.q.to(dev), c.k.to(dev)
-        ref_idx, ref_sc = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, topk, scores=True)
-        n_qblk = c.n_qblk
-        idx = torch.full((c.B * c.H, n_qblk, topk), -1, dtype=torch.int32, device=dev)
-        sc = torch.full((c.B * c.H, n_qblk, c.n_win_blk), float("nan"), dtype=torch.float32, device=dev)
-        a = _args(c.B, c.H, c.Lq, c.k.shape[1], c.window_blk0, c.n_win_blk, topk, q.data_ptr(), k.data_ptr(),
-                  (q.stride(0), q.stride(1), q.stride(2)), (k.stride(0), k.stride(1), k.stride(2)),
-                  idx.data_ptr(), sc.data_ptr())
-        assert vkv.vkv_block_select_noalloc(a, torch.cuda.current_stream().cuda_stream) == 0
-        torch.cuda.synchronize()
-        assert torch.equal(idx, ref_idx)
-        assert torch.allclose(sc, ref_sc, rtol=0, atol=1e-5)
-        outs.append(idx.cpu().numpy())
-    assert not np.array_equal(outs[0][:, :, :9], outs[1][:, :, :9])
+        ref_idx, ref_sc = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, 9, scores=True)
+        idx, sc, _ = _noalloc_call(c, q, k, 9)
+        assert torch.equal(idx, ref_idx), (seed, H, win)
+        assert torch.equal(sc, ref_sc), (seed, H, win)  # same kernels: the same bits
+
+
+@pytest.mark.gpu
+def test_noalloc_with_cached_representatives_and_order():
+    """The two other paths through the selection: window means passed in (kbar, no
+    scratch needed) and the query-block order; idx, scores and order equal the
+    workspace entry point's."""
+    dev = "cuda:0"
+    c = _case(7, 6, 6)
+    q, k = c.q.to(dev), c.k.to(dev)
+    kbar = vkv.block_pool(k, c.window_blk0, c.n_win_blk)
+    ref_idx, ref_sc, ref_ord = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, 18, scores=True, order=True,
+                                                kbar=kbar)
+    idx, sc, od = _noalloc_call(c, q, k, 18, kbar=kbar, order=True)
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(sc, ref_sc)
+    assert torch.equal(od, ref_ord)
+    idx2, _, od2 = _noalloc_call(c, q, k, 18, order=True)  # pooling the window itself: same sets and order
+    assert torch.equal(idx2, ref_idx) and torch.equal(od2, ref_ord)
