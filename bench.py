@@ -11,9 +11,13 @@ their LSEs plus the LSE-merged output).  One step = one vkv_chunk_attn call.
 Metric: effective TFLOP/s counting 4*d per visited (query, key) pair, its
 fraction of the measured bf16 dense peak, and ms per chunk.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own chunk
-(independent seeds) with no collective on the data path (weak scaling); the
-time is the max over ranks; rank 0 prints one JSON line.
+Multi-GPU (torchrun, one process per GPU): by default every rank runs its own
+chunk (independent seeds) with no collective on the data path (weak scaling).
+--split heads / --split keys instead split ONE chunk over the ranks (strong
+scaling): by head (each rank its heads; --gather all-gathers the merged
+output), or by key range (each rank attends over one part of the key set and
+rank 0 merges the partials it receives with the LSE merge).  The time is the
+max over ranks; rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle on the host cores (bounded samples
 of the same workload); under torchrun only rank 0 runs it.
@@ -111,11 +115,22 @@ def load_peaks():
 ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx.cuh")
 
 
+def headline_split(vkv, q, k, v, branches, scale) -> bool:
+    """True when the call's schedule cuts units along the key axis (a non-zero
+    workspace): the piece-enabled attention instantiation runs, then the combine kernel."""
+    return vkv.vkv_chunk_attn_workspace_size(vkv.segments_args(q, k, v, branches, scale)) > 0
+
+
 def headline_kernel_name(vkv, q, k, v, case) -> str:
-    """The attention instantiation the headline call runs: with piece support when
-    its schedule cuts units along the key axis (a non-zero workspace)."""
-    pc = vkv.vkv_chunk_attn_workspace_size(vkv.segments_args(q, k, v, case.branches, case.scale)) > 0
+    """The attention instantiation the headline call runs."""
+    pc = headline_split(vkv, q, k, v, case.branches, case.scale)
     return f"chunk_attn_kernel<128, 0, {int(pc)}>"
+
+
+def mcycles(ms, clocks):
+    """Milliseconds at the median SM clock under load, as millions of SM cycles."""
+    mhz = (clocks or {}).get("sm_mhz")
+    return ms * mhz / 1000.0 if mhz else None
 
 
 def kernel_source_hash() -> str:
@@ -156,7 +171,7 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 100):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.idx, self.period, self.proc, self.out = gpu_index, period_ms, None, ""
 
     def start(self):
@@ -495,6 +510,9 @@ def run_ours(args):
     value = world * fl / (ms_step * 1e-3) / 1e12
     avg_launch = statistics.mean(launch_ms)
     achieved = fl / (avg_launch * 1e-3) / 1e12
+    # our kernels per step: the attention kernel, and the piece combine kernel behind
+    # it when the schedule cuts units along the key axis
+    launches_per_step = 2 if headline_split(vkv, q, k, v, case.branches, case.scale) else 1
     peak = float(peaks["bf16_tflops"])
     peak_sus = float(peaks.get("bf16_tflops_sustained", 0.0)) or None
 
@@ -581,15 +599,136 @@ def run_ours(args):
         "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pipeline": "two buffer sets; upload, call and read-back of consecutive steps overlap"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
     }
+    line["roofline"]["launch_mcycles_median"] = mcycles(line["roofline"]["launch_ms_median"], clocks)
+    line["config"]["mcycles_per_chunk"] = mcycles(ms_step, clocks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if world == 1 and not args.no_extras:
         del q, k, v, out, q2, k2, v2, out2, sets
         torch.cuda.empty_cache()
         line["modes"] = extras(dev, peaks)
+    barrier()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_split(args):
+    """ONE headline chunk split over the ranks (strong scaling): by head or by key range."""
+    from kv_cache_attention_chunk_b200 import build, shard, vkv
+    rank, local, world = dist_setup()
+    if local == 0:
+        build.build()
+    barrier()
+    vkv.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    case = headline_case(0)  # the same chunk on every rank
+    fl = headline_flops()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nccl = world > 1 and torch.distributed.get_backend() == "nccl"
+    if args.split == "heads":
+        h0, h1 = shard.head_range(case.H, world, rank)
+        host = [t[:, :, h0:h1].contiguous() for t in (case.q, case.k, case.v)]
+        branches, merged = case.branches, True
+        part = f"heads {h0}..{h1 - 1}"
+    else:
+        parts = shard.key_parts(case.branches, world)
+        kr, vr, seg = shard.compact_part(case.k, case.v, parts[rank])
+        host = [case.q, kr, vr]
+        branches, merged = [seg], False
+        part = f"keys {sum(n for _, n in parts[rank])} of {sum(n for br in case.branches for _, n in br)}"
+    q, k, v = (t.to(dev) for t in host)
+    out = vkv.chunk_attn_segments(q, k, v, branches, scale=case.scale, merged=merged, err=err)
+    per_attn = 2 if headline_split(vkv, q, k, v, branches, case.scale) else 1
+
+    def step(q, k, v):
+        res = vkv.chunk_attn_segments(q, k, v, branches, scale=case.scale, merged=merged, err=err, out=out,
+                                      stream=stream)
+        if args.split == "heads":
+            o, l = res["o_merged"], res["lse_merged"]
+            if args.gather:
+                o = shard.gather_heads(o, case.H, rank, world)
+            return o, l
+        return shard.merge_to_rank0(res["o"][0], res["lse"][0], rank, world)
+
+    launches_per_step = per_attn + ((world - 1) if (args.split == "keys" and rank == 0) else 0)
+    for _ in range(args.warmup):
+        step(q, k, v)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(vis.split(",")[local].strip() if vis else local)
+    if rank == 0:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(q, k, v)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev if nccl else "cpu")
+    # end to end: this rank's inputs uploaded from pinned host memory every step, and the
+    # result (rank 0's merged output, or each rank's own heads) read back
+    hp = [t.pin_memory() for t in host]
+    o_ref, l_ref = step(q, k, v)
+    h_out = [o_ref.cpu().pin_memory(), l_ref.cpu().pin_memory()] if (rank == 0 or args.split == "heads") else []
+
+    def e2e_step():
+        for d_, h_ in zip((q, k, v), hp):
+            d_.copy_(h_, non_blocking=True)
+        o, l = step(q, k, v)
+        if h_out:
+            h_out[0].copy_(o, non_blocking=True)
+            h_out[1].copy_(l, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1) / e2e_steps, dev if nccl else "cpu")
+    h2d = sum(t.numel() * t.element_size() for t in hp)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    if rank != 0:
+        barrier()
+        return 0
+    value = fl / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "parallelism": f"{args.split} split of one chunk over {world} GPUs"
+                   + (" + all-gather of the merged output" if args.gather and args.split == "heads" else "")
+                   + (" + send/recv of partials to rank 0 and LSE merges" if args.split == "keys" else ""),
+                   "rank0_part": part, "l2": "no flush: the inputs are larger than L2",
+                   "ms_per_chunk": ms_step, "mcycles_per_chunk": mcycles(ms_step, clocks),
+                   "pct_of_bf16_peak": 100.0 * value / world / peak, "flops_per_chunk": fl},
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / world / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst), per GPU"},
+        "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pipeline": "none (rank 0's bytes)"},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks,
+    }
     barrier()
     print(json.dumps(line), flush=True)
     return 0
@@ -669,6 +808,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-mode timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", choices=["none", "heads", "keys"], default="none",
+                    help="split ONE chunk over the ranks (strong scaling) instead of a chunk per rank")
+    ap.add_argument("--gather", action="store_true", help="--split heads: all-gather the merged output")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -677,7 +819,7 @@ def main(argv=None):
     if args.profile:
         return run_profile(args)
     try:
-        return run_ours(args)
+        return run_split(args) if args.split != "none" else run_ours(args)
     finally:
         import torch.distributed as dist
         if dist.is_available() and dist.is_initialized():

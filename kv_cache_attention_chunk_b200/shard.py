@@ -79,16 +79,35 @@ def _default_merge(o_a, lse_a, o_b, lse_b):
     return vkv.lse_merge(o_a, lse_a, o_b, lse_b)
 
 
+def gather_heads(o, H: int, rank: int, world: int, group=None):
+    """All-gather the ranks' head slices o [B, Lq, h1 - h0, d] into the whole
+    [B, Lq, H, d] on every rank (each slice padded to the largest head count)."""
+    import torch.distributed as dist
+    B, Lq, _, d = o.shape
+    h0, h1 = head_range(H, world, rank)
+    hmax = head_range(H, world, 0)[1]
+    mine = torch.zeros((B, Lq, hmax, d), dtype=o.dtype, device=o.device)
+    mine[:, :, :h1 - h0] = o
+    if world > 1:
+        bufs = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(bufs, mine, group=group)
+    else:
+        bufs = [mine]
+    full = torch.empty((B, Lq, H, d), dtype=o.dtype, device=o.device)
+    for r in range(world):
+        a, b = head_range(H, world, r)
+        full[:, :, a:b] = bufs[r][:, :, :b - a]
+    return full
+
+
 def attend_heads(q, k, v, branches, rank: int, world: int, attn=None, gather: bool = False, group=None):
     """Heads [h0, h1) of this rank (strided views of q, k, v: no copies).
 
     Returns (h0, h1, res, full): res is the attention result for the rank's heads
     (dict o, lse, o_merged, lse_merged, as vkv.chunk_attn_segments returns it);
     full is the merged output of all heads [B, Lq, H, d] gathered from every rank
-    when `gather` (each rank's slice padded to the largest head count for the
-    all-gather), else None.
+    when `gather`, else None.
     """
-    import torch.distributed as dist
     attn = attn or _default_attn_heads
     H = q.shape[2]
     h0, h1 = head_range(H, world, rank)
@@ -96,35 +115,25 @@ def attend_heads(q, k, v, branches, rank: int, world: int, attn=None, gather: bo
     full = None
     if gather:
         o = res["o_merged"] if res.get("o_merged") is not None else res["o"][0]
-        B, Lq, _, d = q.shape
-        hmax = head_range(H, world, 0)[1]
-        mine = torch.zeros((B, Lq, hmax, d), dtype=o.dtype, device=o.device)
-        mine[:, :, :h1 - h0] = o
-        bufs = [torch.empty_like(mine) for _ in range(world)]
-        if world > 1:
-            dist.all_gather(bufs, mine, group=group)
-        else:
-            bufs[0] = mine
-        full = torch.empty((B, Lq, H, d), dtype=o.dtype, device=o.device)
-        for r in range(world):
-            a, b = head_range(H, world, r)
-            full[:, :, a:b] = bufs[r][:, :, :b - a]
+        full = gather_heads(o, H, rank, world, group=group)
     return h0, h1, res, full
 
 
-def attend_key_split(q, k, v, branches, rank: int, world: int, attn=None, merge=None, by_branch: bool = False,
-                     group=None):
-    """Partial attention over this rank's key part; rank 0 merges every part.
+def compact_part(k, v, segments):
+    """This rank's key part as its own compact K/V: the part's rows [B, n, H, d]
+    gathered in order, and the one segment [(0, n)] that covers them (attention
+    over a key set does not depend on where the keys sit in the cache)."""
+    idx = torch.cat([torch.arange(a, a + n, device=k.device) for a, n in segments]) if segments else \
+        torch.zeros(0, dtype=torch.long, device=k.device)
+    return k[:, idx].contiguous(), v[:, idx].contiguous(), [(0, int(idx.numel()))] if segments else []
 
-    Returns (o, lse) of the whole key set on rank 0 -- the exact LSE merge of the
-    ranks' partials, folded in rank order -- and this rank's own partial on the
-    other ranks (after its send has completed).
-    """
+
+def merge_to_rank0(o, lse, rank: int, world: int, merge=None, group=None):
+    """Rank 0 receives every other rank's partial (o, lse) into its own memory and
+    folds them in, in rank order, with the exact LSE merge; the other ranks send
+    theirs.  Returns the merged (o, lse) on rank 0, the rank's own partial elsewhere."""
     import torch.distributed as dist
-    attn = attn or _default_attn_keys
     merge = merge or _default_merge
-    parts = key_parts(branches, world, by_branch=by_branch)
-    o, lse = attn(q, k, v, parts[rank])
     if world == 1:
         return o, lse
     if rank != 0:
@@ -138,3 +147,17 @@ def attend_key_split(q, k, v, branches, rank: int, world: int, attn=None, merge=
         dist.recv(rl, src=r, group=group)
         acc_o, acc_l = merge(acc_o, acc_l, ro, rl)
     return acc_o, acc_l
+
+
+def attend_key_split(q, k, v, branches, rank: int, world: int, attn=None, merge=None, by_branch: bool = False,
+                     group=None):
+    """Partial attention over this rank's key part; rank 0 merges every part.
+
+    Returns (o, lse) of the whole key set on rank 0 -- the exact LSE merge of the
+    ranks' partials, folded in rank order -- and this rank's own partial on the
+    other ranks (after its send has completed).
+    """
+    attn = attn or _default_attn_keys
+    parts = key_parts(branches, world, by_branch=by_branch)
+    o, lse = attn(q, k, v, parts[rank])
+    return merge_to_rank0(o, lse, rank, world, merge=merge, group=group)

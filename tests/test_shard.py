@@ -154,3 +154,16 @@ def test_key_split_single_rank_is_whole_key_set():
     c = W.cfg_tiny()
     parts = shard.key_parts(c.branches, 1)
     assert parts == [[s for br in c.branches for s in br]]
+
+
+def test_compact_part_keeps_the_key_set():
+    from kv_cache_attention_chunk_b200 import workloads as W
+    import oracle
+    c = W.cfg_tiny()
+    parts = shard.key_parts(c.branches, 3)
+    for p in parts:
+        kr, vr, seg = shard.compact_part(c.k, c.v, p)
+        a = oracle.segment_attention(c.q, c.k, c.v, [p], c.scale)
+        b = oracle.segment_attention(c.q, kr, vr, [seg], c.scale)
+        assert np.array_equal(a["branch_o"][0], b["branch_o"][0])
+        assert np.array_equal(a["branch_lse"][0], b["branch_lse"][0])
