@@ -379,6 +379,28 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float* v) {
   }
 }
 
+// 32 fp32 values v -> at dst, bf16 of v - float(bf16(v)) (what rounding v to bf16
+// drops; v = bf16(v) + residual to within 2^-17 |v|).
+__device__ __forceinline__ void store_residual32(__nv_bfloat16* dst, const float* v) {
+  float r[32];
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const uint32_t h = pack_bf16x2(v[e], v[e + 1]);
+    r[e] = v[e] - __uint_as_float(h << 16);
+    r[e + 1] = v[e + 1] - __uint_as_float(h & 0xFFFF0000u);
+  }
+  store_row32(dst, r);
+}
+
+// 32 values rebuilt as bf16 row + bf16 residual row (see store_residual32).
+__device__ __forceinline__ void load_residual32(const __nv_bfloat16* row, const __nv_bfloat16* res, float* v) {
+  float a[32], b[32];
+  load_row32(row, a);
+  load_row32(res, b);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = a[e] + b[e];
+}
+
 // 32 fp32 values stored as two bf16-sized rows: the high 16 bits of each value
 // at `hi`, the low 16 bits at `lo` (64 bytes each, 16-byte aligned).
 __device__ __forceinline__ void store_split32(__nv_bfloat16* hi, __nv_bfloat16* lo, const uint32_t* v) {
@@ -426,6 +448,12 @@ __device__ __forceinline__ void load_split32(const __nv_bfloat16* hi, const __nv
 #define VKV_EXP_EMU16 4
 #endif
 constexpr int kExpEmu16 = VKV_EXP_EMU16;
+
+// The fused merge keeps the earlier branch's partial as its final bf16 row plus a
+// bf16 residual row (1), or as an exact high/low 16-bit split rewritten at the end (0).
+#ifndef VKV_MERGE_RESIDUAL
+#define VKV_MERGE_RESIDUAL 1
+#endif
 
 // L2 prefetch of the earlier branch's split rows before the final epilogue (1 = on).
 #ifndef VKV_EPI_PREFETCH
@@ -1090,9 +1118,17 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
               if (row_ok) {
                 if (split_prev) {
+#if VKV_MERGE_RESIDUAL
+                  // this branch's row gets its final value (rounded to bf16); the merged row
+                  // keeps what rounding dropped, so the merge at the end sees the fp32 partial
+                  // to within 2^-17 of its size
+                  store_row32(orow + c0, reinterpret_cast<const float*>(v));
+                  store_residual32(mrow_split + c0, reinterpret_cast<const float*>(v));
+#else
                   // keep the exact fp32 partial for the merge: high halves in the merged
                   // row, low halves in this branch's row; both rows are rewritten at the end
                   store_split32(mrow_split + c0, orow + c0, v);
+#endif
                 } else {
                   store_row32(orow + c0, reinterpret_cast<const float*>(v));
                 }
@@ -1122,9 +1158,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         }
         if (VKV_EPI_PREFETCH && ok && !u.piece && p.om != nullptr && p.n_branches == 2 && !sparse && !ragged &&
             prev_branch >= 0 && row_ok) {
-          // the earlier branch's fp32 partial (its two split rows, written at its close
-          // long before and likely out of L2) is read by the epilogue below: bring it
-          // into L2 while the last PV product completes
+          // the earlier branch's partial (the two rows written at its close, long before
+          // and likely out of L2) is read by the epilogue below: bring it into L2 while
+          // the last PV product completes
           const __nv_bfloat16* mr = p.om + u.b * p.om_sb + (long long)qrow * p.om_st + u.h * p.om_sh;
           const __nv_bfloat16* pr = p.o[prev_branch] + u.b * p.o_sb[prev_branch] +
                                     (long long)qrow * p.o_st[prev_branch] + u.h * p.o_sh[prev_branch];
@@ -1174,9 +1210,14 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               if (do_merge) {
                 float g[32];
                 if (prev_branch >= 0) {
+#if VKV_MERGE_RESIDUAL
+                  // the earlier branch's partial: its bf16 row plus the residual row
+                  load_residual32(prow + c0, mrow + c0, g);
+#else
                   // exact fp32 partial of the earlier branch, stored split at its close
                   load_split32(mrow + c0, prow + c0, g);
                   store_row32(const_cast<__nv_bfloat16*>(prow) + c0, g);
+#endif
 #pragma unroll
                   for (int e = 0; e < 32; ++e) g[e] = c_last * f[e] + c_prev * g[e];
                 } else {
