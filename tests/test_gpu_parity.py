@@ -590,3 +590,40 @@ def test_lse_merge_in_place():
     torch.cuda.synchronize()
     assert_bf16_close(a, ref_o, "in-place merge O")
     assert_lse_close(al, np.moveaxis(ref_l, 2, 1), "in-place merge LSE")
+
+
+# ---------------------------------------------------------------------------
+# full size, every row (the launch configuration the bench times, split
+# schedules with key-axis pieces included)
+# ---------------------------------------------------------------------------
+def test_full_size_wan13b_every_row():
+    """Wan-1.3B-shaped chunk (its schedule cuts units into ~190 key-axis pieces):
+    both branch outputs, their LSEs and the merged output, every element."""
+    c = W.cfg_wan13b()
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    assert vk().vkv_chunk_attn_workspace_size(vk().segments_args(q, k, v, c.branches, c.scale)) > 0
+    check_segments_full(c, run_segments(c))
+
+
+def test_full_size_ragged_every_row():
+    c = W.cfg_ragged()
+    o, l = _run_ragged(c)
+    ro, rl = oracle.ragged_attention(c.q, c.k, c.v, c.cu_seqlens, c.scale)
+    assert_bf16_close(o, ro, "ragged full O")
+    assert_lse_close(l, rl, "ragged full LSE")
+
+
+@pytest.mark.parametrize("K", [9, 144])
+def test_full_size_iid_sparse_every_row(K):
+    c = _iid_sparse()
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    idx, _, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
+    err = err_word()
+    o, l = vk().chunk_attn_block_sparse(q, k, v, torch.from_numpy(c.persist_idx).to(DEV), idx,
+                                        c.window_blk0, c.n_win_blk, scale=c.scale, err=err, qblk_order=order)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    sel = idx.cpu().numpy()
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel, c.window_blk0, c.block, c.scale)
+    assert_bf16_close(o, ro, f"iid sparse full O K={K}")
+    assert_lse_close(l, rl, f"iid sparse full LSE K={K}")
