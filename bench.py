@@ -351,6 +351,7 @@ def extras(dev, peaks):
     c = W.cfg_sparse()
     q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
     pers = torch.from_numpy(c.persist_idx).to(dev)
+    kbar = vkv.block_pool(k, c.window_blk0, c.n_win_blk)  # window block means, cached as blocks enter
     sp = {}
     for frac in W.SPARSE_TOPK_FRACTIONS:
         K = W.topk_for_fraction(frac, c.n_win_blk)
@@ -366,15 +367,28 @@ def extras(dev, peaks):
             q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o, qblk_order=order), 20, st))
         ms_nat = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
             q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o), 20, st))
+        # selection inside the attention kernel (from the cached means; the query-block
+        # order is a previous selection's) against the same two steps as separate launches
+        fsel = torch.empty_like(idx)
+        o_f = vkv.chunk_attn_block_sparse(q, k, v, pers, None, c.window_blk0, c.n_win_blk, scale=c.scale,
+                                          qblk_order=order, kbar=kbar, topk=K, sel_out=fsel)
+        ms_fused = statistics.median(timed(lambda: vkv.chunk_attn_block_sparse(
+            q, k, v, pers, None, c.window_blk0, c.n_win_blk, scale=c.scale, out=o_f, qblk_order=order, kbar=kbar,
+            topk=K, sel_out=fsel), 20, st))
+        ms_two = statistics.median(timed(lambda: (
+            vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws, out_idx=idx, kbar=kbar),
+            vkv.chunk_attn_block_sparse(q, k, v, pers, idx, c.window_blk0, c.n_win_blk, scale=c.scale, out=o,
+                                        qblk_order=order, split=False)), 20, st))
         fl = oracle.visited_flops_sparse(1, 12, c.Lq, 128, 64, c.persist_idx.shape[1], K)
         sel_bytes = (c.Lq + c.n_win_blk * 64) * 12 * 128 * 2
         sp[f"K{K}"] = {"attn_ms": ms_att, "attn_tflops": fl / ms_att / 1e9, "attn_ms_natural_order": ms_nat,
                        "select_ms": ms_sel, "select_gbs": sel_bytes / ms_sel / 1e6,
-                       "chunk_ms": ms_sel + ms_att, "visited_frac": (32 + K) / (32 + c.n_win_blk)}
+                       "chunk_ms": ms_sel + ms_att, "visited_frac": (32 + K) / (32 + c.n_win_blk),
+                       "fused_select": {"ms": ms_fused, "tflops": fl / ms_fused / 1e9,
+                                        "two_launch_ms": ms_two}}
     # representatives of the window blocks cached as blocks enter the cache: selection then
     # pools only the query blocks (14.2 MB read instead of 42.5 MB)
     K = W.topk_for_fraction(W.SPARSE_TOPK_FRACTIONS[0], c.n_win_blk)
-    kbar = vkv.block_pool(k, c.window_blk0, c.n_win_blk)
     ms_pool = statistics.median(timed(lambda: vkv.block_pool(k, c.window_blk0, c.n_win_blk, out=kbar), 30, st,
                                       flush))
     idx, _, order = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, workspace=ws, order=True, kbar=kbar)

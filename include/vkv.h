@@ -167,15 +167,34 @@ typedef struct {
    * Otherwise at least vkv_chunk_attn_workspace_size() bytes, 256-byte aligned,
    * owned by the caller (VKV_ERR_WORKSPACE when smaller): the schedule may then
    * cut some units into pieces over disjoint key ranges that run on different
-   * SMs; each piece leaves its partial output and LSE in the workspace and the
-   * last piece of a unit to finish combines them exactly (the same LSE merge as
-   * the two branches) and writes the outputs.  (BLOCK_SPARSE units learn their
-   * key count on the device: their pieces are cut as fractions of it.)  Results equal those of an
+   * SMs; each piece leaves its partial output and LSE in the workspace, and a
+   * small kernel that the call launches behind the attention kernel combines
+   * each unit's pieces exactly (the same LSE merge as the two branches) and
+   * writes the outputs.  (BLOCK_SPARSE units learn their key count on the
+   * device: their pieces are cut as fractions of it.)  Results equal those of an
    * unsplit run up to fp32 rounding.  Its contents need no initialisation (the
-   * call clears its counters on `stream` first) and are dead after the call;
+   * call marks the partial LSEs on `stream` first) and are dead after the call;
    * calls that overlap on the GPU must not share one. */
   void* workspace;
   size_t workspace_bytes;
+
+  /* VKV_MODE_BLOCK_SPARSE, optional: select the window blocks inside the attention
+   * kernel (Sparse Forcing summary, section 2 components 2 and 3: coarse scores
+   * of the query-block means against one representative per window block, top-K
+   * per query block).  When kbar is not NULL, sel_idx is not read: the kernel
+   * pools each unit's query blocks, scores them against kbar and keeps the top
+   * `topk` window blocks of each, exactly as vkv_block_select does from the same
+   * cached means (the same indices, bit for bit), while the unit's persistent
+   * blocks are already being attended.
+   * kbar:    DEVICE fp32 [B*H][n_win_blk][d], 16-byte aligned: the window block
+   *          means (vkv_block_pool), kept by the caller as blocks enter the cache.
+   * sel_out: optional DEVICE int32 [B*H][ceil(Lq/block)][topk]: receives the
+   *          selection (ascending ids, as vkv_block_select's out_idx), e.g. to
+   *          derive a query-block order for a later call.
+   * Requires 1 <= topk <= n_win_blk <= 512 (else VKV_ERR_SHAPE).  Units are not
+   * split along the key axis in this form (workspace is ignored). */
+  const float* kbar;
+  int32_t* sel_out;
 } vkv_attn_args;
 
 /*

@@ -14,6 +14,8 @@
 
 #include "vkv_attn_kernel.cuh"
 
+static_assert(sizeof(vkv::AttnParams) <= 32764, "kernel parameter space");
+
 namespace vkv {
 
 namespace {
@@ -370,13 +372,13 @@ std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const s
   return plan;
 }
 
-template <int D, bool SP, bool PC>
+template <int D, bool SP, bool PC, bool FS>
 bool set_smem_attr_t(int dev) {
   static std::mutex mu;
   static unsigned long long done = 0;
   std::lock_guard<std::mutex> lk(mu);
   if (done & (1ull << dev)) return true;
-  const void* fn = reinterpret_cast<const void*>(chunk_attn_kernel<D, SP, PC>);
+  const void* fn = reinterpret_cast<const void*>(chunk_attn_kernel<D, SP, PC, FS>);
   cudaFuncAttributes fa;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM_BYTES) !=
           cudaSuccess ||
@@ -391,15 +393,16 @@ bool set_smem_attr_t(int dev) {
 }
 
 // Sets the shared-memory size of the instantiation and launches it.
-template <int D, bool SP, bool PC>
+template <int D, bool SP, bool PC, bool FS = false>
 vkv_status launch_attn_t(int dev, const AttnParams& P, cudaStream_t st) {
-  if (!set_smem_attr_t<D, SP, PC>(dev)) return VKV_ERR_CUDA;
-  chunk_attn_kernel<D, SP, PC><<<P.n_ctas, 384, AttnCfg<D>::SMEM_BYTES, st>>>(P);
+  if (!set_smem_attr_t<D, SP, PC, FS>(dev)) return VKV_ERR_CUDA;
+  chunk_attn_kernel<D, SP, PC, FS><<<P.n_ctas, 384, AttnCfg<D>::SMEM_BYTES, st>>>(P);
   return cudaGetLastError() == cudaSuccess ? VKV_OK : VKV_ERR_CUDA;
 }
 
 template <int D>
 vkv_status launch_attn_d(int dev, bool sp, bool pc, const AttnParams& P, cudaStream_t st) {
+  if (sp && P.kbar) return launch_attn_t<D, true, false, true>(dev, P, st);
   if (sp) return pc ? launch_attn_t<D, true, true>(dev, P, st) : launch_attn_t<D, true, false>(dev, P, st);
   return pc ? launch_attn_t<D, false, true>(dev, P, st) : launch_attn_t<D, false, false>(dev, P, st);
 }
@@ -582,8 +585,22 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
     if (a->n_win_blk > 1024 || a->topk > a->n_win_blk) return VKV_ERR_SHAPE;
     if ((long long)(a->window_blk0 + a->n_win_blk) * 64 > Lkv) return VKV_ERR_RANGE;
     if (a->n_persist + std::min(a->n_win_blk, 4 * a->topk) > kMaxListEntries) return VKV_ERR_UNSUPPORTED;
-    if (check_ptrs && ((a->n_persist > 0 && !a->persist_idx) || (a->topk > 0 && !a->sel_idx)))
+    // selection in the kernel (window block means given): whole units, at least one
+    // block per query block, a window that fits the kernel's ranking keys
+    const bool fs = a->kbar != nullptr;
+    if (fs && (a->topk < 1 || a->n_win_blk > kFsMaxWin)) return VKV_ERR_SHAPE;
+    if (fs) want_split = false;
+    if (check_ptrs && ((a->n_persist > 0 && !a->persist_idx) || (a->topk > 0 && !a->sel_idx && !fs)))
       return VKV_ERR_NULL;
+    if (check_ptrs && fs && (reinterpret_cast<uintptr_t>(a->kbar) & 15)) return VKV_ERR_ALIGN;
+    if (fs) {
+      P->kbar = a->kbar;
+      P->sel_out = a->sel_out;
+      P->qp = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
+      P->q_sb = a->q.sb;
+      P->q_st = a->q.st;
+      P->q_sh = a->q.sh;
+    }
     P->n_persist = a->n_persist;
     P->topk = a->topk;
     P->window_blk0 = a->window_blk0;
@@ -613,7 +630,7 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
       steps1.assign(n_seq, P->sp_est[0]);
     }
     key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
-          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n");
+          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n") + (fs ? "/fs" : "");
   } else {
     if (check_ptrs && !a->cu_seqlens) return VKV_ERR_NULL;
     if (Lkv <= 0) return VKV_ERR_SHAPE;

@@ -41,6 +41,7 @@
 
 #include "vkv_internal.h"
 #include "vkv_ptx.cuh"
+#include "vkv_topk.cuh"
 
 namespace vkv {
 
@@ -69,9 +70,12 @@ struct Ctl {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t list_ready[2], list_free[2], drain;  // one pair per block-list buffer
+  uint64_t list_pers[2];  // FS: the buffer's persistent prefix is written
   uint32_t tmem_base;
   int abort_flag;
   int list_count[2];
+  int pers_count[2];  // FS: entries of the persistent prefix
+  int sel_go;         // FS: the selection warps may write the next list buffer
   uint32_t bitmap[4][32];
   uint32_t list[kMaxListEntries];  // block-list buffer 0 (buffer 1: the ring's last K/V slot)
 };
@@ -278,35 +282,15 @@ __device__ __forceinline__ int unit_steps(const AttnParams& p, int list_count, i
   return (list_count + 1) >> 1;
 }
 
-// Build the unit's block list (BLOCK_SPARSE): persistent blocks (visible to
-// every query block of the unit) followed by the union of the window blocks
-// selected by the unit's query blocks, ascending, each tagged with the query
-// blocks that selected it.  Executed by all 32 lanes of one warp.
-__device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, const UnitInfo& u,
-                                                 uint32_t* list, int* list_count) {
+// The persistent blocks of sequence s at the head of a unit's block list (visible
+// to all nqb query blocks of the unit); an index outside the cache or inside the
+// window records VKV_DEVERR_BAD_INDEX and is skipped.  Returns the entry count.
+// Executed by all 32 lanes of one warp.
+__device__ __forceinline__ int build_persist_prefix(const AttnParams& p, int s, int nqb, uint32_t* list) {
   const uint32_t lane = lane_id();
-  const int qb0 = u.tile0 * 2;
-  const int nqb = min(2 * u.ntiles, p.n_qblk - qb0);
   const uint32_t all_mask = (nqb > 0) ? ((1u << nqb) - 1u) : 0u;
-  const int nwords = (p.n_win_blk + 31) >> 5;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) ctl->bitmap[i][lane] = 0u;
-  __syncwarp();
-  for (int i = 0; i < nqb; ++i) {
-    const int qbi = unit_qblk(p, u.s, qb0 + i, lane == 0);
-    const int* row = p.sel_idx + ((size_t)u.s * p.n_qblk + qbi) * p.topk;
-    for (int e = lane; e < p.topk; e += 32) {
-      const int w = __ldg(row + e);
-      if (w >= 0 && w < p.n_win_blk) {
-        atomicOr(&ctl->bitmap[i][w >> 5], 1u << (w & 31));
-      } else {
-        set_err(p, VKV_DEVERR_BAD_INDEX);
-      }
-    }
-  }
-  __syncwarp();
   int base = 0;
-  const int* prow = p.persist_idx + (size_t)u.s * p.n_persist;
+  const int* prow = p.persist_idx + (size_t)s * p.n_persist;
   for (int e0 = 0; e0 < p.n_persist; e0 += 32) {
     const int e = e0 + (int)lane;
     int blk = -1;
@@ -321,7 +305,18 @@ __device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, 
     if (ok) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)blk | (all_mask << 24);
     base += __popc(bal);
   }
-  // window union: lane L owns window blocks [32L, 32L + 32)
+  return base;
+}
+
+// The union of the window blocks that the unit's nqb query blocks selected
+// (ctl->bitmap[i]: bit w of query block i), ascending, each tagged with the
+// query blocks that selected it, appended at list[base]; the list's length goes
+// to *list_count.  Executed by all 32 lanes of one warp.
+__device__ __forceinline__ void build_window_union(const AttnParams& p, Ctl* ctl, int nqb, uint32_t* list,
+                                                   int base, int* list_count) {
+  const uint32_t lane = lane_id();
+  const int nwords = (p.n_win_blk + 31) >> 5;
+  // lane L owns window blocks [32L, 32L + 32)
   uint32_t m[4], uni = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -349,6 +344,150 @@ __device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, 
   if (lane == 0) *list_count = base + total;
   __threadfence_block();
   __syncwarp();
+}
+
+// Build the unit's block list (BLOCK_SPARSE) from the caller's selection:
+// persistent blocks (visible to every query block of the unit) followed by the
+// union of the window blocks selected by the unit's query blocks, ascending,
+// each tagged with the query blocks that selected it.  Executed by all 32
+// lanes of one warp.
+__device__ __forceinline__ void build_block_list(const AttnParams& p, Ctl* ctl, const UnitInfo& u,
+                                                 uint32_t* list, int* list_count) {
+  const uint32_t lane = lane_id();
+  const int qb0 = u.tile0 * 2;
+  const int nqb = min(2 * u.ntiles, p.n_qblk - qb0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ctl->bitmap[i][lane] = 0u;
+  __syncwarp();
+  for (int i = 0; i < nqb; ++i) {
+    const int qbi = unit_qblk(p, u.s, qb0 + i, lane == 0);
+    const int* row = p.sel_idx + ((size_t)u.s * p.n_qblk + qbi) * p.topk;
+    for (int e = lane; e < p.topk; e += 32) {
+      const int w = __ldg(row + e);
+      if (w >= 0 && w < p.n_win_blk) {
+        atomicOr(&ctl->bitmap[i][w >> 5], 1u << (w & 31));
+      } else {
+        set_err(p, VKV_DEVERR_BAD_INDEX);
+      }
+    }
+  }
+  __syncwarp();
+  const int base = build_persist_prefix(p, u.s, nqb, list);
+  build_window_union(p, ctl, nqb, list, base, list_count);
+}
+
+// ---------------------------------------------------------------------------
+// Selection inside the block-sparse kernel (FS instantiation).  Warps 2-3 choose
+// the window blocks of each unit's query blocks from the cached window block
+// means (Sparse Forcing summary, section 2 component 2 "Blockified
+// Compression": one representative per block for coarse scoring) and publish
+// the unit's block list in two steps: the persistent prefix at once
+// (list_pers), which the other roles start streaming, then the union of the
+// selections (list_ready).  The arithmetic follows the standalone selection
+// kernel operation for operation -- the same row grouping and addition order of
+// the query pooling, the same multiply-add chains of the scores, the same
+// warp_topk -- so the choice equals vkv_block_select's with cached means.
+// ---------------------------------------------------------------------------
+constexpr int kFsMaxWin = 512;  // window blocks the selection keys have room for
+
+// Selection scratch in the block-sparse instantiation's last K/V slot, after the
+// second block list: pooled queries [4][D] fp32, one 256-bin histogram per
+// selection warp, ranking keys [4][kFsMaxWin].
+template <int D>
+struct FsScratch {
+  static constexpr int OFF_QS = 1280;
+  static constexpr int OFF_HIST = OFF_QS + 4 * D * 4;
+  static constexpr int OFF_KEYS = OFF_HIST + 2 * 256 * 4;
+  static constexpr int BYTES = OFF_KEYS + 4 * kFsMaxWin * 4;
+  static_assert(kMaxListEntries * 4 <= OFF_QS, "second block list");
+  static_assert(BYTES <= AttnCfg<D>::KV_BYTES, "selection scratch");
+};
+
+// Named barrier of the two selection warps.
+__device__ __forceinline__ void fs_bar() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+
+// Mean of each of the unit's nq query blocks (positions qb0 .. qb0 + nq - 1 of
+// the unit order) into qs[q][D]: thread
+// (q, c) of the 64 sums the 16-byte column chunk c of the block's rows in row
+// groups g = 0 .. G-1 (rows g, g + G, ...), group by group, then divides by the
+// block's row count -- the standalone kernel's order of additions.
+template <int D>
+__device__ __forceinline__ void fs_pool(const AttnParams& p, const UnitInfo& u, int qb0, int nq, float* qs,
+                                        int st) {
+  constexpr int CPR = D / 8, G = 256 / CPR, RPT = 64 / G;
+  const __nv_bfloat16* base = p.qp + u.b * p.q_sb + u.h * p.q_sh;
+  for (int x = st; x < 4 * CPR; x += 64) {
+    const int q = x / CPR, c = x % CPR;
+    if (q >= nq) continue;
+    const int qb = unit_qblk(p, u.s, qb0 + q, c == 0);
+    float sum[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum[e] = 0.f;
+#pragma unroll 1
+    for (int g0 = 0; g0 < G; g0 += 2) {
+      uint4 v[2][RPT];
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          const int row = qb * 64 + g0 + gi + G * i;
+          v[gi][i] = row < p.Lq ? __ldg(reinterpret_cast<const uint4*>(base + (long long)row * p.q_st) + c)
+                                : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          const uint32_t w[4] = {v[gi][i].x, v[gi][i].y, v[gi][i].z, v[gi][i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += __uint_as_float(w[e] << 16);
+            acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum[e] += acc[e];
+      }
+    }
+    const int nrows = min(64, p.Lq - qb * 64);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qs[q * D + c * 8 + e] = sum[e] * (1.f / (float)nrows);
+  }
+}
+
+// Ranking keys of the n_win_blk window blocks for the nq pooled query blocks:
+// thread st scores blocks st, st + 64, ... from the block means in global memory
+// (four multiply-add chains over the float4 columns, added pairwise at the end).
+template <int D>
+__device__ __forceinline__ void fs_score(const AttnParams& p, int s, int nq, const float* qs, uint32_t* keys,
+                                         int st) {
+  constexpr int CH = D / 4;
+  const float* kb = p.kbar + (size_t)s * p.n_win_blk * D;
+  const float4* q4 = reinterpret_cast<const float4*>(qs);
+  for (int w = st; w < p.n_win_blk; w += 64) {
+    const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)w * D);
+    float acc[4][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+#pragma unroll 8
+    for (int cc = 0; cc < CH; ++cc) {
+      const float4 kv = __ldg(kr + cc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 qv = q4[q * CH + cc];
+        acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
+        acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
+        acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
+        acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq) keys[q * p.n_win_blk + w] = score_key(rank_score((acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3])));
+  }
 }
 
 // 32 fp32 values -> 32 bf16 at dst (64 bytes, 16-byte aligned).
@@ -671,8 +810,12 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xFFFFFFFFu
 // PC: the schedule has key-axis pieces.  Kept apart because the piece paths,
 // though cold, change the register allocation of the softmax step loop (measured
 // ~10 % more cycles per step on whole units with them compiled in).
-template <int D, bool SP, bool PC>
+// FS (with SP, without PC): warps 2-3 select each unit's window blocks from the
+// cached window block means; the other roles read the unit's block list in two
+// steps (the persistent prefix, then the rest once the selection is done).
+template <int D, bool SP, bool PC, bool FS = false>
 __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constant__ AttnParams p) {
+  static_assert(!FS || (SP && !PC), "selection in the kernel: block-sparse, whole units");
   using C = AttnCfg<D>;
   constexpr uint32_t NS = SP ? (uint32_t)C::NSLOT - 1u : (uint32_t)C::NSLOT;  // ring slots
   extern __shared__ uint8_t smem_raw[];
@@ -694,6 +837,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   const uint32_t b_odone0 = smem_u32(&ctl->o_done[0]);
   const uint32_t b_lready0 = smem_u32(&ctl->list_ready[0]);
   const uint32_t b_lfree0 = smem_u32(&ctl->list_free[0]);
+  const uint32_t b_lpers0 = smem_u32(&ctl->list_pers[0]);
   const uint32_t b_drain = smem_u32(&ctl->drain);
 
   if (threadIdx.x == 0) {
@@ -710,7 +854,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_lready0 + 8 * b, 1);
-      mbar_init(b_lfree0 + 8 * b, 9);
+      // readers of a list buffer: the MMA thread, the 8 softmax warps, and with FS the producer
+      mbar_init(b_lfree0 + 8 * b, FS ? 10 : 9);
+      mbar_init(b_lpers0 + 8 * b, 1);
     }
     mbar_init(b_drain, 1);
     ctl->abort_flag = 0;
@@ -752,7 +898,22 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
         int rs = 0, rl = 0;
         const int lb = SP ? (int)(ucnt & 1u) : 0;
-        if (sparse) {
+        const uint32_t uph = (ucnt >> 1) & 1u;  // FS: this list buffer's use parity
+        bool fs_full = true;                     // FS: the whole block list is known
+        if (FS) {
+          // the selection warps build the list: start on its persistent prefix
+          bool w = true;
+          if (lane == 0) w = mbar_wait(b_lpers0 + 8 * lb, uph, abort_flag, p.err);
+          ok = __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if ((ctl->pers_count[lb] >> 1) == 0) {
+            if (lane == 0) w = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+            ok = __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
+            if (!ok) break;
+          } else {
+            fs_full = false;
+          }
+        } else if (sparse) {
           // wait for the unit that used this list buffer before (one unit back with a
           // single buffer, two with two) to release it
           const uint32_t back = SP ? 2u : 1u;
@@ -768,8 +929,17 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ragged_range(p, u.s, rs, rl, lane == 0);
         }
         PieceInfo pi;
-        const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
-        if (nsteps == 0) continue;
+        int nsteps;
+        if (FS) {
+          pi.j0 = 0;
+          nsteps = fs_full ? unit_steps(p, ctl->list_count[lb], 0) : (ctl->pers_count[lb] >> 1);
+        } else {
+          nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
+        }
+        if (nsteps == 0) {
+          if (FS && lane == 0) mbar_arrive(b_lfree0 + 8 * lb);
+          continue;
+        }
         if (lane == 0) {
           if (qcnt > 0) ok = mbar_wait(b_qempty, (qcnt - 1) & 1, abort_flag, p.err);
           if (ok) {
@@ -796,11 +966,21 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             ++qcnt;
           }
           TileIter it;
-          it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
+          it.init(&p, list_buf(lb), (FS && !fs_full) ? ctl->pers_count[lb] : ctl->list_count[lb], rs, rl);
           if (u.piece) it.seek(pi.j0);
           const int kvh = ragged ? 0 : u.h;
           const int kvb = ragged ? 0 : u.b;
-          for (int j = 0; j < nsteps && ok; ++j) {
+          for (int j = 0; (FS || j < nsteps) && ok; ++j) {
+            if (FS && j >= nsteps) {
+              // end of the persistent prefix: the rest of the list once the selection is in
+              if (fs_full) break;
+              ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+              if (!ok) break;
+              fs_full = true;
+              it.count = ctl->list_count[lb];
+              nsteps = unit_steps(p, it.count, 0);
+              if (j >= nsteps) break;
+            }
             const TileDesc td = it.next();
             for (int kv = 0; kv < 2; ++kv) {
               const uint32_t slot = item % NS, use = item / NS;
@@ -825,6 +1005,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               ++item;
             }
           }
+          if (FS && ok) mbar_arrive(b_lfree0 + 8 * lb);  // this unit's list entries are all read
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -867,14 +1048,31 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           const int lb = SP ? (int)(ucnt & 1u) : 0;
           const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);  // this buffer's use parity
           if (sparse) {
-            ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+            ok = mbar_wait((FS ? b_lpers0 : b_lready0) + 8 * lb, uph, abort_flag, p.err);
             if (!ok) break;
           } else if (ragged) {
             ragged_range(p, u.s, rs, rl, false);
           }
           PieceInfo pi;
-          const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
-          if (sparse) mbar_arrive(b_lfree0 + 8 * lb);  // only the step count was needed
+          int nsteps;
+          bool fs_full = true;  // FS: the unit's step count is final
+          if (FS) {
+            // the persistent prefix alone fixes a lower bound; the count itself is
+            // needed one step before the prefix ends (whether another S follows)
+            pi.j0 = 0;
+            nsteps = ctl->pers_count[lb] >> 1;
+            if (nsteps <= 1) {
+              ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+              if (!ok) break;
+              nsteps = unit_steps(p, ctl->list_count[lb], 0);
+              mbar_arrive(b_lfree0 + 8 * lb);
+            } else {
+              fs_full = false;
+            }
+          } else {
+            nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
+            if (sparse) mbar_arrive(b_lfree0 + 8 * lb);  // only the step count was needed
+          }
           if (nsteps == 0) continue;
           TileIter it;
           it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
@@ -888,8 +1086,16 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           tc_fence_after();
           for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % NS);
           mma_commit(b_empty0 + 8 * (item % NS));
+          bool q_rel = nsteps == 1;  // FS: the Q tiles' release is committed
           if (nsteps == 1) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
+            if (FS && !fs_full && j + 1 >= nsteps) {
+              ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+              if (!ok) break;
+              nsteps = unit_steps(p, ctl->list_count[lb], 0);
+              fs_full = true;
+              mbar_arrive(b_lfree0 + 8 * lb);
+            }
             // a piece may start inside a branch: its first step starts the accumulator too
             const bool first = (sparse || ragged) ? (j == 0) : (it.next().first || (PC && j == 0));
             const uint32_t vit = item + 2 * j + 1;
@@ -933,7 +1139,14 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             mma_commit(b_empty0 + 8 * (vit % NS));
             if (has_next) {
               mma_commit(b_empty0 + 8 * (knext % NS));
-              if (j + 2 == nsteps) mma_commit(b_qempty);
+              if (j + 2 == nsteps && fs_full) {
+                mma_commit(b_qempty);
+                q_rel = true;
+              }
+            } else if (FS && !q_rel) {
+              // the count became final only at this last step: release the Q tiles now
+              mma_commit(b_qempty);
+              q_rel = true;
             }
           }
           item += 2 * nsteps;
@@ -943,6 +1156,52 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         mbar_wait_drain(b_drain, 0);
       }
       __syncwarp();
+    } else if (FS) {
+      // ------------------------------------------------------------ selection (warps 2-3)
+      // Runs up to one unit ahead of the other roles: the list buffer of unit i
+      // is free once every reader has finished unit i - 2.
+      const int st = (int)threadIdx.x - 64;
+      const int sw = warp - 2;
+      uint8_t* const scr = reinterpret_cast<uint8_t*>(list1);
+      float* const qs = reinterpret_cast<float*>(scr + FsScratch<D>::OFF_QS);
+      int* const hist = reinterpret_cast<int*>(scr + FsScratch<D>::OFF_HIST);
+      uint32_t* const keys = reinterpret_cast<uint32_t*>(scr + FsScratch<D>::OFF_KEYS);
+      uint32_t ucnt = 0;
+      for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
+        const UnitInfo u = decode_entry<false>(p, p.units[ui]);
+        const int lb = (int)(ucnt & 1u);
+        if (ucnt >= 2) {
+          // one thread waits; both warps take its answer, so they never part ways
+          if (st == 0)
+            ctl->sel_go = mbar_wait(b_lfree0 + 8 * lb, ((ucnt - 2) >> 1) & 1u, abort_flag, p.err) ? 1 : 0;
+          fs_bar();
+          if (!ctl->sel_go) break;
+        }
+        const int qb0 = u.tile0 * 2;
+        const int nqb = min(2 * u.ntiles, p.n_qblk - qb0);
+        uint32_t* const list = list_buf(lb);
+        if (sw == 0) {
+          const int base = build_persist_prefix(p, u.s, nqb, list);
+          if (lane == 0) ctl->pers_count[lb] = base;
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_lpers0 + 8 * lb);
+        }
+        fs_pool<D>(p, u, qb0, nqb, qs, st);
+        fs_bar();
+        fs_score<D>(p, u.s, nqb, qs, keys, st);
+        fs_bar();
+        for (int q = sw; q < nqb; q += 2) {
+          const int qbi = unit_qblk(p, u.s, qb0 + q, false);
+          warp_topk(keys + q * p.n_win_blk, p.n_win_blk, p.topk, hist + sw * 256,
+                    p.sel_out ? p.sel_out + ((size_t)u.s * p.n_qblk + qbi) * p.topk : nullptr, ctl->bitmap[q]);
+        }
+        fs_bar();
+        if (sw == 0) {
+          build_window_union(p, ctl, nqb, list, ctl->pers_count[lb], &ctl->list_count[lb]);
+          if (lane == 0) mbar_arrive(b_lready0 + 8 * lb);
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------------ softmax
@@ -963,9 +1222,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
       int rs = 0, rl = 0;
       const int lb = SP ? (int)(ucnt & 1u) : 0;
+      const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);
       if (sparse) {
-        const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);
-        ok = warp_all(mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err));
+        ok = warp_all(mbar_wait((FS ? b_lpers0 : b_lready0) + 8 * lb, uph, abort_flag, p.err));
         if (!ok) break;
       } else if (ragged) {
         ragged_range(p, u.s, rs, rl, false);
@@ -974,7 +1233,21 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       // is piece_k - 1), so that the step loop keeps no more state live than a
       // whole unit does
       PieceInfo pi0;
-      const int nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi0);
+      int nsteps;
+      bool fs_full = true;  // FS: the whole block list is known
+      if (FS) {
+        pi0.j0 = 0;
+        nsteps = ctl->pers_count[lb] >> 1;
+        if (nsteps == 0) {
+          ok = warp_all(mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err));
+          if (!ok) break;
+          nsteps = unit_steps(p, ctl->list_count[lb], 0);
+        } else {
+          fs_full = false;
+        }
+      } else {
+        nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi0);
+      }
       const bool active = t < u.ntiles;
       int qrow = (u.tile0 + t) * 128 + r;
       if (sparse) {
@@ -988,9 +1261,19 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       int cur_branch = -1, prev_branch = -1;
       if (active && nsteps > 0) {
         TileIter it;
-        it.init(&p, list_buf(lb), ctl->list_count[lb], rs, rl);
+        it.init(&p, list_buf(lb), (FS && !fs_full) ? ctl->pers_count[lb] : ctl->list_count[lb], rs, rl);
         if (u.piece) it.seek(pi0.j0);
-        for (int j = 0; j < nsteps; ++j) {
+        for (int j = 0; FS || j < nsteps; ++j) {
+          if (FS && j >= nsteps) {
+            // end of the persistent prefix: the rest of the list once the selection is in
+            if (fs_full) break;
+            ok = warp_all(mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err));
+            if (!ok) break;
+            fs_full = true;
+            it.count = ctl->list_count[lb];
+            nsteps = unit_steps(p, it.count, 0);
+            if (j >= nsteps) break;
+          }
           const TileDesc td = it.next();
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
           VKV_STAMP(tr);

@@ -47,6 +47,13 @@ struct AttnParams {
   const int* persist_idx;
   const int* sel_idx;
   const int* qblk_order;  // optional [B*H][n_qblk] query-block permutation
+  // BLOCK_SPARSE with the selection in the kernel: the queries (elements, strides
+  // in elements), the window block means [B*H][n_win_blk][d] and where the
+  // selection goes (optional, [B*H][n_qblk][topk])
+  const __nv_bfloat16* qp;
+  long long q_sb, q_st, q_sh;
+  const float* kbar;
+  int* sel_out;
   // RAGGED
   const int* cu_seqlens;
   // outputs

@@ -25,6 +25,7 @@
 #include "vkv_internal.h"
 #include "vkv_pool.cuh"
 #include "vkv_ptx.cuh"
+#include "vkv_topk.cuh"
 
 namespace vkv {
 
@@ -76,15 +77,9 @@ size_t sel_smem_bytes(int n_win, bool stage) {
 //     scores rank last and -0 counts as +0, so equal scores tie on the block
 //     index.  A score becomes its order-preserving 32-bit integer image (larger
 //     score, larger key).
-//  3. Warp q selects the top-K of query block q on its own (warp barriers only):
-//     radix selection of the K-th largest key, 8 bits a pass (4 passes): the
-//     keys still in play (those sharing the threshold's digits found so far)
-//     are counted per digit in the warp's shared-memory histogram, one atomic
-//     per distinct digit and chunk of 32 keys; the lanes scan it from the top and
-//     fix the next digit (where the running count reaches the number still to
-//     take).  Then, in ascending block order, every key above the threshold is
-//     kept, and of the keys equal to it the lowest ids, as many as are still to
-//     take; a ballot gives each kept block its output position.
+//  3. Warp q selects the top-K of query block q on its own (warp_topk: radix
+//     selection of the K-th largest key, then a ballot gives each kept block
+//     its output position).
 template <int D>
 __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
   constexpr int CPR = D / 8;     // 16-byte chunks per row (bf16)
@@ -191,11 +186,9 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
       }
 #pragma unroll
       for (int q = 0; q < kSelQ; ++q) {
-        float v = (acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]);
-        v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+        const float v = rank_score((acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]));
         if (q < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + q) * p.n_win + w] = v;
-        const uint32_t u = __float_as_uint(v);
-        keys[q * p.n_win + w] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);
+        keys[q * p.n_win + w] = score_key(v);
       }
     }
   } else {
@@ -229,10 +222,9 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
           float v = sc[0];
 #pragma unroll
           for (int q = 1; q < kSelQ; ++q) v = (c == q) ? sc[q] : v;
-          v = (v != v) ? -INFINITY : (v == 0.f ? 0.f : v);
+          v = rank_score(v);
           if (c < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + c) * p.n_win + w] = v;
-          const uint32_t u = __float_as_uint(v);
-          keys[c * p.n_win + w] = u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u);
+          keys[c * p.n_win + w] = score_key(v);
         }
       }
     }
@@ -240,75 +232,8 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
   __syncthreads();
   // 3. warp q: top-K of query block q
   if (warp >= nq) return;
-  const uint32_t* kq = keys + warp * p.n_win;
-  int* hq = hist + warp * 256;
-  const uint32_t lt = (1u << lane) - 1u;
-  uint32_t thr = 0u;
-  int need = p.topk;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-#pragma unroll
-    for (int i = 0; i < 8; ++i) hq[lane + 32 * i] = 0;
-    __syncwarp();
-    for (int w0 = 0; w0 < p.n_win; w0 += 32) {
-      const int w = w0 + lane;
-      const uint32_t k = w < p.n_win ? kq[w] : 0u;
-      const bool in_play = w < p.n_win && (k & hi_mask) == thr;
-      const uint32_t digit = in_play ? ((k >> shift) & 255u) : 0xFFFFFFFFu;
-      const unsigned grp = __match_any_sync(0xFFFFFFFFu, digit);
-      if (in_play && (grp & lt) == 0u) atomicAdd(&hq[digit], __popc(grp));
-    }
-    __syncwarp();
-    // lane l holds digits 255 - 8l .. 248 - 8l (lane 0 the largest)
-    int cnt[8], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      cnt[i] = hq[255 - (8 * lane + i)];
-      sum += cnt[i];
-    }
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    int above = incl - sum;  // keys in play with a digit above this lane's bins
-    const bool mine = above < need && need <= incl;
-    uint32_t digit = 0u;
-    int rest = 0;
-    if (mine) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (above + cnt[i] >= need) {
-          digit = (uint32_t)(255 - (8 * lane + i));
-          rest = need - above;
-          break;
-        }
-        above += cnt[i];
-      }
-    }
-    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
-    thr |= __shfl_sync(0xFFFFFFFFu, digit, src) << shift;
-    need = __shfl_sync(0xFFFFFFFFu, rest, src);
-    __syncwarp();  // the histogram is read before the next pass clears it
-  }
-  // keys above the threshold, then the lowest-id keys equal to it, in ascending order
-  int* oi = p.out_idx + ((size_t)s * p.n_qblk + j0 + warp) * p.topk;
-  int written = 0, eq_seen = 0;
-  for (int w0 = 0; w0 < p.n_win; w0 += 32) {
-    const int w = w0 + lane;
-    const uint32_t k = w < p.n_win ? kq[w] : 0u;
-    const bool valid = w < p.n_win;
-    const bool eq = valid && k == thr;
-    const uint32_t beq = __ballot_sync(0xFFFFFFFFu, eq);
-    const bool keep = valid && (k > thr || (eq && eq_seen + __popc(beq & lt) < need));
-    eq_seen += __popc(beq);
-    const uint32_t bk = __ballot_sync(0xFFFFFFFFu, keep);
-    if (keep) oi[written + __popc(bk & lt)] = w;
-    written += __popc(bk);
-  }
+  warp_topk(keys + warp * p.n_win, p.n_win, p.topk, hist + warp * 256,
+            p.out_idx + ((size_t)s * p.n_qblk + j0 + warp) * p.topk, nullptr);
 }
 
 // Query-block order that groups blocks with similar selections (a work-grouping

@@ -64,6 +64,7 @@ class vkv_attn_args(ctypes.Structure):
         ("err_word", c_void_p),
         ("qblk_order", c_void_p),
         ("workspace", c_void_p), ("workspace_bytes", c_size_t),
+        ("kbar", c_void_p), ("sel_out", c_void_p),
     ]
 
 
@@ -421,21 +422,38 @@ def chunk_attn_segments(q, k, v, branches, scale=None, merged=True, err=None, st
 
 
 def chunk_attn_block_sparse(q, k, v, persist_idx, sel_idx, window_blk0, n_win_blk, scale=None,
-                            err=None, stream=None, out=None, qblk_order=None, split=True, workspace=None):
+                            err=None, stream=None, out=None, qblk_order=None, split=True, workspace=None,
+                            kbar=None, topk=None, sel_out=None):
     """Persistent blocks + selected window blocks (device int32 index tensors).
 
     qblk_order (optional device int32 [B*H, nQblk]): query-block permutation that
     groups blocks with similar selections into the same units (from block_select).
     split / workspace: key-axis pieces, as in chunk_attn_segments.
+
+    kbar (optional device fp32 [B*H, n_win_blk, d], from block_pool): the kernel
+    selects the top-`topk` window blocks itself (sel_idx may then be None); the
+    selection is written to sel_out (device int32 [B*H, nQblk, topk]) when given.
     """
     d = q.shape[3]
     a = _base_args(MODE_BLOCK_SPARSE, q, k.shape[1], d, scale, tensor_desc(k), tensor_desc(v), err)
     persist_idx = persist_idx.contiguous()
-    sel_idx = sel_idx.contiguous()
     a.persist_idx = persist_idx.data_ptr() if persist_idx.numel() else None
     a.n_persist = persist_idx.shape[-1]
-    a.sel_idx = sel_idx.data_ptr() if sel_idx.numel() else None
-    a.topk = sel_idx.shape[-1]
+    if kbar is not None:
+        if topk is None:
+            topk = sel_out.shape[-1] if sel_out is not None else sel_idx.shape[-1]
+        if not (kbar.dtype == torch.float32 and kbar.is_contiguous()):
+            raise ValueError("kbar must be a contiguous float32 tensor [B*H, n_win_blk, d]")
+        a.kbar = kbar.data_ptr()
+        if sel_out is not None:
+            if not (sel_out.dtype == torch.int32 and sel_out.is_contiguous()):
+                raise ValueError("sel_out must be a contiguous int32 tensor [B*H, nQblk, topk]")
+            a.sel_out = sel_out.data_ptr()
+        a.topk = int(topk)
+    else:
+        sel_idx = sel_idx.contiguous()
+        a.sel_idx = sel_idx.data_ptr() if sel_idx.numel() else None
+        a.topk = sel_idx.shape[-1]
     a.window_blk0 = int(window_blk0)
     a.n_win_blk = int(n_win_blk)
     if qblk_order is not None:

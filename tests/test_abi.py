@@ -166,6 +166,28 @@ def test_sparse_validation():
         assert call(sparse_args()) == 6
 
 
+def test_sparse_selection_in_kernel_validation():
+    # window block means given: sel_idx is not read, the selection limits apply
+    assert call(sparse_args(kbar=FAKE + 4)) == 3                      # means not 16-byte aligned
+    assert call(sparse_args(kbar=FAKE, topk=0)) == 2                  # nothing to select
+    a = sparse_args(kbar=FAKE, Lkv=1024 * 64, window_blk0=8, n_win_blk=513, n_persist=8)
+    a.k = T(sb=1024 * 64 * 1024)
+    a.v = T(sb=1024 * 64 * 1024)
+    assert call(a) == 2                                               # window beyond 512 blocks
+    a.n_win_blk = 512
+    if not torch.cuda.is_available():
+        assert call(a) == 6                                           # accepted up to the device call
+        assert call(sparse_args(kbar=FAKE, sel_idx=None)) == 6
+    # the selection runs on whole units: the schedule cuts no pieces where it otherwise would
+    a = sparse_args(topk=144, H=2, Lq=256, n_win_blk=144, window_blk0=0, Lkv=64 * 200, n_persist=32)
+    a.k = T(sb=64 * 200 * 1024)
+    a.v = T(sb=64 * 200 * 1024)
+    assert vkv.attn_schedule(a, 148, True)["pieces"].shape[0] > 0
+    a.kbar = FAKE
+    sch = vkv.attn_schedule(a, 148, True)
+    assert sch["pieces"].shape[0] == 0 and sch["n_slots"] == 0
+
+
 def ragged_args(cu_host):
     a = seg_args()
     a.mode = vkv.MODE_RAGGED

@@ -1,0 +1,185 @@
+"""GPU parity of the block-sparse attention that selects its own window blocks.
+
+With cached window block means (kbar) the attention kernel pools each unit's
+query blocks, scores them and keeps the top-K itself.  Its selection must be
+the standalone selection's, index for index (both follow the same arithmetic),
+and therefore the oracle's wherever the fp64 scores leave no near-tie; its
+outputs must be those of the two-launch path (standalone selection, then the
+attention from the selected ids), bit for bit, and within the parity
+tolerances of the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_attention_chunk_b200 import workloads as W
+from parity_util import assert_bf16_close, assert_lse_close, sparse_iid_case, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from kv_cache_attention_chunk_b200 import build, vkv
+    build.build()
+    vkv.lib()
+    assert torch.cuda.is_available()
+    yield
+
+
+def vk():
+    from kv_cache_attention_chunk_b200 import vkv
+    return vkv
+
+
+def err_word():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+def _case(seed, H, d, qf, n_persist, win=4):
+    return W.make_block_sparse("fused", seed=seed, H=H, d=d, frame_tokens=256, block=64, hist_frames=3,
+                               win_frames=win, q_frames=qf, n_persist=n_persist)
+
+
+def _run_pair(c, q, K, order=None, sel_out=True):
+    """(fused o, lse, selection) and (two-launch o, lse, selection) on the same inputs."""
+    k, v = c.k.to(DEV), c.v.to(DEV)
+    pidx = torch.from_numpy(c.persist_idx).to(DEV)
+    kbar = vk().block_pool(k, c.window_blk0, c.n_win_blk)
+    n_qblk = -(-q.shape[1] // 64)
+    sel = torch.full((c.B * c.H, n_qblk, K), -1, dtype=torch.int32, device=DEV) if sel_out else None
+    err = err_word()
+    o, l = vk().chunk_attn_block_sparse(q, k, v, pidx, None, c.window_blk0, c.n_win_blk, scale=c.scale, err=err,
+                                        qblk_order=order, kbar=kbar, topk=K, sel_out=sel)
+    idx, _ = vk().block_select(q, k, c.window_blk0, c.n_win_blk, K, kbar=kbar)
+    err2 = err_word()
+    o2, l2 = vk().chunk_attn_block_sparse(q, k, v, pidx, idx, c.window_blk0, c.n_win_blk, scale=c.scale,
+                                          err=err2, qblk_order=order, split=False)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and int(err2.item()) == 0
+    return (o, l, sel), (o2, l2, idx)
+
+
+def _gap_ok(qn, kn, c, K):
+    s = oracle.block_scores(qn, kn, c.window_blk0, c.n_win_blk, c.block)
+    return oracle.select_topk(s, K), oracle.topk_gap(s, K) > 1e-4
+
+
+# (seed, H, d, q frames, persistent blocks, K, query-block order, query rows cut from the end)
+SMALL = [
+    (90, 2, 128, 2, 5, 3, None, 0),        # odd persistent count: the prefix ends inside a tile
+    (91, 2, 128, 1, 0, 4, None, 0),        # no persistent blocks: everything waits for the selection
+    (92, 3, 64, 2, 2, 1, None, 0),         # a one-step prefix
+    (93, 2, 128, 3, 3, 16, "random", 0),   # every window block (K = n_win)
+    (94, 2, 64, 2, 8, 7, "select", 0),
+    (95, 2, 128, 2, 5, 3, None, 37),       # ragged tail: a partial last query block
+    (96, 3, 128, 3, 4, 5, "random", 100),  # ragged tail under a permuted order
+]
+
+
+@pytest.mark.parametrize("seed,H,d,qf,npers,K,order,cut", SMALL)
+def test_fused_select_small(seed, H, d, qf, npers, K, order, cut):
+    c = _case(seed, H, d, qf, npers)
+    qn = c.q[:, :c.q.shape[1] - cut] if cut else c.q
+    q = qn.contiguous().to(DEV)
+    n_qblk = -(-q.shape[1] // 64)
+    perm = None
+    if order == "random":
+        rng = np.random.default_rng(seed)
+        perm = torch.from_numpy(np.stack([rng.permutation(n_qblk) for _ in range(c.B * c.H)]).astype(np.int32)).to(DEV)
+    elif order == "select":
+        _, _, perm = vk().block_select(q, c.k.to(DEV), c.window_blk0, c.n_win_blk, K, order=True)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, K, perm)
+    assert torch.equal(sel, idx), "in-kernel selection differs from the standalone selection"
+    ref_idx, ok = _gap_ok(qn, c.k, c, K)
+    s = sel.cpu().numpy()
+    assert np.array_equal(s[ok], ref_idx[ok])
+    assert torch.equal(o, o2) and torch.equal(l, l2), "outputs differ from the two-launch path"
+    ro, rl = oracle.block_sparse_attention(qn, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale)
+    assert_bf16_close(o, ro, "fused-select O")
+    assert_lse_close(l, rl, "fused-select LSE")
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_fused_select_several_units_per_cta(d):
+    """More units than SMs: each CTA's selection warps run ahead over both list buffers."""
+    c = _case(97, 96, d, 4, 6)
+    q = c.q.to(DEV)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 5)
+    assert torch.equal(sel, idx)
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+    heads, qblocks = [0, 47, 95], [0, 7, 15]
+    s = sel.cpu().numpy()
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale,
+                                           heads=heads, qblocks=qblocks)
+    rows = [r for j in qblocks for r in range(j * 64, j * 64 + 64)]
+    assert_bf16_close(to_np(o)[:, rows][:, :, heads], ro[:, rows][:, :, heads], "fused-select O (many units)")
+    assert_lse_close(to_np(l)[:, heads][:, :, rows], rl[:, heads][:, :, rows], "fused-select LSE (many units)")
+
+
+_IID = {}
+
+
+def _iid():
+    if "c" not in _IID:
+        _IID["c"] = sparse_iid_case(name="iid")
+    return _IID["c"]
+
+
+@pytest.mark.parametrize("frac", W.SPARSE_TOPK_FRACTIONS)
+def test_fused_select_full_config3(frac):
+    """Config 3 (i.i.d. recipe) at full size, grouped order: the selection equals the
+    oracle's at every K with no row masked, the outputs equal the two-launch path's."""
+    c = _iid()
+    K = W.topk_for_fraction(frac, c.n_win_blk)
+    q, k = c.q.to(DEV), c.k.to(DEV)
+    _, _, order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, K, order)
+    assert torch.equal(sel, idx)
+    ref = oracle.block_select(c.q, c.k, c.window_blk0, c.n_win_blk, c.block, K)[0]
+    assert np.array_equal(sel.cpu().numpy(), ref), f"K={K}"
+    assert torch.equal(o, o2) and torch.equal(l, l2), f"K={K}"
+
+
+def test_fused_select_full_config3_sampled_natural_order():
+    c = _iid()
+    K = W.topk_for_fraction(W.SPARSE_TOPK_FRACTIONS[0], c.n_win_blk)
+    q = c.q.to(DEV)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, K, None)
+    assert torch.equal(sel, idx)
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+    s = sel.cpu().numpy()
+    heads, qblocks = [2, 7, 11], [0, 3, 35, 70, 71]
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale,
+                                           heads=heads, qblocks=qblocks)
+    rows = [r for j in qblocks for r in range(j * 64, j * 64 + 64)]
+    assert_bf16_close(to_np(o)[:, rows][:, :, heads], ro[:, rows][:, :, heads], "fused-select config 3 O")
+    assert_lse_close(to_np(l)[:, heads][:, :, rows], rl[:, heads][:, :, rows], "fused-select config 3 LSE")
+
+
+def test_fused_select_without_selection_output():
+    c = _case(98, 2, 128, 2, 5)
+    q = c.q.to(DEV)
+    (o, l, _), (o2, l2, _) = _run_pair(c, q, 3, sel_out=False)
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+
+
+def test_fused_select_bad_order_sets_error_word():
+    c = _case(99, 2, 128, 2, 5)
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    n_qblk = c.n_qblk
+    perm = np.tile(np.arange(n_qblk, dtype=np.int32), (c.B * c.H, 1))
+    perm[1, 2] = n_qblk + 3  # not a query block
+    kbar = vk().block_pool(k, c.window_blk0, c.n_win_blk)
+    err = err_word()
+    vk().chunk_attn_block_sparse(q, k, v, torch.from_numpy(c.persist_idx).to(DEV), None, c.window_blk0,
+                                 c.n_win_blk, scale=c.scale, err=err, qblk_order=torch.from_numpy(perm).to(DEV),
+                                 kbar=kbar, topk=3)
+    torch.cuda.synchronize()
+    assert int(err.item()) == vk().DEVERR_BAD_INDEX
+    # the device stays usable
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 3)
+    assert torch.equal(sel, idx) and torch.equal(o, o2)
