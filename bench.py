@@ -112,7 +112,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx.cuh")
+ATTN_SOURCES = ("vkv_attn.cu", "vkv_attn_kernel.cuh", "vkv_internal.h", "vkv_ptx.cuh", "vkv_topk.cuh")
 
 
 def headline_split(vkv, q, k, v, branches, scale) -> bool:
@@ -763,12 +763,21 @@ def run_profile(args):
         oa, la, ob, lb = (t.to(dev) for t in W.make_merge_inputs(5, 1, 4680, 40, 128))
         o = vkv.lse_merge(oa, la, ob, lb)
         fn = lambda: vkv.lse_merge(oa, la, ob, lb, out=o)  # noqa: E731
-    elif args.profile in ("select", "sparse9", "sparse144"):
+    elif args.profile in ("select", "sparse9", "sparse144", "sparse9fs"):
         c = W.cfg_sparse()
         q, k, v = c.q.to(dev), c.k.to(dev), c.v.to(dev)
         K = 9 if args.profile != "sparse144" else 144
         idx, _, order = vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
-        if args.profile == "select":
+        if args.profile == "sparse9fs":
+            # the selection inside the attention kernel, from cached window block means
+            pers = torch.from_numpy(c.persist_idx).to(dev)
+            kbar = vkv.block_pool(k, c.window_blk0, c.n_win_blk)
+            o = vkv.chunk_attn_block_sparse(q, k, v, pers, None, c.window_blk0, c.n_win_blk, scale=c.scale,
+                                            qblk_order=order, kbar=kbar, topk=K, sel_out=idx)
+            fn = lambda: vkv.chunk_attn_block_sparse(q, k, v, pers, None, c.window_blk0,  # noqa: E731
+                                                     c.n_win_blk, scale=c.scale, out=o, qblk_order=order,
+                                                     kbar=kbar, topk=K, sel_out=idx)
+        elif args.profile == "select":
             fn = lambda: vkv.block_select(q, k, c.window_blk0, c.n_win_blk, K, out_idx=idx,  # noqa: E731
                                           out_order=order)
         else:
@@ -815,7 +824,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None,
                     help="run one small case for an ncu capture: wan13b, wan14b, merge, select, sparse9, "
-                         "sparse144, ragged, latent, compaction, persist")
+                         "sparse9fs, sparse144, ragged, latent, compaction, persist")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
