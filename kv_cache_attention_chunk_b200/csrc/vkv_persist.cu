@@ -4,211 +4,231 @@
 // or replace blocks of, the persistent memory; component 2: one representative
 // per block for the coarse score).
 //
-// Three launches on the caller's stream, the last two as programmatic dependent
-// launches (each starts while the one before it drains):
-//   pool_kernel          means of the chunk's 64-row query blocks (shared with
-//                        block selection) -> workspace;
-//   cand_pool_kernel     means of the candidate blocks (current persistent
-//                        blocks, then the evicted range) -> workspace, with a
-//                        validity flag per candidate;
-//   persist_pick_kernel  one CTA per (batch, head): the chunk's mean query from
-//                        the block means (weighted by block rows; all threads,
-//                        partial sums in shared memory), one score per
-//                        candidate (a warp each), rank of each candidate among the valid
-//                        ones (higher score first, then the lower block id),
-//                        the C best written in ascending block order.
+// One launch: a thread-block cluster of kPersistSplit CTAs per (batch, head).
+//   1. every CTA sums its slice of the chunk's query rows (16-byte column chunks,
+//      16 rows per thread in flight) into its shared memory, and each of its
+//      warps takes one of the CTA's candidate blocks (the current persistent
+//      blocks, then the evicted range; candidates rank, rank + kPersistSplit,
+//      ...): the block's mean, lanes adding their row subsets by shuffles, to
+//      the workspace;
+//   2. after a cluster barrier every CTA adds the CTAs' query sums from their
+//      shared memory (distributed shared memory, in rank order: every CTA gets
+//      the same mean query) and scores its own candidates (the warp that
+//      pooled a block scores it), writing the scores into CTA 0's shared memory;
+//   3. after a second cluster barrier CTA 0 ranks every candidate among the
+//      valid ones (higher score first, then the lower block id) by counting and
+//      writes the C best in ascending block order.
 // Candidate counts are small (C + evicted <= 2048), so ranking by counting is
 // both exact and cheap.
 #include <cstring>
 
 #include "vkv_internal.h"
-#include "vkv_pool.cuh"
 #include "vkv_ptx.cuh"
 
 namespace vkv {
 namespace {
 
-constexpr int kMaxCand = 2048;
+// Thread-block clusters: the CTA's rank, the cluster barrier, and the shared memory
+// of another CTA of the cluster (distributed shared memory).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
 
-struct CandParams {
+// Every thread of every CTA of the cluster: memory operations before it (shared
+// and global) are visible to all the cluster's threads after it.  All threads of
+// the cluster must execute it the same number of times.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Stores v into CTA `rank`'s shared memory, at the offset of `local` in this CTA's.
+__device__ __forceinline__ void dsmem_st_f32(float* local, uint32_t rank, float v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+// A float of CTA `rank`'s shared memory, at the offset of `local` in this CTA's.
+__device__ __forceinline__ float dsmem_ld_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+constexpr int kMaxCand = 2048;
+constexpr int kPersistSplit = 8;  // CTAs per (batch, head): one cluster
+
+struct PersistParams {
+  const __nv_bfloat16* q;
+  long long q_sb, q_st, q_sh;
   const __nv_bfloat16* k;
   long long k_sb, k_st, k_sh;
   const int* persist_idx;  // [BH][C]
-  int H, C, n_evict, evict_blk0, n_blocks;
-  float* kbar;             // [BH][C + n_evict][d]
-  unsigned char* valid;    // [BH][C + n_evict]
+  int H, Lq, C, n_evict, evict_blk0, n_blocks;
+  float* kbar;             // workspace [BH][C + n_evict][d]: the candidates' block means
+  int* out_idx;            // [BH][C]
+  float* out_scores;       // [BH][C + n_evict] or null
   int* err;
 };
 
-// grid: x = candidate, y = b*H + h; 256 threads: thread (g, c) sums rows
-// g*RPG .. g*RPG + RPG - 1 of 16-byte column c, row groups combined in smem.
-template <int D>
-__global__ void __launch_bounds__(256) cand_pool_kernel(const CandParams p) {
-  constexpr int CPR = D / 8;
-  constexpr int GROUPS = 256 / CPR;
-  constexpr int RPG = 64 / GROUPS;
-  __shared__ float part[GROUPS][D];
-  const int i = blockIdx.x;
-  const int s = blockIdx.y;
-  const int n_cand = p.C + p.n_evict;
-  int blk;
-  bool ok;
+// Candidate i of sequence s: its block id, and whether it may be ranked (a
+// persistent id inside the cache and outside the evicted range).
+__device__ __forceinline__ int cand_block(const PersistParams& p, int s, int i, bool& ok) {
   if (i < p.C) {
-    blk = __ldg(p.persist_idx + (size_t)s * p.C + i);
+    const int blk = __ldg(p.persist_idx + (size_t)s * p.C + i);
     ok = blk >= 0 && blk < p.n_blocks && (blk < p.evict_blk0 || blk >= p.evict_blk0 + p.n_evict);
-    if (!ok && threadIdx.x == 0 && p.err) atomicCAS(p.err, 0, VKV_DEVERR_BAD_INDEX);
-  } else {
-    blk = p.evict_blk0 + (i - p.C);
-    ok = true;
+    return blk;
   }
-  if (threadIdx.x == 0) p.valid[(size_t)s * n_cand + i] = ok ? 1 : 0;
-  if (!ok) {
-    griddep_wait();
-    return;
-  }
-  const int b = s / p.H, h = s - (s / p.H) * p.H;
-  const int c = threadIdx.x % CPR, g = threadIdx.x / CPR;
-  const __nv_bfloat16* base = p.k + b * p.k_sb + h * p.k_sh + (long long)blk * 64 * p.k_st;
-  uint4 v[RPG];
-#pragma unroll
-  for (int r = 0; r < RPG; ++r) v[r] = __ldcs(reinterpret_cast<const uint4*>(base + (long long)(g * RPG + r) * p.k_st) + c);
-  // the pick kernel may be scheduled now; it waits for this grid's completion
-  griddep_launch_dependents();
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-  for (int r = 0; r < RPG; ++r) {
-    const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      acc[2 * e] += __uint_as_float(w[e] << 16);
-      acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) part[g][c * 8 + e] = acc[e];
-  __syncthreads();
-  float* dst = p.kbar + ((size_t)s * n_cand + i) * D;
-  for (int x = threadIdx.x; x < D; x += 256) {
-    float sum = 0.f;
-#pragma unroll
-    for (int gg = 0; gg < GROUPS; ++gg) sum += part[gg][x];
-    dst[x] = sum * (1.f / 64.f);
-  }
-  // this grid reads nothing the query pooling writes and may run beside it; it ends
-  // only after that grid has, so the pick kernel's wait on this grid covers both
-  griddep_wait();
+  ok = true;
+  return p.evict_blk0 + (i - p.C);
 }
 
-struct PickParams {
-  const float* qbar;            // [BH][n_qblk][d]
-  const float* kbar;            // [BH][n_cand][d]
-  const unsigned char* valid;   // [BH][n_cand]
-  const int* persist_idx;       // [BH][C]
-  int C, n_evict, evict_blk0, n_qblk, Lq;
-  int* out_idx;                 // [BH][C]
-  float* out_scores;            // [BH][n_cand] or null
-};
+__device__ __forceinline__ void add_bf16x8(float* acc, const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    acc[2 * e] += __uint_as_float(w[e] << 16);
+    acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+}
 
-// grid: x = b*H + h; 256 threads.
+// grid: x = kPersistSplit (one cluster), y = b*H + h; 256 threads.
 template <int D>
-__global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
+__global__ void __cluster_dims__(kPersistSplit, 1, 1) __launch_bounds__(256)
+    persist_update_kernel(const PersistParams p) {
+  constexpr int CPR = D / 8;     // 16-byte chunks per row
+  constexpr int G = 256 / CPR;   // row groups of the query sum
+  constexpr int RS = 32 / CPR;   // row subsets of a warp pooling one block
+  constexpr int PL = D / 32;     // columns per lane when a warp scores a block
+  constexpr int NW = 256 / 32;
+  constexpr int QU = 16;         // query rows per thread in flight
+  __shared__ float part[G][D];
+  __shared__ float qpart[D];     // this CTA's sum of its query rows (read by every CTA)
   __shared__ float qm[D];
-  __shared__ float sc[kMaxCand];
+  __shared__ float sc[kMaxCand];  // CTA 0: every candidate's score
   __shared__ int ids[kMaxCand];
   __shared__ unsigned char ok[kMaxCand];
   __shared__ unsigned char keep[kMaxCand];
-  constexpr int C4 = D / 4;          // 16-byte column chunks of a row
-  constexpr int G = 256 / C4;        // row groups
-  __shared__ float part[G][D];
-  const int s = blockIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  const int s = blockIdx.y;
+  const int b = s / p.H, h = s - (s / p.H) * p.H;
   const int n_cand = p.C + p.n_evict;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NW = 256 / 32;   // warps
-  constexpr int PB = 8;          // candidates a warp holds in registers at once
-  constexpr int PL = D / 32;     // columns per lane
-  griddep_wait();  // both pooling grids before this one on the stream have completed
-  // candidate ids and validity into shared memory (independent loads, all at once)
-  for (int i = threadIdx.x; i < n_cand; i += 256) {
-    ids[i] = i < p.C ? __ldg(p.persist_idx + (size_t)s * p.C + i) : p.evict_blk0 + (i - p.C);
-    ok[i] = p.valid[(size_t)s * n_cand + i];
-  }
-  // the block means of this warp's first PB candidates (i = warp + NW * b), loaded
-  // now so that their latency overlaps the mean-query reduction below
-  float kreg[PB][PL];
-#pragma unroll
-  for (int b = 0; b < PB; ++b) {
-    const int i = warp + NW * b;
-    const float* kr = p.kbar + ((size_t)s * n_cand + (i < n_cand ? i : 0)) * D;
-#pragma unroll
-    for (int e = 0; e < PL; ++e) kreg[b][e] = (i < n_cand) ? __ldg(kr + lane + 32 * e) : 0.f;
-  }
-  // mean query of the chunk: block means weighted by their rows (the last block may
-  // be short).  Thread (g, c) sums chunk c of query blocks g, g + G, ... (independent
-  // loads, several in flight), then the G partial sums are added in shared memory.
+  // 1a. the sum of this CTA's slice of the query rows; thread (g, c): chunk c of
+  //     rows r0 + g, r0 + g + G, ...
   {
-    const int c = threadIdx.x % C4, g = threadIdx.x / C4;
-    const float4* qb = reinterpret_cast<const float4*>(p.qbar + (size_t)s * p.n_qblk * D) + c;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int j = g; j < p.n_qblk; j += G) {
-      const float w = (float)min(64, p.Lq - j * 64);
-      const float4 v = __ldg(qb + (size_t)j * C4);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
-    part[g][4 * c + 0] = acc.x;
-    part[g][4 * c + 1] = acc.y;
-    part[g][4 * c + 2] = acc.z;
-    part[g][4 * c + 3] = acc.w;
-  }
-  __syncthreads();
-  for (int x = threadIdx.x; x < D; x += blockDim.x) {
-    float acc = 0.f;
+    const int c = threadIdx.x % CPR, g = threadIdx.x / CPR;
+    const int R = (p.Lq + kPersistSplit - 1) / kPersistSplit;
+    const int r0 = (int)rank * R, r1 = min(p.Lq, r0 + R);
+    const __nv_bfloat16* base = p.q + b * p.q_sb + h * p.q_sh;
+    float acc[8];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc += part[g][x];
-    qm[x] = acc / (float)p.Lq;
-  }
-  __syncthreads();
-  // one warp per candidate: lane l takes columns l, l + 32, ... of the block mean
-  // (the first PB candidates of each warp from the registers loaded above)
-  for (int i = warp, b = 0; i < n_cand; i += NW, ++b) {
-    const bool valid = ok[i] != 0;
-    float v = -INFINITY;
-    if (valid) {
-      float a = 0.f;
-      if (b < PB) {
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int row0 = r0 + g; row0 < r1; row0 += QU * G) {
+      uint4 v[QU];
 #pragma unroll
-        for (int bb = 0; bb < PB; ++bb)
-          if (bb == b) {
-#pragma unroll
-            for (int e = 0; e < PL; ++e) a = fmaf(qm[lane + 32 * e], kreg[bb][e], a);
-          }
-      } else {
-        const float* kr = p.kbar + ((size_t)s * n_cand + i) * D;
-#pragma unroll
-        for (int e = 0; e < PL; ++e) a = fmaf(qm[lane + 32 * e], __ldg(kr + lane + 32 * e), a);
+      for (int u = 0; u < QU; ++u) {
+        const int row = row0 + u * G;
+        v[u] = row < r1 ? __ldcs(reinterpret_cast<const uint4*>(base + (long long)row * p.q_st) + c)
+                        : make_uint4(0, 0, 0, 0);
       }
+#pragma unroll
+      for (int u = 0; u < QU; ++u) add_bf16x8(acc, v[u]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[g][c * 8 + e] = acc[e];
+  }
+  // 1b. warp w pools candidates rank + kPersistSplit * (w + NW * t): lane (sub, c) sums
+  //     chunk c of rows sub, sub + RS, ..., then the row subsets are added by shuffles
+  const __nv_bfloat16* kbase = p.k + b * p.k_sb + h * p.k_sh;
+  {
+    const int c = lane % CPR, sub = lane / CPR;
+    for (int i = (int)rank + kPersistSplit * warp; i < n_cand; i += kPersistSplit * NW) {
+      bool v_ok = false;
+      const int blk = cand_block(p, s, i, v_ok);
+      if (!v_ok) continue;
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int r0 = 0; r0 < 64 / RS; r0 += 16) {
+        uint4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          v[u] = __ldcs(reinterpret_cast<const uint4*>(kbase + ((long long)blk * 64 + sub + RS * (r0 + u)) * p.k_st) + c);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) add_bf16x8(acc, v[u]);
+      }
+#pragma unroll
+      for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], o);
+      if (sub == 0) {
+        float4* dst = reinterpret_cast<float4*>(p.kbar + ((size_t)s * n_cand + i) * D + c * 8);
+        dst[0] = make_float4(acc[0] * (1.f / 64.f), acc[1] * (1.f / 64.f), acc[2] * (1.f / 64.f), acc[3] * (1.f / 64.f));
+        dst[1] = make_float4(acc[4] * (1.f / 64.f), acc[5] * (1.f / 64.f), acc[6] * (1.f / 64.f), acc[7] * (1.f / 64.f));
+      }
+    }
+  }
+  __syncthreads();
+  for (int x = threadIdx.x; x < D; x += 256) {
+    float t = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) t += part[gg][x];
+    qpart[x] = t;
+  }
+  // 2. the mean query from every CTA's sum (the same order in every CTA), then the
+  //    scores of this CTA's candidates into CTA 0's shared memory
+  cluster_sync();
+  for (int x = threadIdx.x; x < D; x += 256) {
+    float v[kPersistSplit];
+#pragma unroll
+    for (uint32_t r = 0; r < kPersistSplit; ++r) v[r] = dsmem_ld_f32(&qpart[x], r);
+    float t = 0.f;
+#pragma unroll
+    for (uint32_t r = 0; r < kPersistSplit; ++r) t += v[r];
+    qm[x] = t / (float)p.Lq;
+  }
+  __syncthreads();
+  for (int i = (int)rank + kPersistSplit * warp; i < n_cand; i += kPersistSplit * NW) {
+    bool v_ok = false;
+    cand_block(p, s, i, v_ok);
+    float v = -INFINITY;
+    if (v_ok) {
+      // the block mean this warp wrote in step 1 (ordered by the barriers since)
+      const float* kr = p.kbar + ((size_t)s * n_cand + i) * D;
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < PL; ++e) a = fmaf(qm[lane + 32 * e], __ldcg(kr + lane + 32 * e), a);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
       v = (a != a) ? -INFINITY : (a == 0.f ? 0.f : a);  // NaN ranks last; -0 ties with +0
     }
     if (lane == 0) {
-      sc[i] = v;
-      if (p.out_scores) p.out_scores[(size_t)s * n_cand + i] = valid ? v : -INFINITY;
+      dsmem_st_f32(&sc[i], 0, v);
+      if (p.out_scores) p.out_scores[(size_t)s * n_cand + i] = v;
     }
+  }
+  cluster_sync();  // every score is in CTA 0; no CTA reads another's memory after this
+  if (rank != 0) return;
+  // 3. rank by counting; the C best, ascending
+  for (int i = threadIdx.x; i < n_cand; i += 256) {
+    bool v = false;
+    ids[i] = cand_block(p, s, i, v);
+    ok[i] = v ? 1 : 0;
+    if (!v && p.err) atomicCAS(p.err, 0, VKV_DEVERR_BAD_INDEX);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-    int rank = 0;
+    int r = 0;
     const float si = sc[i];
     const int di = ids[i];
-    for (int j = 0; j < n_cand; ++j)
-      rank += (ok[j] && (sc[j] > si || (sc[j] == si && ids[j] < di))) ? 1 : 0;
-    keep[i] = (ok[i] && rank < p.C) ? 1 : 0;
+    for (int j = 0; j < n_cand; ++j) r += (ok[j] && (sc[j] > si || (sc[j] == si && ids[j] < di))) ? 1 : 0;
+    keep[i] = (ok[i] && r < p.C) ? 1 : 0;
   }
   __syncthreads();
   int* out = p.out_idx + (size_t)s * p.C;
@@ -227,27 +247,6 @@ __global__ void __launch_bounds__(256) persist_pick_kernel(const PickParams p) {
   }
 }
 
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-// Programmatic dependent launch of a 256-thread kernel with one parameter struct:
-// the grid may start while the one before it on the stream is still running, and
-// orders itself with griddep_wait.
-template <class P>
-bool launch_dependent(const void* fn, dim3 grid, cudaStream_t st, P* params) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  void* args[1] = {params};
-  return cudaLaunchKernelExC(&cfg, fn, args) == cudaSuccess;
-}
-
 }  // namespace
 }  // namespace vkv
 
@@ -256,11 +255,9 @@ using namespace vkv;
 extern "C" size_t vkv_persist_update_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_persist,
                                                     int32_t n_evict, int32_t block, int32_t d) {
   if (B <= 0 || H <= 0 || Lq <= 0 || n_persist <= 0 || n_evict < 0 || block <= 0 || d <= 0) return 0;
-  const size_t BH = (size_t)B * H;
-  const size_t n_qblk = (size_t)(Lq + block - 1) / block;
-  const size_t n_cand = (size_t)n_persist + n_evict;
-  return align256(BH * n_qblk * d * sizeof(float)) + align256(BH * n_cand * d * sizeof(float)) +
-         align256(BH * n_cand);
+  // the candidates' block means
+  const size_t bytes = (size_t)B * H * ((size_t)n_persist + n_evict) * d * sizeof(float);
+  return (bytes + 255) & ~(size_t)255;
 }
 
 extern "C" vkv_status vkv_persist_update(const vkv_persist_args* a, vkv_stream_t stream) {
@@ -278,64 +275,28 @@ extern "C" vkv_status vkv_persist_update(const vkv_persist_args* a, vkv_stream_t
   if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return VKV_ERR_ALIGN;
   int dev = 0;
   if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = a->B * a->H;
-  const int n_qblk = (a->Lq + 63) / 64;
-  const int n_cand = a->n_persist + a->n_evict;
-  uint8_t* ws = reinterpret_cast<uint8_t*>(a->workspace);
-  float* qbar = reinterpret_cast<float*>(ws);
-  float* kbar = reinterpret_cast<float*>(ws + align256((size_t)BH * n_qblk * a->d * sizeof(float)));
-  unsigned char* valid = reinterpret_cast<unsigned char*>(kbar) + align256((size_t)BH * n_cand * a->d * sizeof(float));
-  // 1. query block means
-  PoolParams pp;
+  PersistParams pp;
   std::memset(&pp, 0, sizeof(pp));
   pp.q = reinterpret_cast<const __nv_bfloat16*>(a->q.ptr);
   pp.q_sb = a->q.sb; pp.q_st = a->q.st; pp.q_sh = a->q.sh;
-  pp.B = a->B;
+  pp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
+  pp.k_sb = a->k.sb; pp.k_st = a->k.st; pp.k_sh = a->k.sh;
+  pp.persist_idx = a->persist_idx;
   pp.H = a->H;
-  pp.d = a->d;
   pp.Lq = a->Lq;
-  pp.n_qblk = n_qblk;
-  pp.n_win = 0;
-  pp.qbar = qbar;
-  const int ph = a->d == 128 ? pool_heads<128>() : pool_heads<64>();
-  const dim3 pg(n_qblk, a->B * ((a->H + ph - 1) / ph));
+  pp.C = a->n_persist;
+  pp.n_evict = a->n_evict;
+  pp.evict_blk0 = a->evict_blk0;
+  pp.n_blocks = a->Lkv / 64;
+  pp.kbar = reinterpret_cast<float*>(a->workspace);
+  pp.out_idx = a->out_idx;
+  pp.out_scores = a->out_scores;
+  pp.err = a->err_word;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(kPersistSplit, (unsigned)(a->B * a->H));
   if (a->d == 128)
-    pool_kernel<128><<<pg, 256, 0, st>>>(pp);
+    persist_update_kernel<128><<<grid, 256, 0, st>>>(pp);
   else
-    pool_kernel<64><<<pg, 256, 0, st>>>(pp);
-  if (cudaGetLastError() != cudaSuccess) return VKV_ERR_CUDA;
-  // 2. candidate block means
-  CandParams cp;
-  cp.k = reinterpret_cast<const __nv_bfloat16*>(a->k.ptr);
-  cp.k_sb = a->k.sb; cp.k_st = a->k.st; cp.k_sh = a->k.sh;
-  cp.persist_idx = a->persist_idx;
-  cp.H = a->H;
-  cp.C = a->n_persist;
-  cp.n_evict = a->n_evict;
-  cp.evict_blk0 = a->evict_blk0;
-  cp.n_blocks = a->Lkv / 64;
-  cp.kbar = kbar;
-  cp.valid = valid;
-  cp.err = a->err_word;
-  if (!launch_dependent(a->d == 128 ? (const void*)cand_pool_kernel<128> : (const void*)cand_pool_kernel<64>,
-                        dim3(n_cand, BH), st, &cp))
-    return VKV_ERR_CUDA;
-  // 3. scores and the top C
-  PickParams kp;
-  kp.qbar = qbar;
-  kp.kbar = kbar;
-  kp.valid = valid;
-  kp.persist_idx = a->persist_idx;
-  kp.C = a->n_persist;
-  kp.n_evict = a->n_evict;
-  kp.evict_blk0 = a->evict_blk0;
-  kp.n_qblk = n_qblk;
-  kp.Lq = a->Lq;
-  kp.out_idx = a->out_idx;
-  kp.out_scores = a->out_scores;
-  if (!launch_dependent(a->d == 128 ? (const void*)persist_pick_kernel<128> : (const void*)persist_pick_kernel<64>,
-                        dim3(BH), st, &kp))
-    return VKV_ERR_CUDA;
-  return VKV_OK;
+    persist_update_kernel<64><<<grid, 256, 0, st>>>(pp);
+  return cudaGetLastError() == cudaSuccess ? VKV_OK : VKV_ERR_CUDA;
 }

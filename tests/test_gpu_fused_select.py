@@ -39,9 +39,9 @@ def err_word():
     return torch.zeros(1, dtype=torch.int32, device=DEV)
 
 
-def _case(seed, H, d, qf, n_persist, win=4):
+def _case(seed, H, d, qf, n_persist, win=4, B=1):
     return W.make_block_sparse("fused", seed=seed, H=H, d=d, frame_tokens=256, block=64, hist_frames=3,
-                               win_frames=win, q_frames=qf, n_persist=n_persist)
+                               win_frames=win, q_frames=qf, n_persist=n_persist, B=B)
 
 
 def _run_pair(c, q, K, order=None, sel_out=True):
@@ -158,6 +158,20 @@ def test_fused_select_full_config3_sampled_natural_order():
     rows = [r for j in qblocks for r in range(j * 64, j * 64 + 64)]
     assert_bf16_close(to_np(o)[:, rows][:, :, heads], ro[:, rows][:, :, heads], "fused-select config 3 O")
     assert_lse_close(to_np(l)[:, heads][:, :, rows], rl[:, heads][:, :, rows], "fused-select config 3 LSE")
+
+
+def test_fused_select_batch_of_two():
+    c = _case(100, 3, 128, 3, 5, B=2)
+    q = c.q.to(DEV)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 4)
+    assert torch.equal(sel, idx)
+    ref_idx, ok = _gap_ok(c.q, c.k, c, 4)
+    assert np.array_equal(sel.cpu().numpy()[ok], ref_idx[ok])
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel.cpu().numpy(), c.window_blk0, c.block,
+                                           c.scale)
+    assert_bf16_close(o, ro, "fused-select O (B = 2)")
+    assert_lse_close(l, rl, "fused-select LSE (B = 2)")
 
 
 def test_fused_select_without_selection_output():
