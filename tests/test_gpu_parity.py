@@ -605,6 +605,16 @@ def test_full_size_wan13b_every_row():
     check_segments_full(c, run_segments(c))
 
 
+def test_full_size_wan14b_every_row():
+    """The headline workload (Wan-14B-shaped, 40 heads) in the launch configuration the
+    bench times (head-major split schedule, combine kernel, fused merge): both branch
+    outputs, their LSEs and the merged output, every element."""
+    c = W.cfg_wan14b()
+    q, k, v = c.q.to(DEV), c.k.to(DEV), c.v.to(DEV)
+    assert vk().vkv_chunk_attn_workspace_size(vk().segments_args(q, k, v, c.branches, c.scale)) > 0
+    check_segments_full(c, run_segments(c))
+
+
 def test_full_size_ragged_every_row():
     c = W.cfg_ragged()
     o, l = _run_ragged(c)
