@@ -460,7 +460,8 @@ __device__ __forceinline__ void fs_pool(const AttnParams& p, const UnitInfo& u, 
 
 // Ranking keys of the n_win_blk window blocks for the nq pooled query blocks:
 // thread st scores blocks st, st + 64, ... from the block means in global memory
-// (four multiply-add chains over the float4 columns, added pairwise at the end).
+// (four multiply-add chains over the float4 columns, two of them per paired
+// f32x2 operation, added pairwise at the end).
 template <int D>
 __device__ __forceinline__ void fs_score(const AttnParams& p, int s, int nq, const float* qs, uint32_t* keys,
                                          int st) {
@@ -469,24 +470,27 @@ __device__ __forceinline__ void fs_score(const AttnParams& p, int s, int nq, con
   const float4* q4 = reinterpret_cast<const float4*>(qs);
   for (int w = st; w < p.n_win_blk; w += 64) {
     const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)w * D);
-    float acc[4][4];
+    uint64_t acc[4][2];  // per query block: chains (x, y) and (z, w)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+    for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = 0ull;
 #pragma unroll 8
     for (int cc = 0; cc < CH; ++cc) {
       const float4 kv = __ldg(kr + cc);
+      const uint64_t k01 = pack2f(kv.x, kv.y), k23 = pack2f(kv.z, kv.w);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float4 qv = q4[q * CH + cc];
-        acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
-        acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
-        acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
-        acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+        acc[q][0] = fma2f(pack2f(qv.x, qv.y), k01, acc[q][0]);
+        acc[q][1] = fma2f(pack2f(qv.z, qv.w), k23, acc[q][1]);
       }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < nq) keys[q * p.n_win_blk + w] = score_key(rank_score((acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3])));
+    for (int q = 0; q < 4; ++q) {
+      float a0, a1, a2, a3;
+      unpack2f(acc[q][0], a0, a1);
+      unpack2f(acc[q][1], a2, a3);
+      if (q < nq) keys[q * p.n_win_blk + w] = score_key(rank_score((a0 + a1) + (a2 + a3)));
+    }
   }
 }
 

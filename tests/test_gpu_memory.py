@@ -57,20 +57,22 @@ def test_persist_update_no_evicted_blocks_sorts_the_set():
     assert np.array_equal(ids.cpu().numpy(), np.sort(pers, axis=1))
 
 
-def test_persist_update_full_sparse_config():
-    # config-3 shape: 32 persistent blocks per head; the oldest window frame (24 blocks) leaves
+@pytest.mark.parametrize("n_evict", [24, 100])
+def test_persist_update_full_sparse_config(n_evict):
+    # config-3 shape: 32 persistent blocks per head; the oldest window frame (24 blocks)
+    # leaves, or 100 blocks (132 candidates: every warp of the cluster pools several)
     c = W.cfg_sparse()
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
     ids, sc = vk().persist_update(c.q.to(DEV), c.k.to(DEV), torch.from_numpy(c.persist_idx).to(DEV),
-                                  c.window_blk0, 24, scores=True, err=err)
+                                  c.window_blk0, n_evict, scores=True, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    ref_ids, ref_sc = oracle.persist_update(c.q, c.k, c.persist_idx, c.window_blk0, 24)
+    ref_ids, ref_sc = oracle.persist_update(c.q, c.k, c.persist_idx, c.window_blk0, n_evict)
     assert np.abs(to_np(sc) - ref_sc).max() < 1e-3
     got = ids.cpu().numpy()
     C = c.persist_idx.shape[1]
     for s in range(got.shape[0]):
-        cands = list(c.persist_idx[s]) + list(range(c.window_blk0, c.window_blk0 + 24))
+        cands = list(c.persist_idx[s]) + list(range(c.window_blk0, c.window_blk0 + n_evict))
         score = dict(zip(cands, ref_sc[s]))
         assert len(set(got[s])) == C and list(got[s]) == sorted(got[s])
         kept = set(int(x) for x in got[s])
