@@ -17,11 +17,13 @@
 //                 cache (Pyramid Forcing summary, methodology section 3).
 //
 // Warp roles (384 threads):
-//   warp 0       TMA producer: Q tiles, K/V tiles into a ring of smem slots;
-//                builds the block list in BLOCK_SPARSE mode.
+//   warp 0       TMA producer: Q tiles, K/V tiles into a ring of smem slots.
 //   warp 1       MMA issuer: S_t = Q_t K^T and O_t += P_t V with tcgen05.mma,
 //                accumulators in tensor memory (TMEM); owns the TMEM allocation.
-//   warps 2-3    idle.
+//   warps 2-3    BLOCK_SPARSE: warp 2 builds each unit's block list from the
+//                caller's selection, one unit ahead of the other roles; or, with
+//                the selection in the kernel (FS), warps 2-3 select the window
+//                blocks themselves.  Idle in the other modes.
 // With key-axis pieces (PC), a piece leaves fp32 partials in a workspace and
 // piece_combine_kernel, launched behind this grid, merges them.
 //   warps 4-7    softmax + epilogue for query tile 0 (one thread per row).
@@ -858,8 +860,9 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_lready0 + 8 * b, 1);
-      // readers of a list buffer: the MMA thread, the 8 softmax warps, and with FS the producer
-      mbar_init(b_lfree0 + 8 * b, FS ? 10 : 9);
+      // readers of a list buffer: the MMA thread, the 8 softmax warps, and in the
+      // block-sparse instantiation (whose lists warps 2-3 build) the producer
+      mbar_init(b_lfree0 + 8 * b, SP ? 10 : 9);
       mbar_init(b_lpers0 + 8 * b, 1);
     }
     mbar_init(b_drain, 1);
@@ -917,6 +920,12 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           } else {
             fs_full = false;
           }
+        } else if (SP) {
+          // warp 2 builds the list
+          bool w = true;
+          if (lane == 0) w = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
+          ok = __shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) != 0;
+          if (!ok) break;
         } else if (sparse) {
           // wait for the unit that used this list buffer before (one unit back with a
           // single buffer, two with two) to release it
@@ -941,7 +950,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi);
         }
         if (nsteps == 0) {
-          if (FS && lane == 0) mbar_arrive(b_lfree0 + 8 * lb);
+          if (SP && lane == 0) mbar_arrive(b_lfree0 + 8 * lb);
           continue;
         }
         if (lane == 0) {
@@ -1009,7 +1018,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               ++item;
             }
           }
-          if (FS && ok) mbar_arrive(b_lfree0 + 8 * lb);  // this unit's list entries are all read
+          if (SP && ok) mbar_arrive(b_lfree0 + 8 * lb);  // this unit's list entries are all read
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -1160,6 +1169,23 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         mbar_wait_drain(b_drain, 0);
       }
       __syncwarp();
+    } else if (SP && !FS && warp == 2) {
+      // ------------------------------------------------------------ block lists (warp 2)
+      // Each unit's block list from the caller's selection, up to one unit ahead of the
+      // other roles (the list buffer of unit i is free once every reader has finished
+      // unit i - 2), so the producer only waits for it.
+      uint32_t ucnt = 0;
+      for (int ui = u_begin; ui < u_end; ++ui, ++ucnt) {
+        const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
+        const int lb = (int)(ucnt & 1u);
+        if (ucnt >= 2) {
+          bool w = true;
+          if (lane == 0) w = mbar_wait(b_lfree0 + 8 * lb, ((ucnt - 2) >> 1) & 1u, abort_flag, p.err);
+          if (__shfl_sync(0xFFFFFFFFu, w ? 1 : 0, 0) == 0) break;
+        }
+        build_block_list(p, ctl, u, list_buf(lb), &ctl->list_count[lb]);
+        if (lane == 0) mbar_arrive(b_lready0 + 8 * lb);
+      }
     } else if (FS) {
       // ------------------------------------------------------------ selection (warps 2-3)
       // Runs up to one unit ahead of the other roles: the list buffer of unit i
