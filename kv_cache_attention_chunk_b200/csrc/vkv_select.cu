@@ -169,24 +169,26 @@ __global__ void __launch_bounds__(256) select_kernel(const SelParams p) {
     }
     for (int w = tid; w < p.n_win; w += 256) {
       const float4* kr = reinterpret_cast<const float4*>(kbs + (size_t)w * RS);
-      float acc[kSelQ][4];
+      uint64_t acc[kSelQ][2];  // per query block: chains (x, y) and (z, w), two per f32x2 multiply-add
 #pragma unroll
-      for (int q = 0; q < kSelQ; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+      for (int q = 0; q < kSelQ; ++q) acc[q][0] = acc[q][1] = 0ull;
 #pragma unroll 8
       for (int cc = 0; cc < CH; ++cc) {
         const float4 kv = kr[cc];
+        const uint64_t k01 = pack2f(kv.x, kv.y), k23 = pack2f(kv.z, kv.w);
 #pragma unroll
         for (int q = 0; q < kSelQ; ++q) {
           const float4 qv = reinterpret_cast<const float4*>(qs + q * D)[cc];
-          acc[q][0] = fmaf(qv.x, kv.x, acc[q][0]);
-          acc[q][1] = fmaf(qv.y, kv.y, acc[q][1]);
-          acc[q][2] = fmaf(qv.z, kv.z, acc[q][2]);
-          acc[q][3] = fmaf(qv.w, kv.w, acc[q][3]);
+          acc[q][0] = fma2f(pack2f(qv.x, qv.y), k01, acc[q][0]);
+          acc[q][1] = fma2f(pack2f(qv.z, qv.w), k23, acc[q][1]);
         }
       }
 #pragma unroll
       for (int q = 0; q < kSelQ; ++q) {
-        const float v = rank_score((acc[q][0] + acc[q][1]) + (acc[q][2] + acc[q][3]));
+        float a0, a1, a2, a3;
+        unpack2f(acc[q][0], a0, a1);
+        unpack2f(acc[q][1], a2, a3);
+        const float v = rank_score((a0 + a1) + (a2 + a3));
         if (q < nq && p.out_scores) p.out_scores[((size_t)s * p.n_qblk + j0 + q) * p.n_win + w] = v;
         keys[q * p.n_win + w] = score_key(v);
       }
