@@ -110,9 +110,9 @@ __global__ void __cluster_dims__(kPersistSplit, 1, 1) __launch_bounds__(256)
   __shared__ float qpart[D];     // this CTA's sum of its query rows (read by every CTA)
   __shared__ float qm[D];
   __shared__ float sc[kMaxCand];  // CTA 0: every candidate's score
-  __shared__ int ids[kMaxCand];
-  __shared__ unsigned char ok[kMaxCand];
-  __shared__ unsigned char keep[kMaxCand];
+  __shared__ int ids[kMaxCand];   // CTA 0: block id, then (INT_MAX unless kept) for the output order
+  __shared__ unsigned long long rk[kMaxCand];  // CTA 0: ranking key (0 for an invalid candidate)
+  __shared__ int n_valid;
   const uint32_t rank = cluster_ctarank();
   const int s = blockIdx.y;
   const int b = s / p.H, h = s - (s / p.H) * p.H;
@@ -215,36 +215,59 @@ __global__ void __cluster_dims__(kPersistSplit, 1, 1) __launch_bounds__(256)
   }
   cluster_sync();  // every score is in CTA 0; no CTA reads another's memory after this
   if (rank != 0) return;
-  // 3. rank by counting; the C best, ascending
-  for (int i = threadIdx.x; i < n_cand; i += 256) {
-    bool v = false;
-    ids[i] = cand_block(p, s, i, v);
-    ok[i] = v ? 1 : 0;
-    if (!v && p.err) atomicCAS(p.err, 0, VKV_DEVERR_BAD_INDEX);
-  }
+  // 3. rank by counting.  A valid candidate's key is its score's order-preserving
+  //    image above the complement of its block id (higher score first, then the
+  //    lower id); an invalid one's key is 0, below every valid key.
+  if (threadIdx.x == 0) n_valid = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
+  int my_valid = 0;
+  int my_id[kMaxCand / 256];
+  unsigned long long my_key[kMaxCand / 256];
+#pragma unroll
+  for (int t = 0; t < kMaxCand / 256; ++t) {
+    const int i = threadIdx.x + 256 * t;
+    my_id[t] = 0;
+    my_key[t] = 0ull;
+    if (i < n_cand) {
+      bool v = false;
+      my_id[t] = cand_block(p, s, i, v);
+      if (!v && p.err) atomicCAS(p.err, 0, VKV_DEVERR_BAD_INDEX);
+      if (v) {
+        const uint32_t u = __float_as_uint(sc[i]);
+        my_key[t] = ((unsigned long long)(u ^ ((u >> 31) ? 0xFFFFFFFFu : 0x80000000u)) << 32) |
+                    (unsigned long long)(0xFFFFFFFFu - (uint32_t)my_id[t]);
+        ++my_valid;
+      }
+      rk[i] = my_key[t];
+    }
+  }
+  if (my_valid) atomicAdd(&n_valid, my_valid);
+  __syncthreads();
+  // the kept ones' ids (the others INT_MAX) give the ascending output positions
+#pragma unroll
+  for (int t = 0; t < kMaxCand / 256; ++t) {
+    const int i = threadIdx.x + 256 * t;
+    if (i >= n_cand) break;
     int r = 0;
-    const float si = sc[i];
-    const int di = ids[i];
-    for (int j = 0; j < n_cand; ++j) r += (ok[j] && (sc[j] > si || (sc[j] == si && ids[j] < di))) ? 1 : 0;
-    keep[i] = (ok[i] && r < p.C) ? 1 : 0;
+#pragma unroll 8
+    for (int j = 0; j < n_cand; ++j) r += rk[j] > my_key[t] ? 1 : 0;
+    ids[i] = (my_key[t] != 0ull && r < p.C) ? my_id[t] : 0x7FFFFFFF;
   }
   __syncthreads();
   int* out = p.out_idx + (size_t)s * p.C;
-  for (int i = threadIdx.x; i < n_cand; i += blockDim.x) {
-    if (!keep[i]) continue;
+#pragma unroll
+  for (int t = 0; t < kMaxCand / 256; ++t) {
+    const int i = threadIdx.x + 256 * t;
+    if (i >= n_cand) break;
+    const int id = ids[i];
+    if (id == 0x7FFFFFFF) continue;
     int pos = 0;
-    for (int j = 0; j < n_cand; ++j) pos += (keep[j] && ids[j] < ids[i]) ? 1 : 0;
-    out[pos] = ids[i];
+#pragma unroll 8
+    for (int j = 0; j < n_cand; ++j) pos += ids[j] < id ? 1 : 0;
+    out[pos] = id;
   }
   // fewer than C valid candidates (only after an invalid persistent id): pad with -1
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int kept = 0;
-    for (int i = 0; i < n_cand; ++i) kept += keep[i];
-    for (int x = kept; x < p.C; ++x) out[x] = -1;
-  }
+  for (int x = min(p.C, n_valid) + (int)threadIdx.x; x < p.C; x += 256) out[x] = -1;
 }
 
 }  // namespace
