@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(256) order_kernel(const OrderParams p) {
   for (int j = threadIdx.x; j < p.n_qblk; j += blockDim.x) {
     const unsigned long long kj = sig[j];
     int rank = 0;
+#pragma unroll 8
     for (int i = 0; i < p.n_qblk; ++i) {
       const unsigned long long ki = sig[i];
       rank += (ki < kj || (ki == kj && i < j)) ? 1 : 0;
