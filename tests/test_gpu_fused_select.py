@@ -174,6 +174,24 @@ def test_fused_select_batch_of_two():
     assert_lse_close(l, rl, "fused-select LSE (B = 2)")
 
 
+def test_fused_select_largest_window():
+    """A window of 512 blocks, the largest the kernel's ranking keys hold (the
+    standalone kernel then scores from L2 in another summation order: the planted
+    margins keep the choice the same)."""
+    c = W.make_block_sparse("fused", seed=101, H=1, d=128, frame_tokens=256, block=64, hist_frames=3,
+                            win_frames=128, q_frames=2, n_persist=6)
+    assert c.n_win_blk == 512
+    q = c.q.to(DEV)
+    (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 16)
+    assert torch.equal(sel, idx)
+    ref_idx, ok = _gap_ok(c.q, c.k, c, 16)
+    assert ok.all() and np.array_equal(sel.cpu().numpy(), ref_idx)
+    assert torch.equal(o, o2) and torch.equal(l, l2)
+    ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, ref_idx, c.window_blk0, c.block, c.scale)
+    assert_bf16_close(o, ro, "fused-select O (512-block window)")
+    assert_lse_close(l, rl, "fused-select LSE (512-block window)")
+
+
 def test_fused_select_without_selection_output():
     c = _case(98, 2, 128, 2, 5)
     q = c.q.to(DEV)
