@@ -295,6 +295,24 @@ size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t
 vkv_status vkv_block_select(const vkv_select_args* args, vkv_stream_t stream);
 
 /*
+ * vkv_block_order -- the query-block order of vkv_block_select's out_order,
+ * from a selection the caller already holds (for instance the sel_out of a
+ * vkv_chunk_attn call that selected inside the attention kernel), to pass as
+ * a later call's qblk_order.  A work-grouping aid, not part of the pages'
+ * method.
+ *   sel_idx:   DEVICE int32 [BH][n_qblk][topk], each row's window block ids
+ *              ascending, each below 1024 (as the selection writes them);
+ *   out_order: DEVICE int32 [BH][n_qblk]: for each of the BH sequences a
+ *              permutation of its query blocks, ascending lexicographic order
+ *              of the first six selected ids, then by block index.
+ * Requires BH >= 1, 1 <= n_qblk <= 4096 and topk >= 1 (VKV_ERR_SHAPE /
+ * VKV_ERR_UNSUPPORTED otherwise).  Asynchronous on `stream`, after the work
+ * queued before it.
+ */
+vkv_status vkv_block_order(const int32_t* sel_idx, int32_t* out_order, int32_t BH, int32_t n_qblk,
+                           int32_t topk, vkv_stream_t stream);
+
+/*
  * vkv_block_pool -- the representative (fp32 mean of the rows) of each of the
  * 64-row blocks [blk0, blk0 + n_blk) of x [B, L, H, d] (Sparse Forcing summary,
  * section 2 component 2), written to out [B*H][n_blk][d] (DEVICE fp32, caller

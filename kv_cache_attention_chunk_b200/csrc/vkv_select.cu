@@ -338,6 +338,17 @@ bool launch_select(int d, dim3 g, bool after_pool, cudaStream_t st, const SelPar
 
 using namespace vkv;
 
+extern "C" vkv_status vkv_block_order(const int32_t* sel_idx, int32_t* out_order, int32_t BH, int32_t n_qblk,
+                                      int32_t topk, vkv_stream_t stream) {
+  if (!sel_idx || !out_order) return VKV_ERR_NULL;
+  if (BH <= 0 || n_qblk <= 0 || topk <= 0) return VKV_ERR_SHAPE;
+  if (n_qblk > kOrderMaxQblk || BH > 0x7FFFFFFF / n_qblk) return VKV_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (device_sm_count(&dev) <= 0) return VKV_ERR_CUDA;
+  return launch_order(sel_idx, out_order, BH, n_qblk, topk, reinterpret_cast<cudaStream_t>(stream)) ? VKV_OK
+                                                                                                    : VKV_ERR_CUDA;
+}
+
 extern "C" size_t vkv_block_select_workspace_size(int32_t B, int32_t H, int32_t Lq, int32_t n_win_blk,
                                                   int32_t block, int32_t d) {
   if (B <= 0 || H <= 0 || Lq <= 0 || n_win_blk <= 0 || block <= 0 || d <= 0) return 0;

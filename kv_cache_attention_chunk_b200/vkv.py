@@ -183,6 +183,8 @@ def _load(path: str) -> ctypes.CDLL:
     L.vkv_block_select_noalloc.restype = c_int32
     L.vkv_block_select_workspace_size.argtypes = [c_int32] * 6
     L.vkv_block_select_workspace_size.restype = c_size_t
+    L.vkv_block_order.argtypes = [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p]
+    L.vkv_block_order.restype = c_int32
     L.vkv_lse_merge.argtypes = [vkv_tensor, c_void_p, vkv_tensor, c_void_p, vkv_tensor, c_void_p,
                                 c_int32, c_int32, c_int32, c_int32, c_void_p]
     L.vkv_lse_merge.restype = c_int32
@@ -254,6 +256,23 @@ def vkv_block_select(args: vkv_select_args, stream: int | None) -> int:
 def vkv_block_select_noalloc(args: vkv_select_args, stream: int | None) -> int:
     """vkv_block_select with the library's own fixed scratch array (no workspace argument)."""
     return int(lib().vkv_block_select_noalloc(ctypes.byref(args), c_void_p(stream or 0)))
+
+
+def vkv_block_order(sel_idx, out_order, BH, n_qblk, topk, stream: int | None) -> int:
+    return int(lib().vkv_block_order(c_void_p(sel_idx), c_void_p(out_order), int(BH), int(n_qblk), int(topk),
+                                     c_void_p(stream or 0)))
+
+
+def block_order(sel_idx, out=None, stream=None):
+    """Query-block order [B*H, nQblk] grouping similar selections, from a selection
+    sel_idx (device int32 [B*H, nQblk, topk], e.g. the sel_out of chunk_attn_block_sparse
+    with kbar), for a later call's qblk_order."""
+    sel_idx = sel_idx.contiguous()
+    BH, n_qblk, topk = sel_idx.shape
+    order = out if out is not None else torch.empty((BH, n_qblk), dtype=torch.int32, device=sel_idx.device)
+    _check(vkv_block_order(sel_idx.data_ptr(), order.data_ptr(), BH, n_qblk, topk, _stream(stream)),
+           "vkv_block_order")
+    return order
 
 
 def vkv_block_pool(x: vkv_tensor, B, L, H, d, blk0, n_blk, out, stream: int | None) -> int:

@@ -215,6 +215,17 @@ def test_ragged_host_offsets_checked():
         assert call(ragged_args([0, 10, 20, 30])) == 6
 
 
+def test_block_order_validation():
+    assert vkv.vkv_block_order(0, FAKE, 12, 72, 9, None) == 1
+    assert vkv.vkv_block_order(FAKE, 0, 12, 72, 9, None) == 1
+    assert vkv.vkv_block_order(FAKE, FAKE, 0, 72, 9, None) == 2
+    assert vkv.vkv_block_order(FAKE, FAKE, 12, 0, 9, None) == 2
+    assert vkv.vkv_block_order(FAKE, FAKE, 12, 72, 0, None) == 2
+    assert vkv.vkv_block_order(FAKE, FAKE, 12, 4097, 9, None) == 5
+    if not torch.cuda.is_available():
+        assert vkv.vkv_block_order(FAKE, FAKE, 12, 72, 9, None) == 6
+
+
 def test_block_select_validation_and_workspace_size():
     ws = vkv.vkv_block_select_workspace_size(1, 12, 4608, 144, 64, 128)
     assert ws == 12 * 144 * 128 * 4  # the window block means (query blocks pool in shared memory)

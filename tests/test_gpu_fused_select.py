@@ -144,6 +144,23 @@ def test_fused_select_full_config3(frac):
     assert torch.equal(o, o2) and torch.equal(l, l2), f"K={K}"
 
 
+def test_order_from_a_fused_selection():
+    """vkv_block_order on the in-kernel selection equals the order vkv_block_select
+    writes with the same selection (a grouped order for the next call)."""
+    c = _iid()
+    K = W.topk_for_fraction(W.SPARSE_TOPK_FRACTIONS[1], c.n_win_blk)
+    q, k = c.q.to(DEV), c.k.to(DEV)
+    (o, l, sel), (_, _, idx) = _run_pair(c, q, K, None)
+    _, _, ref_order = vk().block_select(q, k, c.window_blk0, c.n_win_blk, K, order=True)
+    order = vk().block_order(sel)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, idx)
+    assert torch.equal(order, ref_order)
+    # and the grouped call with it reproduces the fused result of the grouped order
+    (o2, l2, sel2), _ = _run_pair(c, q, K, order)
+    assert torch.equal(sel2, sel)
+
+
 def test_fused_select_full_config3_sampled_natural_order():
     c = _iid()
     K = W.topk_for_fraction(W.SPARSE_TOPK_FRACTIONS[0], c.n_win_blk)
