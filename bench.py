@@ -261,6 +261,13 @@ def cpu_baseline(case, seconds: float = 15.0):
                       f"+ LSE merge, fp64 NumPy), {t:.1f} s"}
 
 
+def headline_config(world: int) -> dict:
+    """The workload of the headline line (the same for every arm of the same launch)."""
+    return {"workload": WORKLOAD, "parallelism": f"independent chunk per GPU x{world}",
+            "l2": "no flush: each step reads 961 MB of inputs, larger than the 126 MB L2",
+            "flops_per_chunk": headline_flops()}
+
+
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
@@ -280,9 +287,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_step": rows, "sample_head": 0},
+            "data": "synthetic", "config": headline_config(world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
-                             "sample": f"head 0, query rows 0..{rows - 1} per step"},
+                             "sample": f"head 0, query rows 0..{rows - 1} of the chunk per step (both branches "
+                                       f"+ LSE merge, fp64 NumPy)"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -616,10 +624,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "parallelism": f"independent chunk per GPU x{world}",
-                   "l2": "no flush: each step reads 961 MB of inputs, larger than the 126 MB L2",
-                   "ms_per_chunk": ms_step, "pct_of_bf16_peak": 100.0 * value / world / peak,
-                   "flops_per_chunk": fl},
+        "config": headline_config(world),
+        "chunk": {"ms": ms_step, "pct_of_bf16_peak": 100.0 * value / world / peak},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(),
                      "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": headline_kernel_name(vkv, q, k, v, case),
@@ -636,7 +642,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     line["roofline"]["launch_mcycles_median"] = mcycles(line["roofline"]["launch_ms_median"], clocks)
-    line["config"]["mcycles_per_chunk"] = mcycles(ms_step, clocks)
+    line["chunk"]["mcycles"] = mcycles(ms_step, clocks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if world == 1 and not args.no_extras:
@@ -752,8 +758,8 @@ def run_split(args):
                    + (" + all-gather of the merged output" if args.gather and args.split == "heads" else "")
                    + (" + send/recv of partials to rank 0 and LSE merges" if args.split == "keys" else ""),
                    "rank0_part": part, "l2": "no flush: the inputs are larger than L2",
-                   "ms_per_chunk": ms_step, "mcycles_per_chunk": mcycles(ms_step, clocks),
-                   "pct_of_bf16_peak": 100.0 * value / world / peak, "flops_per_chunk": fl},
+                   "flops_per_chunk": fl},
+        "chunk": {"ms": ms_step, "mcycles": mcycles(ms_step, clocks), "pct_of_bf16_peak": 100.0 * value / world / peak},
         "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": "TFLOP/s",
                      "frac": value / world / peak, "traffic": None,
                      "peak_source": f"{peak_src} bf16 dense (burst), per GPU"},
