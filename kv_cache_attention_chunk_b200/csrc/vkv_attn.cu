@@ -53,6 +53,32 @@ double single_tile_cost() {
   return c;
 }
 
+// One-tile units of the block-sparse kernel that selects for itself: their key
+// steps alternate between the two softmax warpgroups (VKV_KX=0 turns this off;
+// the other instantiations keep lone tiles on one warpgroup, whose code this
+// would slow down by a few per cent), so that a lone tile overlaps
+// two softmax passes as a pair does.  Such a unit costs kx_rate() of its steps
+// plus the fixed cost of a unit, above one half because each of its K/V tiles
+// feeds one query tile instead of two, so its loads run twice as fast per
+// product and its ring holds half as many steps (measured on B200: 0.65
+// balances K = 9 to 144 best; VKV_KX_RATE overrides it).
+bool kx_enabled() {
+  static bool on = [] {
+    const char* e = std::getenv("VKV_KX");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+double kx_rate() {
+  static double c = [] {
+    const char* e = std::getenv("VKV_KX_RATE");
+    double v = e ? std::atof(e) : 0.0;
+    return (v > 0.05 && v <= 1.0) ? v : 0.65;
+  }();
+  return c;
+}
+
 // Longest-processing-time assignment of `units` to `g` CTAs; returns makespan.
 double lpt(std::vector<Cand>& units, int g, Plan* out) {
   std::stable_sort(units.begin(), units.end(), [](const Cand& a, const Cand& b) { return a.cost > b.cost; });
@@ -125,10 +151,11 @@ constexpr double kSplitGain = VKV_SPLIT_GAIN;  // a split schedule is used below
 // head's query tiles (its odd last tile included) run at the same time and its
 // K/V is read from DRAM about once; only the last wave is cut into pieces.
 // Otherwise longest first (for unequal costs: ragged caches), the rest of a cut
-// unit going back into the queue by its cost.
+// unit going back into the queue by its cost.  whole_singles: one-tile units are
+// never cut (their steps alternate between the warpgroups, which a piece does not do).
 bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
                 const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
-                bool head_major, Plan* out, double* mk_out) {
+                bool head_major, bool whole_singles, Plan* out, double* mk_out) {
   struct Item {
     double cost;
     uint32_t code;
@@ -137,6 +164,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
     double rate;
     int k;       // pieces already cut from this unit
     int unit;    // index of the unit (for its piece list)
+    bool cut;    // may be cut into pieces
   };
   auto cmp = [](const Item& a, const Item& b) {
     if (a.cost != b.cost) return a.cost < b.cost;  // max-heap on cost
@@ -145,9 +173,10 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
   std::vector<Item> base;
   for (int s = 0; s < n_seq; ++s) {
     for (int i = 0; i < T / 2; ++i)
-      base.push_back({pair_cost[s], unit_code(s, 2 * i, true), steps[s], 0, steps[s], 1.0, 0, 0});
+      base.push_back({pair_cost[s], unit_code(s, 2 * i, true), steps[s], 0, steps[s], 1.0, 0, 0, true});
     if (T & 1)
-      base.push_back({one_cost[s], unit_code(s, T - 1, false), steps1[s], 0, steps1[s], 0.0, 0, 0});
+      base.push_back(
+          {one_cost[s], unit_code(s, T - 1, false), steps1[s], 0, steps1[s], 0.0, 0, 0, !whole_singles});
   }
   if (base.empty() || (long long)base.size() > kMaxUnits) return false;
   double tot = 0, lb_piece = 0;
@@ -156,7 +185,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
     base[i].rate = base[i].cost / (base[i].S + kUnitOverhead);
     tot += base[i].cost;
     // no CTA can finish before a unit cut into the most pieces allowed
-    const int most = std::max(1, std::min(kMaxPiecesPerUnit, base[i].S / min_steps));
+    const int most = base[i].cut ? std::max(1, std::min(kMaxPiecesPerUnit, base[i].S / min_steps)) : 1;
     lb_piece = std::max(lb_piece, base[i].rate * ((double)base[i].S / most + kPieceOverhead));
   }
   const int g = n_sm;
@@ -190,7 +219,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
       heap.pop();
       const bool whole_unit = it.k == 0;
       int n = it.j1 - it.j0;
-      if (e.first + it.cost > cap && it.k < kMaxPiecesPerUnit - 1 && it.S <= 0xFFFF) {
+      if (e.first + it.cost > cap && it.cut && it.k < kMaxPiecesPerUnit - 1 && it.S <= 0xFFFF) {
         int fit = (int)((cap - e.first) / it.rate - kPieceOverhead);
         // leave at least a minimum piece for the rest rather than overfilling this CTA
         if (fit >= min_steps && n - fit < min_steps) fit = n - min_steps;
@@ -286,7 +315,7 @@ bool split_plan(int n_seq, int T, const std::vector<double>& pair_cost, const st
 // into pieces of at least min_steps, when that shortens it by 12 % or more.
 bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std::vector<double>& one_cost,
                const std::vector<int>& steps, const std::vector<int>& steps1, int min_steps, int n_sm,
-               bool head_major, Plan* plan) {
+               bool head_major, bool whole_singles, Plan* plan) {
   // sequences by decreasing pair cost: their pairs are split first
   std::vector<int> order(n_seq);
   for (int s = 0; s < n_seq; ++s) order[s] = s;
@@ -340,7 +369,8 @@ bool make_plan(int n_seq, int T, const std::vector<double>& pair_cost, const std
     // always uses n_sm CTAs); pieces add a workspace fill, partial stores and the
     // combine launch, so a split must model a few per cent of gain (measured on
     // B200: the Wan-14B shape, modelled 11 % shorter, ran 5-8 % faster split)
-    if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, head_major, &sp, &mk_split) &&
+    if (split_plan(n_seq, T, pair_cost, one_cost, steps, steps1, min_steps, n_sm, head_major, whole_singles, &sp,
+                   &mk_split) &&
         mk_split < kSplitGain * best) {
       *plan = std::move(sp);
       return true;
@@ -358,14 +388,16 @@ std::map<std::string, std::shared_ptr<Plan>> g_plans;
 
 std::shared_ptr<Plan> get_plan(const std::string& key, int n_seq, int T, const std::vector<double>& pc,
                                const std::vector<double>& oc, const std::vector<int>& steps,
-                               const std::vector<int>& steps1, int min_steps, int n_sm, bool head_major) {
+                               const std::vector<int>& steps1, int min_steps, int n_sm, bool head_major,
+                               bool whole_singles) {
   {
     std::lock_guard<std::mutex> lk(g_plan_mu);
     auto it = g_plans.find(key);
     if (it != g_plans.end()) return it->second;
   }
   auto plan = std::make_shared<Plan>();
-  if (!make_plan(n_seq, T, pc, oc, steps, steps1, min_steps, n_sm, head_major, plan.get())) return nullptr;
+  if (!make_plan(n_seq, T, pc, oc, steps, steps1, min_steps, n_sm, head_major, whole_singles, plan.get()))
+    return nullptr;
   std::lock_guard<std::mutex> lk(g_plan_mu);
   if (g_plans.size() > 256) g_plans.clear();
   g_plans[key] = plan;
@@ -617,9 +649,11 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
     const double u2 = std::min<double>(a->n_win_blk, (grouped ? 1.25 : 2.0) * a->topk);
     const double sp = (a->n_persist + u4) * 0.5 + 2.0;
     const double s1 = (a->n_persist + u2) * 0.5 + 2.0;
+    P->kx = (fs && kx_enabled()) ? 1 : 0;
+    const double s1_cost = P->kx ? kx_rate() * (a->n_persist + u2) * 0.5 + kUnitOverhead : c1 * s1;
     for (long long s = 0; s < n_seq; ++s) {
       pc[s] = sp;
-      oc[s] = c1 * s1;
+      oc[s] = s1_cost;
     }
     // pieces are cut in these estimated steps and scaled on the device to the
     // unit's real step count
@@ -630,7 +664,7 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
       steps1.assign(n_seq, P->sp_est[0]);
     }
     key = "B" + std::to_string(n_seq) + "/" + std::to_string(T) + "/" + std::to_string(a->n_persist) + "/" +
-          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n") + (fs ? "/fs" : "");
+          std::to_string(a->topk) + "/" + std::to_string(a->n_win_blk) + (grouped ? "/g" : "/n") + (fs ? "/fs" : "") + (P->kx ? "/kx" : "");
   } else {
     if (check_ptrs && !a->cu_seqlens) return VKV_ERR_NULL;
     if (Lkv <= 0) return VKV_ERR_SHAPE;
@@ -689,7 +723,8 @@ vkv_status attn_setup(const vkv_attn_args* a, bool check_ptrs, bool want_split, 
   if (steps1.empty()) steps1 = steps;
   // equal unit costs (every mode but ragged): units dealt out head by head
   const bool head_major = VKV_HEAD_MAJOR && mode != VKV_MODE_RAGGED;
-  std::shared_ptr<Plan> plan = get_plan(key, (int)n_seq, T, pc, oc, steps, steps1, min_steps, g_max, head_major);
+  std::shared_ptr<Plan> plan =
+      get_plan(key, (int)n_seq, T, pc, oc, steps, steps1, min_steps, g_max, head_major, P->kx != 0);
   if (!plan) return VKV_ERR_UNSUPPORTED;
   P->n_ctas = plan->n_ctas;
   std::copy(plan->cta_begin.begin(), plan->cta_begin.end(), P->cta_begin);

@@ -28,6 +28,9 @@
 // piece_combine_kernel, launched behind this grid, merges them.
 //   warps 4-7    softmax + epilogue for query tile 0 (one thread per row).
 //   warps 8-11   softmax + epilogue for query tile 1.
+// In the selecting (FS) kernel a one-tile unit gives its even key steps to
+// warps 4-7 (S_0, O_0) and its odd ones to warps 8-11 (S_1, O_1); the two
+// partial states are merged by their LSEs at the end of the unit.
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
 // The softmax threads read S_t, then write P_t (bf16, two per 32-bit column)
@@ -80,6 +83,7 @@ struct Ctl {
   int sel_go;         // FS: the selection warps may write the next list buffer
   uint32_t bitmap[4][32];
   uint32_t list[kMaxListEntries];  // block-list buffer 0 (buffer 1: the ring's last K/V slot)
+  uint64_t kx_sync;  // FS one-tile unit split over both warpgroups: states written, then read
 };
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
 
@@ -403,6 +407,17 @@ struct FsScratch {
   static constexpr int BYTES = OFF_KEYS + 4 * kFsMaxWin * 4;
   static_assert(kMaxListEntries * 4 <= OFF_QS, "second block list");
   static_assert(BYTES <= AttnCfg<D>::KV_BYTES, "selection scratch");
+};
+
+// A one-tile unit of the selecting (FS) kernel, whose key tiles alternate between
+// the two softmax warpgroups, ends with both warpgroups' row states (m, l) side by side,
+// float [warpgroup 2][m, l][row 128], at the end of the ring's last K/V slot:
+// past the second block list and the selection scratch, and used by one unit
+// at a time (a warpgroup leaves the unit only once both have read them).
+template <int D>
+struct KxScratch {
+  static constexpr int OFF = AttnCfg<D>::KV_BYTES - 2048;
+  static_assert(FsScratch<D>::BYTES <= OFF, "exchange area after the selection scratch");
 };
 
 // Named barrier of the two selection warps.
@@ -845,6 +860,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
   const uint32_t b_lfree0 = smem_u32(&ctl->list_free[0]);
   const uint32_t b_lpers0 = smem_u32(&ctl->list_pers[0]);
   const uint32_t b_drain = smem_u32(&ctl->drain);
+  const uint32_t b_kx = smem_u32(&ctl->kx_sync);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -866,6 +882,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       mbar_init(b_lpers0 + 8 * b, 1);
     }
     mbar_init(b_drain, 1);
+    if (FS) mbar_init(smem_u32(&ctl->kx_sync), 8);
     ctl->abort_flag = 0;
     ctl->list_count[0] = 0;
     ctl->list_count[1] = 0;
@@ -1038,15 +1055,16 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
         uint32_t item = 0, qcnt = 0, ucnt = 0;
-        uint32_t pv_cnt[2] = {0, 0};
+        uint32_t pv_cnt[2] = {0, 0};  // PV products issued on accumulator t
+        uint32_t pv_par = 0;          // FS: bit t = parity of pv_cnt[t] (t varies per step there)
         int piece_k = p.cta_piece0[blockIdx.x];
         bool ok = true;
         auto wait_item = [&](uint32_t it_) {
           return mbar_wait(b_full0 + 8 * (it_ % NS), (it_ / NS) & 1, abort_flag, p.err);
         };
-        auto issue_qk = [&](int t, uint32_t kslot) {
+        auto issue_qk = [&](int t, uint32_t kslot, int qt) {
           const uint32_t d_tm = tmem + (uint32_t)(t * 128);
-          const uint32_t qa = sQ + t * C::QT_BYTES;
+          const uint32_t qa = sQ + qt * C::QT_BYTES;
           const uint32_t kb = sKV + kslot * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -1057,6 +1075,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         };
         for (int ui = u_begin; ui < u_end && ok; ++ui, ++ucnt) {
           const UnitInfo u = decode_entry<PC>(p, p.units[ui]);
+          const bool kx = FS && p.kx && u.ntiles == 1;
           int rs = 0, rl = 0;
           const int lb = SP ? (int)(ucnt & 1u) : 0;
           const uint32_t uph = SP ? ((ucnt >> 1) & 1u) : (ucnt & 1u);  // this buffer's use parity
@@ -1071,10 +1090,11 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           bool fs_full = true;  // FS: the unit's step count is final
           if (FS) {
             // the persistent prefix alone fixes a lower bound; the count itself is
-            // needed one step before the prefix ends (whether another S follows)
+            // needed one step before the prefix ends (whether another S follows; two
+            // steps before it when the steps alternate between the accumulators)
             pi.j0 = 0;
             nsteps = ctl->pers_count[lb] >> 1;
-            if (nsteps <= 1) {
+            if (nsteps <= (kx ? 2 : 1)) {
               ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
               if (!ok) break;
               nsteps = unit_steps(p, ctl->list_count[lb], 0);
@@ -1093,16 +1113,28 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           ok = mbar_wait(b_qfull, qcnt & 1, abort_flag, p.err);
           ++qcnt;
           if (!ok) break;
-          // prologue: S_t(0) = Q_t K_0^T
+          // prologue: S_t(0) = Q_t K_0^T.  A one-tile unit whose key steps alternate
+          // between the accumulators (kx) computes S_(j&1) = Q K_j^T and
+          // O_(j&1) += P_(j&1) V_j instead, so the two softmax warpgroups overlap as
+          // on two tiles: its prologue is S_0 = Q K_0^T and S_1 = Q K_1^T, and each
+          // S_t is next computed two steps later.
+          const int kxi = kx ? 1 : 0;
           ok = wait_item(item);
           if (!ok) break;
           tc_fence_after();
-          for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % NS);
+          for (int t = 0; t < u.ntiles; ++t) issue_qk(t, item % NS, t);
           mma_commit(b_empty0 + 8 * (item % NS));
-          bool q_rel = nsteps == 1;  // FS: the Q tiles' release is committed
-          if (nsteps == 1) mma_commit(b_qempty);
+          if (kx && nsteps > 1) {
+            ok = wait_item(item + 2);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(1, (item + 2) % NS, 0);
+            mma_commit(b_empty0 + 8 * ((item + 2) % NS));
+          }
+          bool q_rel = kx ? nsteps <= 2 : nsteps == 1;  // the Q tiles' release is committed
+          if (q_rel) mma_commit(b_qempty);
           for (int j = 0; j < nsteps && ok; ++j) {
-            if (FS && !fs_full && j + 1 >= nsteps) {
+            if (FS && !fs_full && j + 1 + kxi >= nsteps) {
               ok = mbar_wait(b_lready0 + 8 * lb, uph, abort_flag, p.err);
               if (!ok) break;
               nsteps = unit_steps(p, ctl->list_count[lb], 0);
@@ -1110,17 +1142,18 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               mbar_arrive(b_lfree0 + 8 * lb);
             }
             // a piece may start inside a branch: its first step starts the accumulator too
-            const bool first = (sparse || ragged) ? (j == 0) : (it.next().first || (PC && j == 0));
+            const bool first = (sparse || ragged) ? (kx ? j <= 1 : j == 0) : (it.next().first || (PC && j == 0));
             const uint32_t vit = item + 2 * j + 1;
-            const uint32_t knext = item + 2 * j + 2;
-            const bool has_next = j + 1 < nsteps;
+            const uint32_t knext = item + 2 * j + 2 + 2 * kxi;
+            const bool has_next = j + 1 + kxi < nsteps;
             const int trm = (pv_cnt[0] < 256) ? 16384 + (int)(pv_cnt[0]) * 16 : -100;
             ok = wait_item(vit);
             if (!ok) break;
             VKV_STAMP(trm);
             bool k_ready = false;
-            for (int t = 0; t < u.ntiles && ok; ++t) {
-              ok = mbar_wait(b_pfull0 + 8 * t, pv_cnt[t] & 1, abort_flag, p.err);
+            const int t_end = kx ? (j & 1) + 1 : u.ntiles;
+            for (int t = kx ? (j & 1) : 0; t < t_end && ok; ++t) {
+              ok = mbar_wait(b_pfull0 + 8 * t, FS ? ((pv_par >> t) & 1u) : (pv_cnt[t] & 1u), abort_flag, p.err);
               if (!ok) break;
               VKV_STAMP(trm + 1 + 4 * t);
               tc_fence_after();
@@ -1135,7 +1168,10 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
               }
               mma_commit(b_odone0 + 8 * t);
               VKV_STAMP(trm + 2 + 4 * t);
-              ++pv_cnt[t];
+              if (FS)
+                pv_par ^= 1u << t;
+              else
+                ++pv_cnt[t];
               if (has_next) {
                 if (!k_ready) {
                   ok = wait_item(knext);
@@ -1144,7 +1180,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
                   k_ready = true;
                   VKV_STAMP(trm + 3 + 4 * t);
                 }
-                issue_qk(t, knext % NS);
+                issue_qk(t, knext % NS, kx ? 0 : t);
                 VKV_STAMP(trm + 4 + 4 * t);
               }
             }
@@ -1152,7 +1188,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             mma_commit(b_empty0 + 8 * (vit % NS));
             if (has_next) {
               mma_commit(b_empty0 + 8 * (knext % NS));
-              if (j + 2 == nsteps && fs_full) {
+              if (j + 2 + kxi == nsteps && fs_full) {
                 mma_commit(b_qempty);
                 q_rel = true;
               }
@@ -1278,14 +1314,18 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
       } else {
         nsteps = entry_steps(p, u, unit_steps(p, ctl->list_count[lb], rl), piece_k, pi0);
       }
-      const bool active = t < u.ntiles;
-      int qrow = (u.tile0 + t) * 128 + r;
+      // a one-tile unit whose key steps alternate between the warpgroups: both
+      // work on query tile 0, warpgroup t on the steps j with j % 2 == t
+      const bool kx = FS && p.kx && u.ntiles == 1;
+      const int tq = kx ? 0 : t;  // the query tile of this thread's row
+      const bool active = kx || t < u.ntiles;
+      int qrow = (u.tile0 + tq) * 128 + r;
       if (sparse) {
-        const int qbr = unit_qblk(p, u.s, 2 * (u.tile0 + t) + (r >> 6), false);
+        const int qbr = unit_qblk(p, u.s, 2 * (u.tile0 + tq) + (r >> 6), false);
         qrow = qbr >= 0 ? qbr * 64 + (r & 63) : p.Lq;
       }
       const bool row_ok = qrow < p.Lq;
-      const int qb = 2 * t + (r >> 6);
+      const int qb = 2 * tq + (r >> 6);
       float m = -INFINITY, l = 0.f;            // running state of the current branch
       float m_prev = -INFINITY, l_prev = 0.f;  // state of the branch closed before it
       int cur_branch = -1, prev_branch = -1;
@@ -1305,6 +1345,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             if (j >= nsteps) break;
           }
           const TileDesc td = it.next();
+          if (kx && (j & 1) != t) continue;  // the other warpgroup's step (its first is j = t)
           const int tr = (lane == 0 && sf_cnt < 128) ? t * 8192 + quarter * 2048 + (int)sf_cnt * 16 : -1;
           VKV_STAMP(tr);
           ok = warp_all(mbar_wait(b_sfull, sf_cnt & 1, abort_flag, p.err));
@@ -1321,7 +1362,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
           reg_fence<128>(sr);
           VKV_STAMP(tr < 0 ? -1 : tr + 2);
           bool pending_epi = false;
-          if (td.first || (PC && j == 0)) {
+          if (td.first || (PC && j == 0) || (kx && j == t)) {
             if (cur_branch >= 0) {
               pending_epi = true;
               prev_branch = cur_branch;
@@ -1483,8 +1524,62 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
             prefetch_l2(pr + c0);
           }
         }
-        if (ok) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
-        if (ok && !u.piece) {
+        // (with alternating steps, warpgroup 1 has none in a one-step unit)
+        if (ok && (!kx || nsteps > t)) ok = warp_all(mbar_wait(b_odone, (np - 1) & 1, abort_flag, p.err));
+        if (kx) {
+          // merge the two warpgroups' states (the LSE merge of two key subsets):
+          // each publishes its rows' (m, l); once both have, warpgroup t writes
+          // columns [t D/2, (t+1) D/2) of each row from both accumulators; neither
+          // leaves the unit (after which the MMA may overwrite its O) before both
+          // have read.  Both take both barrier phases on every path.
+          float* const kxs =
+              reinterpret_cast<float*>(smem + C::OFF_KV + (C::NSLOT - 1) * C::KV_BYTES + KxScratch<D>::OFF);
+          kxs[(2 * t) * 128 + r] = m;
+          kxs[(2 * t + 1) * 128 + r] = l;
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_kx);
+          const bool ok_a = warp_all(mbar_wait(b_kx, 0, abort_flag, p.err));
+          if (ok && ok_a) {
+            tc_fence_after();
+            const float m0 = kxs[r], l0 = kxs[128 + r], m1 = kxs[256 + r], l1 = kxs[384 + r];
+            const bool h0 = l0 > 0.f, h1 = l1 > 0.f;
+            const float mm = fmaxf(h0 ? m0 : -INFINITY, h1 ? m1 : -INFINITY);
+            const float a0 = h0 ? ex2_approx(m0 - mm) : 0.f;
+            const float a1 = h1 ? ex2_approx(m1 - mm) : 0.f;
+            const float den = a0 * l0 + a1 * l1;
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            const float w0 = a0 * inv, w1 = a1 * inv;
+            __nv_bfloat16* orow = p.o[0] + u.b * p.o_sb[0] + (long long)qrow * p.o_st[0] + u.h * p.o_sh[0];
+            const uint32_t tO0 = tmem + lane_base + C::TM_O;
+#pragma unroll
+            for (int cc = 0; cc < D / 2; cc += 32) {
+              const int c0 = t * (D / 2) + cc;
+              uint32_t v0[32], v1[32];
+              tmem_ld32(tO0 + (uint32_t)c0, v0);
+              tmem_ld32(tO0 + (uint32_t)(D + c0), v1);
+              tmem_ld_wait();
+              reg_fence<32>(v0);
+              reg_fence<32>(v1);
+              float f[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                // an accumulator without keys for this row (or never written in this
+                // unit) is left out, not multiplied by zero
+                const float x = h0 ? w0 * __uint_as_float(v0[e]) : 0.f;
+                f[e] = h1 ? fmaf(w1, __uint_as_float(v1[e]), x) : x;
+              }
+              if (row_ok) store_row32(orow + c0, f);
+            }
+            if (t == 0 && row_ok)
+              p.lse[0][(size_t)u.s * p.Lq + qrow] = den > 0.f ? (mm + lg2_approx(den)) * kLn2 : -INFINITY;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_kx);
+          const bool ok_b = warp_all(mbar_wait(b_kx, 1, abort_flag, p.err));
+          ok = ok && ok_a && ok_b;
+        } else if (ok && !u.piece) {
           tc_fence_after();
           // close the last branch, and merge with the one before it when asked
           const int lb = cur_branch;
@@ -1555,7 +1650,7 @@ __global__ void __launch_bounds__(384, 1) chunk_attn_kernel(const __grid_constan
         tc_fence_after();
         piece_close_branch<D>(p, piece_slot(p, piece_k - 1), t, cur_branch, r, row_ok, tO, m, l);
       }
-      if (ok && active && row_ok && !u.piece) {
+      if (ok && active && row_ok && !u.piece && (!kx || t == 0)) {
         // branches without any key tile: O = 0, LSE = -inf
         const int nb = (sparse || ragged) ? 1 : p.n_branches;
         for (int br = 0; br < nb; ++br) {

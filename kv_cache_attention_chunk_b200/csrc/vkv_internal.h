@@ -69,6 +69,10 @@ struct AttnParams {
   // [slot][tile 2][branch n_branches][row 128][d] and their LSEs (natural log)
   // [slot][tile][branch][row]
   int sp_est[2];  // BLOCK_SPARSE: key steps the schedule assumed for a 1- / 2-tile unit
+  // BLOCK_SPARSE with the selection in the kernel: a one-tile unit splits its key tiles
+  // between the two softmax warpgroups (even steps S_0/O_0, odd steps S_1/O_1) and
+  // merges the two by LSE
+  int kx;
   float* ws_o;
   float* ws_l;
   // schedule: CTA c runs units[cta_begin[c] .. cta_begin[c+1])

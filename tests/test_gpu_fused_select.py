@@ -5,8 +5,11 @@ query blocks, scores them and keeps the top-K itself.  Its selection must be
 the standalone selection's, index for index (both follow the same arithmetic),
 and therefore the oracle's wherever the fp64 scores leave no near-tie; its
 outputs must be those of the two-launch path (standalone selection, then the
-attention from the selected ids), bit for bit, and within the parity
-tolerances of the fp64 oracle.
+attention from the selected ids) within the bounds a key-axis split is held
+to, and within the parity tolerances of the fp64 oracle.  (A one-tile unit of
+the selecting kernel splits its key steps over two accumulators and merges
+them by LSE at the end, so its rows round differently from the two-launch
+path's; pairs of tiles follow the same arithmetic in both.)
 """
 import numpy as np
 import pytest
@@ -63,6 +66,13 @@ def _run_pair(c, q, K, order=None, sel_out=True):
     return (o, l, sel), (o2, l2, idx)
 
 
+def _same_as_two_launch(o, l, o2, l2):
+    """Outputs of the two paths within 2e-2, LSEs within 1e-4: the bounds the key-axis
+    split is held to against the whole unit, the same kind of LSE merge of two key
+    subsets (each subset's P is rounded to bf16 against its own running maximum)."""
+    return (o.float() - o2.float()).abs().max().item() <= 2e-2 and (l - l2).abs().max().item() <= 1e-4
+
+
 def _gap_ok(qn, kn, c, K):
     s = oracle.block_scores(qn, kn, c.window_blk0, c.n_win_blk, c.block)
     return oracle.select_topk(s, K), oracle.topk_gap(s, K) > 1e-4
@@ -97,7 +107,7 @@ def test_fused_select_small(seed, H, d, qf, npers, K, order, cut):
     ref_idx, ok = _gap_ok(qn, c.k, c, K)
     s = sel.cpu().numpy()
     assert np.array_equal(s[ok], ref_idx[ok])
-    assert torch.equal(o, o2) and torch.equal(l, l2), "outputs differ from the two-launch path"
+    assert _same_as_two_launch(o, l, o2, l2), "outputs differ from the two-launch path"
     ro, rl = oracle.block_sparse_attention(qn, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale)
     assert_bf16_close(o, ro, "fused-select O")
     assert_lse_close(l, rl, "fused-select LSE")
@@ -110,7 +120,7 @@ def test_fused_select_several_units_per_cta(d):
     q = c.q.to(DEV)
     (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 5)
     assert torch.equal(sel, idx)
-    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert _same_as_two_launch(o, l, o2, l2)
     heads, qblocks = [0, 47, 95], [0, 7, 15]
     s = sel.cpu().numpy()
     ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale,
@@ -141,7 +151,7 @@ def test_fused_select_full_config3(frac):
     assert torch.equal(sel, idx)
     ref = oracle.block_select(c.q, c.k, c.window_blk0, c.n_win_blk, c.block, K)[0]
     assert np.array_equal(sel.cpu().numpy(), ref), f"K={K}"
-    assert torch.equal(o, o2) and torch.equal(l, l2), f"K={K}"
+    assert _same_as_two_launch(o, l, o2, l2), f"K={K}"
 
 
 def test_order_from_a_fused_selection():
@@ -167,7 +177,7 @@ def test_fused_select_full_config3_sampled_natural_order():
     q = c.q.to(DEV)
     (o, l, sel), (o2, l2, idx) = _run_pair(c, q, K, None)
     assert torch.equal(sel, idx)
-    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert _same_as_two_launch(o, l, o2, l2)
     s = sel.cpu().numpy()
     heads, qblocks = [2, 7, 11], [0, 3, 35, 70, 71]
     ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, s, c.window_blk0, c.block, c.scale,
@@ -184,7 +194,7 @@ def test_fused_select_batch_of_two():
     assert torch.equal(sel, idx)
     ref_idx, ok = _gap_ok(c.q, c.k, c, 4)
     assert np.array_equal(sel.cpu().numpy()[ok], ref_idx[ok])
-    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert _same_as_two_launch(o, l, o2, l2)
     ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, sel.cpu().numpy(), c.window_blk0, c.block,
                                            c.scale)
     assert_bf16_close(o, ro, "fused-select O (B = 2)")
@@ -203,7 +213,7 @@ def test_fused_select_largest_window():
     assert torch.equal(sel, idx)
     ref_idx, ok = _gap_ok(c.q, c.k, c, 16)
     assert ok.all() and np.array_equal(sel.cpu().numpy(), ref_idx)
-    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert _same_as_two_launch(o, l, o2, l2)
     ro, rl = oracle.block_sparse_attention(c.q, c.k, c.v, c.persist_idx, ref_idx, c.window_blk0, c.block, c.scale)
     assert_bf16_close(o, ro, "fused-select O (512-block window)")
     assert_lse_close(l, rl, "fused-select LSE (512-block window)")
@@ -213,7 +223,7 @@ def test_fused_select_without_selection_output():
     c = _case(98, 2, 128, 2, 5)
     q = c.q.to(DEV)
     (o, l, _), (o2, l2, _) = _run_pair(c, q, 3, sel_out=False)
-    assert torch.equal(o, o2) and torch.equal(l, l2)
+    assert _same_as_two_launch(o, l, o2, l2)
 
 
 def test_fused_select_bad_order_sets_error_word():
@@ -231,4 +241,4 @@ def test_fused_select_bad_order_sets_error_word():
     assert int(err.item()) == vk().DEVERR_BAD_INDEX
     # the device stays usable
     (o, l, sel), (o2, l2, idx) = _run_pair(c, q, 3)
-    assert torch.equal(sel, idx) and torch.equal(o, o2)
+    assert torch.equal(sel, idx) and _same_as_two_launch(o, l, o2, l2)

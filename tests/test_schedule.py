@@ -25,6 +25,7 @@ from kv_cache_attention_chunk_b200 import build, vkv
 PIECE = 1 << 12
 TWO = 1 << 13
 C1 = 0.9  # single-tile cost relative to a pair over the same keys (the library's default)
+KX_RATE = 0.65  # the selecting kernel's one-tile unit: cost per key step relative to a pair (the library's default)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -62,7 +63,7 @@ def _ragged_args(Lq, lens, d=128):
     return a, [(n + 127) // 128 for n in lens]
 
 
-def _check_cover(sch, n_seq, T, steps, n_sm):
+def _check_cover(sch, n_seq, T, steps, n_sm, kx=False):
     cb, cp, units, pieces = sch["cta_begin"], sch["cta_piece0"], sch["units"], sch["pieces"]
     assert len(cb) <= n_sm + 1 and cb[0] == 0 and cb[-1] == len(units)
     assert np.all(np.diff(cb) >= 0)
@@ -91,7 +92,9 @@ def _check_cover(sch, n_seq, T, steps, n_sm):
             else:
                 assert (s, tiles) not in seen
                 seen[(s, tiles)] = "whole"
-                load[c] += rate * (S + 2.0)
+                # a whole one-tile unit of the selecting kernel splits its key steps
+                # over the two softmax warpgroups
+                load[c] += (KX_RATE * S + 2.0) if (kx and not two) else rate * (S + 2.0)
         assert k == cp[c + 1]
     # every query tile of every sequence exactly once
     covered = {}
@@ -235,6 +238,32 @@ def test_block_sparse_split_schedule_covers_and_balances(topk, grouped):
     ls = _check_cover(sp, 12, 36, steps, 148)
     ideal = 216 * (S2 + 2.0) / 148
     assert ls.max() <= 0.88 * lw.max() and ls.max() <= 1.15 * ideal
+
+
+@pytest.mark.parametrize("topk,grouped", [(9, True), (9, False), (36, True), (144, True)])
+def test_selecting_kernel_balances_with_alternating_one_tile_units(topk, grouped):
+    """With the selection in the kernel (window block means given) units stay
+    whole.  216 two-tile units on 148 SMs would leave some SMs with two and others
+    with one; a one-tile unit there splits its key steps over the two softmax
+    warpgroups and costs about 0.65 of its steps, so the schedule mixes pairs and
+    such units and the busiest SM carries well under two pairs."""
+    a = vkv.vkv_attn_args()
+    a.mode = vkv.MODE_BLOCK_SPARSE
+    a.B, a.H, a.Lq, a.Lkv, a.d = 1, 12, 4608, 36 * 1536, 128
+    a.scale, a.block, a.n_persist, a.topk = 0.088, 64, 32, topk
+    a.window_blk0, a.n_win_blk = 30 * 1536 // 64, 144
+    a.qblk_order = 1 if grouped else None  # only NULL or not matters to the schedule
+    a.kbar = 16                            # likewise: the kernel selects for itself
+    u4 = min(144, (1.5 if grouped else 4.0) * topk)
+    u2 = min(144, (1.25 if grouped else 2.0) * topk)
+    S2, S1 = int(np.ceil((32 + u4) / 2)), int(np.ceil((32 + u2) / 2))
+    steps = lambda s, two: S2 if two else S1  # noqa: E731
+    for split in (False, True):
+        sch = vkv.attn_schedule(a, 148, split)
+        assert len(sch["pieces"]) == 0
+        assert np.any((sch["units"] & TWO) == 0), "expected one-tile units"
+        load = _check_cover(sch, 12, 36, steps, 148, kx=True)
+        assert load.max() <= 0.85 * 2 * (S2 + 2.0)
 
 
 @pytest.mark.parametrize("topk", [9, 18, 36])
