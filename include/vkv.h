@@ -192,7 +192,11 @@ typedef struct {
    *          selection (ascending ids, as vkv_block_select's out_idx), e.g. to
    *          derive a query-block order for a later call.
    * Requires 1 <= topk <= n_win_blk <= 512 (else VKV_ERR_SHAPE).  Units are not
-   * split along the key axis in this form (workspace is ignored). */
+   * split along the key axis in this form (workspace is ignored); a unit of one
+   * 128-row query tile instead splits its key tiles between two accumulators
+   * that are merged by their LSEs, so its output rows may differ from those of
+   * the attention from sel_idx in the last bits (both are the same softmax
+   * attention over the same key set). */
   const float* kbar;
   int32_t* sel_out;
 } vkv_attn_args;
